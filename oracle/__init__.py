@@ -1,0 +1,160 @@
+"""Python access to the CPU oracle (test infrastructure only).
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg use this
+package.  It loads oracle/_build/liboracle.so (built from
+specdec_oracle.cpp by oracle/build.py) and wraps each entry point so that it
+takes numpy arrays.  Nothing here is imported by the CUDA verifier.
+"""
+from __future__ import annotations
+
+import ctypes
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+_override = None
+
+DTYPE_CODE = {"f32": 0, "bf16": 1}
+
+
+def _bind(path):
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    i32, i64, u32, u64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_double
+    L.oracle_philox4x32_10.argtypes = [P, P, P]
+    L.oracle_uniforms.argtypes = [u64, u64, u32, u32, P, P]
+    L.oracle_argmax_rows.argtypes = [P, i32, i64, i64, i32, P]
+    L.oracle_topk_rows.argtypes = [P, i32, i64, i64, i32, i32, P, P]
+    L.oracle_verify_greedy.argtypes = [P, i32, i64, P, i32, i32, i32, P, P, i32, P, P]
+    L.oracle_verify_tree.argtypes = [P, i32, i64, P, P, i32, i32, i32, i32, P, P, P]
+    L.oracle_verify_rejection.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f64, u64, u64,
+                                          P, P, P, P]
+    for f in ("oracle_philox4x32_10", "oracle_uniforms", "oracle_argmax_rows", "oracle_topk_rows",
+              "oracle_verify_greedy", "oracle_verify_tree", "oracle_verify_rejection"):
+        getattr(L, f).restype = None
+    return L
+
+
+def lib():
+    global _lib
+    if _override is not None:
+        return _override
+    if _lib is None:
+        _lib = _bind(_build.build())
+    return _lib
+
+
+class use_library:
+    """Context manager: route every wrapper below to another build of the
+    oracle source (used by the tests that check the pins catch mistakes)."""
+
+    def __init__(self, path):
+        self.L = _bind(path)
+
+    def __enter__(self):
+        global _override
+        self._prev = _override
+        _override = self.L
+        return self
+
+    def __exit__(self, *exc):
+        global _override
+        _override = self._prev
+        return False
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def _c(a, dt=None):
+    return np.ascontiguousarray(a if dt is None else np.asarray(a, dtype=dt))
+
+
+def _logit_array(logits, dtype):
+    if dtype == "bf16":
+        return _c(logits, np.uint16)
+    return _c(logits, np.float32)
+
+
+def philox4x32_10(ctr, key):
+    c = _c(ctr, np.uint32)
+    k = _c(key, np.uint32)
+    out = np.zeros(4, np.uint32)
+    lib().oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def uniforms(seed, offset, b, i):
+    ua = ctypes.c_double()
+    ur = ctypes.c_double()
+    lib().oracle_uniforms(seed, offset, b, i, ctypes.byref(ua), ctypes.byref(ur))
+    return ua.value, ur.value
+
+
+def argmax_rows(logits, dtype):
+    x = _logit_array(logits, dtype)
+    V = x.shape[-1]
+    R = x.size // V if V else 0
+    am = np.zeros(R, np.int32)
+    lib().oracle_argmax_rows(_ptr(x), DTYPE_CODE[dtype], V, R, V, _ptr(am))
+    return am.reshape(x.shape[:-1])
+
+
+def topk_rows(logits, dtype, topk):
+    x = _logit_array(logits, dtype)
+    V = x.shape[-1]
+    R = x.size // V
+    ids = np.zeros((R, topk), np.int32)
+    vals = np.zeros((R, topk), np.float32)
+    lib().oracle_topk_rows(_ptr(x), DTYPE_CODE[dtype], V, R, V, topk, _ptr(ids), _ptr(vals))
+    return ids.reshape(x.shape[:-1] + (topk,)), vals.reshape(x.shape[:-1] + (topk,))
+
+
+def verify_greedy(logits, dtype, drafts, topk=0):
+    """logits [B, k+1, V]; drafts [B, k] -> (accept_len, out_tokens[, topk_ids, topk_vals])."""
+    x = _logit_array(logits, dtype)
+    B, k1, V = x.shape
+    k = k1 - 1
+    d = _c(drafts, np.int32).reshape(B, k)
+    al = np.zeros(B, np.int32)
+    out = np.zeros((B, k1), np.int32)
+    ids = np.zeros((B, k1, max(topk, 1)), np.int32)
+    vals = np.zeros((B, k1, max(topk, 1)), np.float32)
+    lib().oracle_verify_greedy(_ptr(x), DTYPE_CODE[dtype], V, _ptr(d), B, k, V, _ptr(al), _ptr(out),
+                               topk, _ptr(ids), _ptr(vals))
+    if topk > 0:
+        return al, out, ids, vals
+    return al, out
+
+
+def verify_tree(logits, dtype, parents, node_tokens, max_depth):
+    """logits [B, N+1, V] -> (accept_len, accept_nodes, out_tokens)."""
+    x = _logit_array(logits, dtype)
+    B, n1, V = x.shape
+    par = _c(parents, np.int32).reshape(B, n1)
+    tok = _c(node_tokens, np.int32).reshape(B, n1)
+    al = np.zeros(B, np.int32)
+    nodes = np.zeros((B, max_depth), np.int32)
+    out = np.zeros((B, max_depth + 1), np.int32)
+    lib().oracle_verify_tree(_ptr(x), DTYPE_CODE[dtype], V, _ptr(par), _ptr(tok), B, n1 - 1, V, max_depth,
+                             _ptr(al), _ptr(nodes), _ptr(out))
+    return al, nodes, out
+
+
+def verify_rejection(target, dtype, q, drafts, temperature, seed, offset):
+    """target [B, k+1, V]; q [B, k, V] float32 -> (accept_len, out_tokens, p_draft, margin)."""
+    x = _logit_array(target, dtype)
+    B, k1, V = x.shape
+    k = k1 - 1
+    qq = _c(q, np.float32).reshape(B, k, V) if k > 0 else np.zeros((B, 0, V), np.float32)
+    d = _c(drafts, np.int32).reshape(B, k)
+    al = np.zeros(B, np.int32)
+    out = np.zeros((B, k1), np.int32)
+    pd = np.zeros((B, max(k, 1)), np.float64)
+    mg = np.zeros(B, np.float64)
+    lib().oracle_verify_rejection(_ptr(x), DTYPE_CODE[dtype], V, _ptr(qq), V, _ptr(d), B, k, V,
+                                  float(temperature), int(seed), int(offset),
+                                  _ptr(al), _ptr(out), _ptr(pd), _ptr(mg))
+    return al, out, pd[:, :k], mg

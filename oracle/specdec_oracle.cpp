@@ -1,0 +1,392 @@
+// specdec_oracle.cpp — plain CPU oracle for the speculative-decoding verifier.
+//
+// TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+// benchmark's CPU-baseline leg may load this library.  The product path (the
+// CUDA verifier) never calls it and shares no code with it: no headers, no
+// helpers, no tables, no pre- or post-processing.
+//
+// It is deliberately slow and obvious: one thread, plain loops, fp64 wherever
+// floating point is involved, each step written as the pages state it.
+//
+// Sources (web pages on speculative decoding):
+//   [ARCTIC]   "Arctic Inference / Arctic Training speculative decoding" (juejin
+//              rendering): "What is speculative decoding" (proposer / scorer /
+//              verifier), "A Simple Example" (Fig. 3), "Verifier optimisation"
+//              (greedy verification: only tokens agreeing with greedy decoding
+//              are accepted), "Whole-system optimisation" (TopK instead of
+//              sampling).
+//   [HANDBOOK] "Speculative decoding", LLM inference handbook: "How does
+//              speculative decoding work" (accept the longest agreeing prefix
+//              of h tokens, the target emits token h+1), "Key metrics" (tau),
+//              "Medusa" (candidates form a tree; the longest accepted candidate
+//              prefix is kept), "EAGLE" (EAGLE-2 dynamic draft tree).
+//   [VLLM]     "vLLM features 03: speculative decoding", section 1 "Principle":
+//              stop at the first wrong draft and put the target's own token
+//              there, so every step gains at least one token; at temperature
+//              > 0 rejection sampling keeps the target's distribution
+//              (Leviathan et al. 2023; Chen et al. 2023); greedy output must be
+//              identical.
+//   Philox4x32-10: Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+//              Easy as 1, 2, 3", SC'11, section on the Philox family.
+//
+// Readings taken where the pages are silent (all listed in the design notes):
+//   * argmax ties go to the lowest index; NaN ranks below -inf; -0 == +0;
+//   * row j of a request scores the token after the verified prefix plus
+//     drafts d_0..d_{j-1}; row k is the bonus row;
+//   * a draft token outside [0, V) never matches;
+//   * rejection rule: accept d_i iff u * q_i(d_i) < p_i(d_i) (strict), u from
+//     Philox; on the first rejection at position h resample from
+//     norm(max(0, p_h - q_h)), falling back to p_h when that mass is 0; after k
+//     acceptances sample the bonus from p_k;
+//   * Philox counter = (request, position, offset_lo, offset_hi), key = seed;
+//     u_acc = (x0 + 0.5) 2^-32, u_res = (x1 + 0.5) 2^-32;
+//   * a tree request is invalid (accept_len = -1, all outputs -1) when
+//     parents[0] != -1, a parent is not in [0, c), or a node is deeper than
+//     max_depth; a rejection request is invalid when one of its target rows
+//     holds a NaN or +inf, or only -inf.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Reading stored logits: dtype 0 = float32, dtype 1 = bfloat16 (the upper 16
+// bits of a float32, so widening is exact).
+// ---------------------------------------------------------------------------
+float logit_at(const void* base, int dtype, int64_t row_stride, int64_t row, int64_t x) {
+    if (dtype == 1) {
+        uint16_t h = static_cast<const uint16_t*>(base)[row * row_stride + x];
+        uint32_t w = static_cast<uint32_t>(h) << 16;
+        float f;
+        std::memcpy(&f, &w, sizeof f);
+        return f;
+    }
+    return static_cast<const float*>(base)[row * row_stride + x];
+}
+
+// Total order used for the greedy choice: NaN is below every number (-inf
+// included), all NaNs are equal, -0 equals +0, otherwise numeric order.
+// Returns -1, 0, +1.
+int logit_cmp(float a, float b) {
+    bool na = std::isnan(a), nb = std::isnan(b);
+    if (na && nb) return 0;
+    if (na) return -1;
+    if (nb) return 1;
+    if (a < b) return -1;
+    if (a > b) return 1;
+    return 0;
+}
+
+// Greedy choice of one row: the lowest index holding the largest value.
+int32_t row_argmax(const void* logits, int dtype, int64_t row_stride, int64_t row, int V) {
+    int32_t best = 0;
+    for (int x = 1; x < V; ++x) {
+        if (logit_cmp(logit_at(logits, dtype, row_stride, row, x),
+                      logit_at(logits, dtype, row_stride, row, best)) > 0)
+            best = x;
+    }
+    return best;
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11).  Counter of four 32-bit words, key of
+// two; each round multiplies words 0 and 2 by the two Philox multipliers,
+// XORs the high halves with the other two words and the round key, and
+// permutes; the key is bumped by the two Weyl constants between rounds.
+// ---------------------------------------------------------------------------
+constexpr uint32_t PHILOX_M4x32_0 = 0xD2511F53u;
+constexpr uint32_t PHILOX_M4x32_1 = 0xCD9E8D57u;
+constexpr uint32_t PHILOX_W32_0 = 0x9E3779B9u;  // golden ratio
+constexpr uint32_t PHILOX_W32_1 = 0xBB67AE85u;  // sqrt(3) - 1
+
+void philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4]) {
+    uint32_t c[4] = {ctr_in[0], ctr_in[1], ctr_in[2], ctr_in[3]};
+    uint32_t k[2] = {key_in[0], key_in[1]};
+    for (int round = 0; round < 10; ++round) {
+        uint64_t p0 = static_cast<uint64_t>(PHILOX_M4x32_0) * c[0];
+        uint64_t p1 = static_cast<uint64_t>(PHILOX_M4x32_1) * c[2];
+        uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+        uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
+        uint32_t n0 = hi1 ^ c[1] ^ k[0];
+        uint32_t n1 = lo1;
+        uint32_t n2 = hi0 ^ c[3] ^ k[1];
+        uint32_t n3 = lo0;
+        c[0] = n0; c[1] = n1; c[2] = n2; c[3] = n3;
+        k[0] += PHILOX_W32_0;
+        k[1] += PHILOX_W32_1;
+    }
+    out[0] = c[0]; out[1] = c[1]; out[2] = c[2]; out[3] = c[3];
+}
+
+// Uniforms for request b, position i: word 0 drives the accept test, word 1
+// the resample.  (x + 0.5) * 2^-32 is exact in fp64 and lies strictly inside
+// (0, 1).
+void uniforms(uint64_t seed, uint64_t offset, uint32_t b, uint32_t i, double* u_acc, double* u_res) {
+    uint32_t ctr[4] = {b, i, static_cast<uint32_t>(offset), static_cast<uint32_t>(offset >> 32)};
+    uint32_t key[2] = {static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32)};
+    uint32_t x[4];
+    philox4x32_10(ctr, key, x);
+    const double two_m32 = 1.0 / 4294967296.0;
+    *u_acc = (static_cast<double>(x[0]) + 0.5) * two_m32;
+    *u_res = (static_cast<double>(x[1]) + 0.5) * two_m32;
+}
+
+}  // namespace
+
+extern "C" {
+
+// Philox block function, exported for the pins.
+void oracle_philox4x32_10(const uint32_t* ctr, const uint32_t* key, uint32_t* out) {
+    philox4x32_10(ctr, key, out);
+}
+
+void oracle_uniforms(uint64_t seed, uint64_t offset, uint32_t b, uint32_t i, double* u_acc, double* u_res) {
+    uniforms(seed, offset, b, i, u_acc, u_res);
+}
+
+// Greedy choice of R rows.
+void oracle_argmax_rows(const void* logits, int dtype, int64_t row_stride, int64_t R, int V, int32_t* am) {
+    for (int64_t r = 0; r < R; ++r) am[r] = row_argmax(logits, dtype, row_stride, r, V);
+}
+
+// The topk entries of each row, ordered by value (descending; NaN lowest,
+// -0 == +0) then by index (ascending): the first topk of a full sort of the
+// row under that order.  Values are the stored logits widened exactly.
+void oracle_topk_rows(const void* logits, int dtype, int64_t row_stride, int64_t R, int V, int topk,
+                      int32_t* ids, float* vals) {
+    std::vector<int32_t> idx(V);
+    for (int64_t r = 0; r < R; ++r) {
+        for (int x = 0; x < V; ++x) idx[x] = x;
+        auto before = [&](int32_t a, int32_t b) {
+            int c = logit_cmp(logit_at(logits, dtype, row_stride, r, a), logit_at(logits, dtype, row_stride, r, b));
+            return c > 0 || (c == 0 && a < b);
+        };
+        int m = std::min(topk, V);
+        std::partial_sort(idx.begin(), idx.begin() + m, idx.end(), before);
+        for (int j = 0; j < topk; ++j) {
+            if (j < m) {
+                ids[r * topk + j] = idx[j];
+                vals[r * topk + j] = logit_at(logits, dtype, row_stride, r, idx[j]);
+            } else {
+                ids[r * topk + j] = -1;
+                vals[r * topk + j] = std::numeric_limits<float>::quiet_NaN();
+            }
+        }
+    }
+}
+
+// Greedy verification of B requests with k drafts each.
+//   logits     [B, k+1, V] rows at logits + r * row_stride elements
+//   drafts     [B, k]
+//   accept_len [B]       h = number of leading drafts equal to the target's
+//                        greedy choice at their position
+//   out_tokens [B, k+1]  d_0..d_{h-1}, then the target's choice at position h
+//                        (the correction or bonus token), then -1
+//   topk_ids / topk_vals [B, k+1, topk] when topk > 0
+// [HANDBOOK] "How does speculative decoding work", steps 2-4; [VLLM] section 1;
+// [ARCTIC] "Verifier optimisation" and "A Simple Example".
+void oracle_verify_greedy(const void* logits, int dtype, int64_t row_stride, const int32_t* drafts,
+                          int B, int k, int V, int32_t* accept_len, int32_t* out_tokens,
+                          int topk, int32_t* topk_ids, float* topk_vals) {
+    std::vector<int32_t> am(k + 1);
+    for (int b = 0; b < B; ++b) {
+        for (int j = 0; j <= k; ++j) am[j] = row_argmax(logits, dtype, row_stride, (int64_t)b * (k + 1) + j, V);
+        int h = 0;
+        while (h < k) {
+            int32_t d = drafts[(int64_t)b * k + h];
+            if (d < 0 || d >= V || d != am[h]) break;  // first disagreement stops the scan
+            ++h;
+        }
+        accept_len[b] = h;
+        int32_t* out = out_tokens + (int64_t)b * (k + 1);
+        for (int i = 0; i <= k; ++i) {
+            if (i < h) out[i] = drafts[(int64_t)b * k + i];
+            else if (i == h) out[i] = am[h];
+            else out[i] = -1;
+        }
+    }
+    if (topk > 0)
+        oracle_topk_rows(logits, dtype, row_stride, (int64_t)B * (k + 1), V, topk, topk_ids, topk_vals);
+}
+
+// Greedy verification of a draft tree per request.
+//   logits      [B, N+1, V]; row c scores the children of node c (row 0 = root,
+//               the last verified token)
+//   parents     [B, N+1]; parents[0] = -1, 0 <= parents[c] < c
+//   node_tokens [B, N+1]; entry 0 (the root's own token) is not verified
+//   accept_len  [B]; accept_nodes [B, max_depth]; out_tokens [B, max_depth+1]
+// A node is accepted when its parent is accepted and its token equals the
+// parent's greedy choice; the deepest accepted node (lowest index among equals)
+// ends the accepted path, and its own row supplies the bonus token.
+// [HANDBOOK] "Medusa" (longest accepted candidate prefix) and "EAGLE" (EAGLE-2
+// draft tree).
+void oracle_verify_tree(const void* logits, int dtype, int64_t row_stride, const int32_t* parents,
+                        const int32_t* node_tokens, int B, int N, int V, int max_depth,
+                        int32_t* accept_len, int32_t* accept_nodes, int32_t* out_tokens) {
+    const int n1 = N + 1;
+    std::vector<int32_t> depth(n1), am(n1);
+    std::vector<char> ok(n1);
+    for (int b = 0; b < B; ++b) {
+        const int32_t* par = parents + (int64_t)b * n1;
+        const int32_t* tok = node_tokens + (int64_t)b * n1;
+        int32_t* nodes_out = accept_nodes + (int64_t)b * max_depth;
+        int32_t* out = out_tokens + (int64_t)b * (max_depth + 1);
+
+        bool valid = (par[0] == -1);
+        depth[0] = 0;
+        for (int c = 1; c < n1 && valid; ++c) {
+            if (par[c] < 0 || par[c] >= c) { valid = false; break; }
+            depth[c] = depth[par[c]] + 1;
+            if (depth[c] > max_depth) valid = false;
+        }
+        if (!valid) {
+            accept_len[b] = -1;
+            for (int i = 0; i < max_depth; ++i) nodes_out[i] = -1;
+            for (int i = 0; i <= max_depth; ++i) out[i] = -1;
+            continue;
+        }
+        for (int c = 0; c < n1; ++c) am[c] = row_argmax(logits, dtype, row_stride, (int64_t)b * n1 + c, V);
+        ok[0] = 1;
+        for (int c = 1; c < n1; ++c) {
+            int32_t t = tok[c];
+            ok[c] = ok[par[c]] && t >= 0 && t < V && t == am[par[c]];
+        }
+        int best = 0;
+        for (int c = 1; c < n1; ++c)
+            if (ok[c] && depth[c] > depth[best]) best = c;
+        int d = depth[best];
+        accept_len[b] = d;
+        for (int i = 0; i < max_depth; ++i) nodes_out[i] = -1;
+        for (int i = 0; i <= max_depth; ++i) out[i] = -1;
+        int c = best;
+        for (int i = d - 1; i >= 0; --i) {  // walk back to the root
+            nodes_out[i] = c;
+            out[i] = tok[c];
+            c = par[c];
+        }
+        out[d] = am[best];
+    }
+}
+
+// Rejection-sampling verification (Leviathan et al.; Chen et al.), as the vLLM
+// page's section 1 and the Arctic page's "What is speculative decoding" name it.
+//   target     [B, k+1, V] target logits; p_i = softmax(l_i / T)
+//   q          [B, k, V] float32 proposer probabilities (taken as given)
+//   drafts     [B, k]
+//   accept_len [B], out_tokens [B, k+1]  as in greedy mode
+//   p_draft    [B, k] p_i(d_i) in fp64 (0 for an out-of-range draft)
+//   margin     [B]  the smallest distance of any decision of the request from
+//              its boundary: |u_acc - p/q| per accept test (p itself when
+//              q = 0), and for the sampled token the distance of u_res * S to
+//              the nearer edge of the chosen token's bin, over S, and S itself
+//              when the residual was used.
+// Steps per request:
+//   1. m_i = max_x l_i(x)/T, Z_i = sum_x exp(l_i(x)/T - m_i) (sequential fp64).
+//   2. For i = 0..k-1: accept iff 0 <= d_i < V and u_acc(b,i) * q_i(d_i) <
+//      p_i(d_i); stop at the first rejection h (h = k if none).
+//   3. r = max(0, p_h - q_h) if h < k (p_h if that has no mass), r = p_k if
+//      h = k; S = sum r; the token is the smallest x with cumsum r > u_res * S
+//      (the last x with r > 0 if rounding leaves none).
+void oracle_verify_rejection(const void* target, int dtype, int64_t row_stride,
+                             const float* q, int64_t q_row_stride, const int32_t* drafts,
+                             int B, int k, int V, double temperature, uint64_t seed, uint64_t offset,
+                             int32_t* accept_len, int32_t* out_tokens, double* p_draft, double* margin) {
+    const double T = temperature;
+    std::vector<double> m(k + 1), Z(k + 1), r(V);
+    for (int b = 0; b < B; ++b) {
+        int32_t* out = out_tokens + (int64_t)b * (k + 1);
+        const int32_t* d = drafts + (int64_t)b * k;
+        // 1. softmax statistics of every target row of the request
+        bool valid = true;
+        for (int i = 0; i <= k; ++i) {
+            int64_t row = (int64_t)b * (k + 1) + i;
+            bool any_above_neg_inf = false, bad = false;
+            double mi = -std::numeric_limits<double>::infinity();
+            for (int x = 0; x < V; ++x) {
+                float l = logit_at(target, dtype, row_stride, row, x);
+                if (std::isnan(l) || (std::isinf(l) && l > 0)) bad = true;
+                if (!(std::isinf(l) && l < 0)) any_above_neg_inf = true;
+                double s = static_cast<double>(l) / T;
+                if (s > mi) mi = s;
+            }
+            if (bad || !any_above_neg_inf) { valid = false; break; }
+            double zi = 0.0;
+            for (int x = 0; x < V; ++x) {
+                double s = static_cast<double>(logit_at(target, dtype, row_stride, row, x)) / T;
+                zi += std::exp(s - mi);
+            }
+            m[i] = mi;
+            Z[i] = zi;
+        }
+        if (!valid) {
+            accept_len[b] = -1;
+            for (int i = 0; i <= k; ++i) out[i] = -1;
+            for (int i = 0; i < k; ++i) p_draft[(int64_t)b * k + i] = std::numeric_limits<double>::quiet_NaN();
+            margin[b] = std::numeric_limits<double>::infinity();
+            continue;
+        }
+        auto p_of = [&](int i, int x) {
+            int64_t row = (int64_t)b * (k + 1) + i;
+            double s = static_cast<double>(logit_at(target, dtype, row_stride, row, x)) / T;
+            return std::exp(s - m[i]) / Z[i];
+        };
+        auto q_of = [&](int i, int x) {
+            return static_cast<double>(q[((int64_t)b * k + i) * q_row_stride + x]);
+        };
+        for (int i = 0; i < k; ++i)
+            p_draft[(int64_t)b * k + i] = (d[i] >= 0 && d[i] < V) ? p_of(i, d[i]) : 0.0;
+
+        // 2. accept test, position by position
+        double mg = std::numeric_limits<double>::infinity();
+        int h = 0;
+        for (; h < k; ++h) {
+            double ua, ur;
+            uniforms(seed, offset, (uint32_t)b, (uint32_t)h, &ua, &ur);
+            if (d[h] < 0 || d[h] >= V) break;
+            double p = p_draft[(int64_t)b * k + h];
+            double qd = q_of(h, d[h]);
+            mg = std::min(mg, qd > 0.0 ? std::fabs(ua - p / qd) : p);
+            if (!(ua * qd < p)) break;
+        }
+        // 3. the correction (h < k) or bonus (h = k) token
+        double ua, ur;
+        uniforms(seed, offset, (uint32_t)b, (uint32_t)h, &ua, &ur);
+        double S = 0.0;
+        if (h < k) {
+            for (int x = 0; x < V; ++x) { r[x] = std::max(0.0, p_of(h, x) - q_of(h, x)); S += r[x]; }
+            mg = std::min(mg, S);
+            if (!(S > 0.0)) {
+                S = 0.0;
+                for (int x = 0; x < V; ++x) { r[x] = p_of(h, x); S += r[x]; }
+            }
+        } else {
+            for (int x = 0; x < V; ++x) { r[x] = p_of(k, x); S += r[x]; }
+        }
+        double t = ur * S;
+        double c = 0.0, prev = 0.0;
+        int tokv = -1;
+        for (int x = 0; x < V; ++x) {
+            prev = c;
+            c += r[x];
+            if (c > t) { tokv = x; break; }
+        }
+        if (tokv < 0) {
+            for (int x = V - 1; x >= 0; --x)
+                if (r[x] > 0.0) { tokv = x; break; }
+            if (tokv < 0) tokv = V - 1;
+            mg = 0.0;
+        } else {
+            mg = std::min(mg, std::min(t - prev, c - t) / S);
+        }
+        accept_len[b] = h;
+        for (int i = 0; i <= k; ++i) out[i] = (i < h) ? d[i] : (i == h ? tokv : -1);
+        margin[b] = mg;
+    }
+}
+
+}  // extern "C"
