@@ -1,0 +1,500 @@
+#!/usr/bin/env python
+"""Throughput of the B200 speculative-decoding verifier.
+
+One step = one verify call over one batch of B requests (B*(k+1) logit rows
+of V entries), inputs already resident in HBM.  Default workload: greedy
+verification at the Llama-3 vocabulary, B=64, k=5, V=128256, bf16.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+Prints one JSON line.  Multi-GPU: launched with torch.distributed.run, one
+rank per GPU; every rank verifies its own batch (requests are independent;
+no collective on the data path) and the time is the max over ranks.
+
+The timed steps replay a CUDA graph of the C-ABI calls over a rotation of
+input sets whose total exceeds 4x the L2 cache, so every step streams its
+logits from HBM.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gen  # noqa: E402
+
+METRIC = "verified rows/s and achieved HBM GB/s (% of B200 peak) for B×(k+1)×V verify"
+KERNEL_SOURCES = ["speculative_decoding_draft_decode_b200/csrc/verify_kernels.cuh",
+                  "speculative_decoding_draft_decode_b200/csrc/device_utils.cuh",
+                  "speculative_decoding_draft_decode_b200/csrc/specdec_api.cu",
+                  "speculative_decoding_draft_decode_b200/csrc/geometry.h",
+                  "speculative_decoding_draft_decode_b200/csrc/philox.cuh"]
+FALLBACK_HBM_GBS = 6650.0
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("kernel_hash") == kernel_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# Workloads
+# ---------------------------------------------------------------------------
+def make_workload(name, seed_offset=0):
+    base = {"greedy_llama3": (gen.greedy_llama3, 1), "greedy_tiny": (gen.greedy_tiny, 0),
+            "greedy_large_batch": (gen.greedy_large_batch, 3), "tree_medusa": (gen.tree_medusa, 4),
+            "rejection_qwen": (gen.rejection_qwen, 2)}
+    fn, seed = base[name]
+    return fn(seed=seed + 1000 * seed_offset)
+
+
+def describe(inp):
+    if isinstance(inp, gen.TreeInputs):
+        return {"B": inp.B, "N": inp.N, "V": inp.V, "rows": inp.B * (inp.N + 1), "max_depth": inp.max_depth}
+    d = {"B": inp.B, "k": inp.k, "V": inp.V, "rows": inp.B * (inp.k + 1)}
+    if isinstance(inp, gen.GreedyInputs) and inp.topk:
+        d["topk"] = inp.topk
+    if isinstance(inp, gen.RejectionInputs):
+        d["temperature"] = inp.temperature
+    return d
+
+
+def rows_of(inp):
+    return inp.B * ((inp.N + 1) if isinstance(inp, gen.TreeInputs) else (inp.k + 1))
+
+
+# ---------------------------------------------------------------------------
+# Device side
+# ---------------------------------------------------------------------------
+def host_tensors(inp):
+    """The workload's arrays as CPU torch tensors (bf16 logits keep their bits)."""
+    import torch
+
+    def logits_t(a, dt):
+        if dt == gen.BF16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+
+    def i32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32))
+
+    if isinstance(inp, gen.TreeInputs):
+        return {"logits": logits_t(inp.logits, inp.dtype), "parents": i32(inp.parents),
+                "node_tokens": i32(inp.node_tokens)}
+    if isinstance(inp, gen.RejectionInputs):
+        return {"target": logits_t(inp.target, inp.dtype),
+                "q": torch.from_numpy(np.ascontiguousarray(inp.q, dtype=np.float32)), "drafts": i32(inp.drafts)}
+    return {"logits": logits_t(inp.logits, inp.dtype), "drafts": i32(inp.drafts)}
+
+
+def host_pinned(inp):
+    return {k: v.pin_memory() for k, v in host_tensors(inp).items()}
+
+
+class DeviceSets:
+    """`n` input sets on the device: set 0 from the generator, set i > 0 the
+    same batch rolled by i*97 positions along the vocabulary (draft and node
+    tokens rolled with it), so every set has the workload's structure but
+    its own memory."""
+
+    def __init__(self, inp, n, device):
+        import torch
+        self.inp = inp
+        self.sets = []
+        base = {k: v.to(device) for k, v in host_tensors(inp).items()}
+        V = inp.V
+        for i in range(n):
+            s = (i * 97) % V
+            if s == 0:
+                self.sets.append(base)
+                continue
+            d = {}
+            for key, t in base.items():
+                if key in ("logits", "target", "q"):
+                    d[key] = torch.roll(t, shifts=s, dims=-1).contiguous()
+                elif key in ("drafts", "node_tokens"):
+                    d[key] = torch.where(t >= 0, (t + s) % V, t)
+                else:
+                    d[key] = t
+            self.sets.append(d)
+
+
+def setup_calls(inp, sets, ver, device):
+    """Static outputs and a list of per-set call closures (each one C-ABI
+    call on the current stream)."""
+    import torch
+    import speculative_decoding_draft_decode_b200 as sd
+    B = inp.B
+    calls = []
+    if isinstance(inp, gen.TreeInputs):
+        al = torch.empty(B, dtype=torch.int32, device=device)
+        nodes = torch.empty(B, inp.max_depth, dtype=torch.int32, device=device)
+        ot = torch.empty(B, inp.max_depth + 1, dtype=torch.int32, device=device)
+        outs = (al, nodes, ot)
+        for s in sets:
+            calls.append(lambda s=s: ver.tree(s["logits"], s["parents"], s["node_tokens"], inp.max_depth, out=outs))
+        kernels = 1
+    elif isinstance(inp, gen.RejectionInputs):
+        al = torch.empty(B, dtype=torch.int32, device=device)
+        ot = torch.empty(B, inp.k + 1, dtype=torch.int32, device=device)
+        pd = torch.empty(B, max(inp.k, 1), dtype=torch.float32, device=device)
+        outs = (al, ot, pd)
+        for s in sets:
+            calls.append(lambda s=s: ver.rejection(s["target"], s["q"], s["drafts"], inp.temperature, inp.seed,
+                                                   inp.offset, out=outs))
+        kernels = 2
+    else:
+        k1 = inp.k + 1
+        al = torch.empty(B, dtype=torch.int32, device=device)
+        ot = torch.empty(B, k1, dtype=torch.int32, device=device)
+        ids = torch.empty(B, k1, max(inp.topk, 1), dtype=torch.int32, device=device)
+        vals = torch.empty(B, k1, max(inp.topk, 1), dtype=torch.float32, device=device)
+        outs = (al, ot, ids, vals)
+        for s in sets:
+            calls.append(lambda s=s: ver.greedy(s["logits"], s["drafts"], topk=inp.topk, out=outs))
+        kernels = 1
+    return calls, outs, kernels
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) while the GPU runs the workload."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % index)
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    mx = float(p[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import speculative_decoding_draft_decode_b200 as sd
+    from speculative_decoding_draft_decode_b200 import build as sd_build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if rank == 0 or world == 1:
+        sd_build.build()
+    if world > 1:
+        dist.barrier()
+
+    inp = make_workload(args.workload, seed_offset=rank)
+    set_bytes = gen.algorithmic_bytes(inp)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    n_sets = max(2, math.ceil(4 * l2 / set_bytes) + 1) if args.sets is None else args.sets
+    sets = DeviceSets(inp, n_sets, device).sets
+    ver = sd.Verifier(device)
+    calls, outs, kpl = setup_calls(inp, sets, ver, device)
+
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for c in calls:  # allocates the workspace, loads the kernels
+            c()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for c in calls:
+            c()
+    per_replay = len(calls)
+
+    def run_steps(n):
+        full, rest = divmod(n, per_replay)
+        for _ in range(full):
+            graph.replay()
+        with torch.cuda.stream(stream):
+            for i in range(rest):
+                calls[i]()
+
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup)
+    stream.synchronize()
+
+    # clocks: sample across a 1 s burst of the same steps and the timed region
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_probe = time.time()
+    with torch.cuda.stream(stream):
+        while time.time() - t_probe < args.clock_probe_seconds:
+            run_steps(per_replay * 50)
+            stream.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        run_steps(args.steps)
+        ev1.record(stream)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    clocks = sampler.stop()
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # end to end: inputs from pinned host memory, H2D + verify + D2H each step
+    e2e = run_e2e(inp, ver, device, stream, args.e2e_steps) if args.e2e_steps > 0 else None
+    if world > 1 and e2e is not None:
+        t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["ms_per_step"] = float(t.item())
+
+    rows = rows_of(inp)
+    ms_step = ms_max / args.steps
+    value = rows * world / (ms_step / 1e3)
+    peak, peak_kind = measured_peak()
+    achieved = set_bytes / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "rows/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": inp.dtype,
+        "data": "synthetic",
+        "config": dict(workload=args.workload, **describe(inp), requests_per_s=inp.B * world / (ms_step / 1e3),
+                       l2="rotating %d input sets, %.0f MB > 4x L2 (%d MB)" % (n_sets, n_sets * set_bytes / 1e6,
+                                                                             l2 // 2**20),
+                       launch="CUDA graph of %d C-ABI calls, replayed" % per_replay,
+                       parallelism="dp%d (requests per rank, no collective)" % world),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                     % peak_kind if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "algorithmic_bytes_per_launch": set_bytes, "traffic": recorded_traffic(args.workload),
+                     "duration_us": ms_step * 1e3, "kernels_per_step": kpl,
+                     "note": "duration = timed region / steps (launch gaps included)"},
+        "gpu_launches": args.steps * kpl,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = {"value": rows * world / (e2e["ms_per_step"] / 1e3), "unit": "rows/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": e2e["ms_per_step"]}
+    if rank == 0 and args.cpu_baseline_seconds > 0:
+        line["cpu_baseline"] = cpu_baseline(inp, args.cpu_baseline_seconds)
+    if world > 1:
+        dist.barrier()
+        del graph
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(inp, ver, device, stream, steps):
+    """Public API end to end: pinned host inputs -> device, verify, result -> host."""
+    import torch
+    h = host_pinned(inp)
+    d = {k: torch.empty_like(v, device=device) for k, v in h.items()}
+    calls, outs, _ = setup_calls(inp, [d], ver, device)
+    res_h = [torch.empty_like(o, device="cpu").pin_memory() for o in outs[:2]]
+    h2d = sum(v.numel() * v.element_size() for v in h.values())
+    d2h = sum(o.numel() * o.element_size() for o in res_h)
+
+    def step():
+        for key, v in h.items():
+            d[key].copy_(v, non_blocking=True)
+        calls[0]()
+        for o, r in zip(outs[:2], res_h):
+            r.copy_(o, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+    stream.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(steps):
+            step()
+        ev1.record(stream)
+    stream.synchronize()
+    return {"ms_per_step": ev0.elapsed_time(ev1) / steps, "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_call(inp, req):
+    """The oracle on requests [0, req) of the workload."""
+    import oracle
+    if isinstance(inp, gen.TreeInputs):
+        return oracle.verify_tree(inp.logits[:req], inp.dtype, inp.parents[:req], inp.node_tokens[:req],
+                                  inp.max_depth)
+    if isinstance(inp, gen.RejectionInputs):
+        return oracle.verify_rejection(inp.target[:req], inp.dtype, inp.q[:req], inp.drafts[:req],
+                                       inp.temperature, inp.seed, inp.offset)
+    return oracle.verify_greedy(inp.logits[:req], inp.dtype, inp.drafts[:req], topk=inp.topk)
+
+
+def time_oracle(inp, seconds):
+    rpr = rows_of(inp) // inp.B
+    t0 = time.perf_counter()
+    oracle_call(inp, 1)
+    one = max(time.perf_counter() - t0, 1e-6)
+    req = int(max(1, min(inp.B, seconds / 4 / one)))
+    rows, el = 0, 0.0
+    while el < seconds:
+        t0 = time.perf_counter()
+        oracle_call(inp, req)
+        el += time.perf_counter() - t0
+        rows += req * rpr
+    return rows / el, req, rows
+
+
+def cpu_baseline(inp, seconds):
+    v, req, rows = time_oracle(inp, seconds)
+    return {"value": v, "unit": "rows/s", "cores": 1, "kind": "oracle",
+            "sample": "first %d requests of the workload, repeated for %.0f s (%d rows), single-threaded "
+                      "fp64 C++ oracle" % (req, seconds, rows)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = make_workload(args.workload)
+    budget = 120.0
+    # each step verifies a bounded sample of requests so the run fits the budget
+    v1, req1, _ = time_oracle(inp, 2.0)
+    rpr = rows_of(inp) // inp.B
+    step_budget = budget / max(1, args.steps + args.warmup)
+    req = int(max(1, min(inp.B, step_budget * v1 / rpr)))
+    for _ in range(args.warmup):
+        oracle_call(inp, req)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_call(inp, req)
+    el = time.perf_counter() - t0
+    value = req * rpr * args.steps / el
+    sample = "first %d of %d requests per step, single-threaded fp64 C++ oracle" % (req, inp.B)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype,
+            "data": "synthetic", "config": dict(workload=args.workload, **describe(inp)),
+            "cpu_baseline": {"value": value, "unit": "rows/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="greedy_llama3",
+                    choices=["greedy_llama3", "greedy_tiny", "rejection_qwen", "greedy_large_batch", "tree_medusa"])
+    ap.add_argument("--sets", type=int, default=None, help="input sets in the rotation (default: > 4x L2)")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--clock-probe-seconds", type=float, default=1.0,
+                    help="untimed burst of the same steps while nvidia-smi samples clocks")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * specdec.h — C-ABI of the batched speculative-decoding verifier (sm_100a).
+ *
+ * The verifier is the third role of a speculative-decoding step: a proposer
+ * offers k draft tokens, the scorer (the target model) scores the verified
+ * prefix plus the drafts in one forward pass, and the verifier decides which
+ * drafts are kept (Arctic Inference page, "What is speculative decoding").
+ * It keeps the longest prefix of drafts the target agrees with, h tokens, and
+ * the target itself supplies token h+1 (LLM inference handbook, "How does
+ * speculative decoding work"), so every step gains at least one token (vLLM
+ * features 03 page, section 1).
+ *
+ * Three modes:
+ *   greedy     a draft is kept while it equals the target's greedy choice
+ *              (Arctic page, "Verifier optimisation"); optional per-position
+ *              top-k (Arctic page, "Whole-system optimisation": TopK in place
+ *              of sampling).
+ *   rejection  Leviathan/Chen rejection sampling at temperature T > 0 (vLLM
+ *              page, section 1): keep d_i with probability min(1, p/q), else
+ *              resample from norm(max(0, p - q)); after k acceptances sample
+ *              the bonus token from p_k.
+ *   tree       Medusa / EAGLE-2 draft trees given as parent arrays (handbook,
+ *              "Medusa" and "EAGLE"): keep the longest root-to-node path whose
+ *              every token equals its parent's greedy choice.
+ *
+ * Conventions for every entry point
+ *   - All array arguments are DEVICE pointers to caller-owned memory.  The
+ *     library never allocates, frees or synchronises; every call enqueues its
+ *     kernels on `stream` and returns.  Outputs are valid once the stream
+ *     reaches that point.
+ *   - Argument errors are reported synchronously, before anything is
+ *     launched; nothing is written in that case.  A failed launch returns
+ *     SPECDEC_ERR_CUDA.
+ *   - Problems in the DATA never trap and never read or write out of bounds:
+ *     a draft or node token outside [0, V) simply does not match; an invalid
+ *     tree or an undefined target distribution makes that request's
+ *     accept_len -1 with all its token outputs -1.
+ *   - Logit row r (r = b*(k+1) + j, or b*(N+1) + c for trees) starts at
+ *     logits + r * row_stride ELEMENTS; row_stride >= V.  When the base
+ *     pointer and row_stride * element_size are multiples of 16 bytes the
+ *     kernels stream 16-byte vectors; otherwise a scalar path is used (same
+ *     results, lower bandwidth).
+ *   - Row j of a request scores the token after the verified prefix and the
+ *     drafts d_0..d_{j-1}; row k is the bonus row.
+ *   - Greedy choice: the lowest index holding the largest value; NaN ranks
+ *     below -inf and -0 equals +0.  bf16 logits are widened exactly.
+ *   - The workspace is caller-owned device memory of at least
+ *     specdec_workspace_size() bytes, zeroed once by specdec_workspace_init().
+ *     Every call leaves its counters at zero again, so one workspace serves
+ *     any sequence of calls of any mode and shape that fits its size,
+ *     including CUDA-graph replays.  Calls that may overlap on the GPU (other
+ *     streams) must use different workspaces.
+ *
+ * Limits: 0 <= B <= SPECDEC_MAX_B; 0 <= k <= SPECDEC_MAX_K; 1 <= V <=
+ * SPECDEC_MAX_V; tree: 0 <= N < SPECDEC_MAX_TREE_NODES, 1 <= max_depth <=
+ * SPECDEC_MAX_DEPTH; topk <= SPECDEC_MAX_TOPK.
+ */
+#ifndef SPECDEC_H_
+#define SPECDEC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA runtime's cudaStream_t is `struct CUstream_st *`; pass it here
+ * (NULL = the legacy default stream). */
+struct CUstream_st;
+
+#define SPECDEC_ABI_VERSION 1
+
+#define SPECDEC_MAX_B 65536
+#define SPECDEC_MAX_K 32
+#define SPECDEC_MAX_V (1 << 24)
+#define SPECDEC_MAX_TREE_NODES 1024 /* N + 1, root included */
+#define SPECDEC_MAX_DEPTH 32
+#define SPECDEC_MAX_TOPK 8
+
+typedef enum {
+    SPECDEC_OK = 0,
+    SPECDEC_ERR_INVALID_ARG = 1, /* null pointer, size out of range, bad stride, T <= 0 */
+    SPECDEC_ERR_UNSUPPORTED = 2, /* dtype or mode not supported */
+    SPECDEC_ERR_WORKSPACE = 3,   /* workspace null, too small or misaligned */
+    SPECDEC_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    SPECDEC_ERR_TIMEOUT = 5      /* reserved: no kernel of this version waits on another */
+} specdec_status;
+
+typedef enum { SPECDEC_F32 = 0, SPECDEC_BF16 = 1 } specdec_dtype;
+
+typedef enum {
+    SPECDEC_MODE_GREEDY = 0,
+    SPECDEC_MODE_REJECTION = 1,
+    SPECDEC_MODE_TREE = 2
+} specdec_mode;
+
+/* Bytes of workspace a call of `mode` needs for B requests with k drafts
+ * (tree: N draft nodes) over a vocabulary of V.  The size does not depend on
+ * the dtype argument beyond validation, and a workspace sized for the largest
+ * shape serves every smaller one.  Returns 0 for arguments outside the
+ * limits. */
+size_t specdec_workspace_size(specdec_mode mode, int B, int k_or_N, int V, specdec_dtype dtype);
+
+/* Zero `bytes` of workspace on `stream` (asynchronous).  Needed once after
+ * allocation; the 256-byte alignment of cudaMalloc is required. */
+specdec_status specdec_workspace_init(void* ws, size_t bytes, struct CUstream_st* stream);
+
+/* Greedy verification (Arctic page, "Verifier optimisation"; handbook,
+ * "How does speculative decoding work"; vLLM page, section 1).
+ *   logits      [B, k+1, V] of `dtype`, row stride `row_stride` elements
+ *   draft_tokens[B, k] int32
+ *   accept_len  [B] int32 out: h = number of leading drafts equal to the
+ *               greedy choice of their row
+ *   out_tokens  [B, k+1] int32 out: d_0..d_{h-1}, then the greedy choice of
+ *               row h (correction or bonus token), then -1
+ *   topk        0..8; when > 0, topk_ids [B, k+1, topk] int32 and topk_vals
+ *               [B, k+1, topk] float32 receive each row's topk entries by
+ *               value (descending, NaN last) then index (ascending), values
+ *               being the stored logits widened exactly; rows shorter than
+ *               topk are padded with id -1 and a quiet NaN.  Both may be NULL
+ *               when topk == 0. */
+specdec_status specdec_verify_greedy(const void* logits, specdec_dtype dtype, int64_t row_stride,
+                                     const int32_t* draft_tokens, int B, int k, int V,
+                                     int32_t* accept_len, int32_t* out_tokens,
+                                     int topk, int32_t* topk_ids, float* topk_vals,
+                                     void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
+/* Rejection-sampling verification (vLLM page, section 1; Leviathan et al.,
+ * Chen et al.).
+ *   target_logits [B, k+1, V] of `dtype`, row stride `row_stride`;
+ *                 p_i = softmax(l_i / temperature)
+ *   draft_probs   [B, k, V] float32 q_i of the proposer, row stride
+ *                 `q_row_stride` elements (finite, non-negative); may be NULL
+ *                 when k == 0
+ *   draft_tokens  [B, k] int32, d_i drawn from q_i
+ *   temperature   finite, normal, > 0
+ *   seed, offset  Philox4x32-10 key and stream position: request b, position
+ *                 i uses counter (b, i, offset_lo, offset_hi) and key
+ *                 (seed_lo, seed_hi); word 0 gives the accept uniform, word 1
+ *                 the resample uniform, each (x + 0.5) * 2^-32
+ *   accept_len    [B] int32 out; out_tokens [B, k+1] int32 out, as greedy
+ *   p_draft_out   [B, k] float32 out, p_i(d_i) (0 for an out-of-range draft);
+ *                 may be NULL
+ * Draft i is kept iff 0 <= d_i < V and u * q_i(d_i) < p_i(d_i); at the first
+ * rejection h the token is drawn by inverse CDF from max(0, p_h - q_h) (from
+ * p_h if that has no mass); with no rejection from p_k.  A request whose
+ * target rows hold NaN or +inf, or a row of only -inf, gets accept_len -1.
+ * Two kernels are enqueued (a streaming pass over every target row, then a
+ * pass over the one row h of each request). */
+specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
+                                        const float* draft_probs, int64_t q_row_stride,
+                                        const int32_t* draft_tokens, int B, int k, int V,
+                                        float temperature, uint64_t seed, uint64_t offset,
+                                        int32_t* accept_len, int32_t* out_tokens, float* p_draft_out,
+                                        void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
+/* Tree verification (handbook, "Medusa": candidates form a tree and the
+ * longest accepted candidate prefix is kept; "EAGLE": EAGLE-2 draft trees).
+ *   logits       [B, N+1, V]; row c scores the children of node c; row 0 is
+ *                the root (the last verified token)
+ *   parents      [B, N+1] int32; parents[0] = -1, 0 <= parents[c] < c
+ *   node_tokens  [B, N+1] int32; entry 0 (the root's own token) is unused
+ *   max_depth    bound on node depth and width of the path outputs
+ *   accept_len   [B] int32 out: depth of the chosen node (the deepest node
+ *                whose every ancestor edge matches, lowest index among equals)
+ *   accept_nodes [B, max_depth] int32 out: node indices of the path, -1 padded
+ *   out_tokens   [B, max_depth+1] int32 out: tokens of the path, then the
+ *                chosen node's greedy choice (bonus), then -1
+ * A request with parents[0] != -1, a parent outside [0, c) or a node deeper
+ * than max_depth gets accept_len -1 and all outputs -1. */
+specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int64_t row_stride,
+                                   const int32_t* parents, const int32_t* node_tokens,
+                                   int B, int N, int V, int max_depth,
+                                   int32_t* accept_len, int32_t* accept_nodes, int32_t* out_tokens,
+                                   void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
+/* Static text for a status code. */
+const char* specdec_status_string(specdec_status status);
+
+/* SPECDEC_ABI_VERSION of the loaded library. */
+int specdec_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPECDEC_H_ */

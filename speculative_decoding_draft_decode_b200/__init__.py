@@ -1,0 +1,299 @@
+"""B200-native batched speculative-decoding verifier.
+
+The verifier decides, for every request of a batch, how many of the
+proposer's k draft tokens the target model keeps and which token the target
+adds after them (the correction or bonus token).  All of the work runs in the
+sm_100a CUDA kernels of ``libspecdec.so``; this module only marshals
+arguments to its C-ABI (``include/specdec.h``).  PyTorch provides device
+memory and streams.
+
+Two layers:
+
+* ``specdec_*`` functions with the C names and C argument order.  Pointer
+  arguments accept a ``torch.Tensor`` (its ``data_ptr()``), an ``int`` address
+  or ``None``; the stream argument accepts a ``torch.cuda.Stream``, an ``int``
+  handle or ``None`` (the current torch stream).  They return the status code.
+* ``Verifier``: owns a workspace and returns freshly allocated outputs for
+  torch tensors.
+
+There is no CPU fallback: if the CUDA library is missing, loading it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "SPECDEC_OK", "SPECDEC_F32", "SPECDEC_BF16", "SPECDEC_MODE_GREEDY", "SPECDEC_MODE_REJECTION",
+    "SPECDEC_MODE_TREE", "SpecdecError", "lib", "library_path", "header_path",
+    "specdec_workspace_size", "specdec_workspace_init", "specdec_verify_greedy",
+    "specdec_verify_rejection", "specdec_verify_tree", "specdec_status_string", "specdec_abi_version",
+    "Verifier",
+]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(HERE, "libspecdec.so")
+header_path = os.path.join(os.path.dirname(HERE), "include", "specdec.h")
+
+SPECDEC_OK = 0
+SPECDEC_ERR_INVALID_ARG = 1
+SPECDEC_ERR_UNSUPPORTED = 2
+SPECDEC_ERR_WORKSPACE = 3
+SPECDEC_ERR_CUDA = 4
+SPECDEC_ERR_TIMEOUT = 5
+
+SPECDEC_F32 = 0
+SPECDEC_BF16 = 1
+
+SPECDEC_MODE_GREEDY = 0
+SPECDEC_MODE_REJECTION = 1
+SPECDEC_MODE_TREE = 2
+
+MAX_B = 65536
+MAX_K = 32
+MAX_TOPK = 8
+MAX_DEPTH = 32
+MAX_TREE_NODES = 1024
+
+
+class SpecdecError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = specdec_status_string(status) if _lib is not None else str(status)
+        super().__init__("%s: %s (status %d)" % (what or "specdec", msg, status))
+
+
+_lib = None
+
+
+def lib():
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise RuntimeError("libspecdec.so is not built (python -m speculative_decoding_draft_decode_b200.build); "
+                               "there is no CPU fallback")
+        L = ctypes.CDLL(library_path)
+        P, i32, i64, u64, sz, f32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64,
+                                     ctypes.c_size_t, ctypes.c_float)
+        L.specdec_abi_version.argtypes = []
+        L.specdec_abi_version.restype = i32
+        L.specdec_status_string.argtypes = [i32]
+        L.specdec_status_string.restype = ctypes.c_char_p
+        L.specdec_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.specdec_workspace_size.restype = sz
+        L.specdec_workspace_init.argtypes = [P, sz, P]
+        L.specdec_workspace_init.restype = i32
+        L.specdec_verify_greedy.argtypes = [P, i32, i64, P, i32, i32, i32, P, P, i32, P, P, P, sz, P]
+        L.specdec_verify_greedy.restype = i32
+        L.specdec_verify_rejection.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f32, u64, u64,
+                                               P, P, P, P, sz, P]
+        L.specdec_verify_rejection.restype = i32
+        L.specdec_verify_tree.argtypes = [P, i32, i64, P, P, i32, i32, i32, i32, P, P, P, P, sz, P]
+        L.specdec_verify_tree.restype = i32
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------------------
+# Argument marshalling
+# ---------------------------------------------------------------------------
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ---------------------------------------------------------------------------
+# C-ABI mirrors
+# ---------------------------------------------------------------------------
+def specdec_abi_version() -> int:
+    return lib().specdec_abi_version()
+
+
+def specdec_status_string(status: int) -> str:
+    return lib().specdec_status_string(int(status)).decode()
+
+
+def specdec_workspace_size(mode: int, B: int, k_or_N: int, V: int, dtype: int) -> int:
+    return lib().specdec_workspace_size(mode, B, k_or_N, V, dtype)
+
+
+def specdec_workspace_init(ws, nbytes: int, stream=None) -> int:
+    return lib().specdec_workspace_init(_ptr(ws), nbytes, _stream(stream))
+
+
+def specdec_verify_greedy(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len, out_tokens,
+                          topk, topk_ids, topk_vals, ws, ws_bytes, stream=None) -> int:
+    return lib().specdec_verify_greedy(_ptr(logits), dtype, row_stride, _ptr(draft_tokens), B, k, V,
+                                       _ptr(accept_len), _ptr(out_tokens), topk, _ptr(topk_ids),
+                                       _ptr(topk_vals), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def specdec_verify_rejection(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens,
+                             B, k, V, temperature, seed, offset, accept_len, out_tokens, p_draft_out,
+                             ws, ws_bytes, stream=None) -> int:
+    return lib().specdec_verify_rejection(_ptr(target_logits), dtype, row_stride, _ptr(draft_probs),
+                                          q_row_stride, _ptr(draft_tokens), B, k, V, float(temperature),
+                                          int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
+                                          _ptr(accept_len), _ptr(out_tokens), _ptr(p_draft_out),
+                                          _ptr(ws), ws_bytes, _stream(stream))
+
+
+def specdec_verify_tree(logits, dtype, row_stride, parents, node_tokens, B, N, V, max_depth,
+                        accept_len, accept_nodes, out_tokens, ws, ws_bytes, stream=None) -> int:
+    return lib().specdec_verify_tree(_ptr(logits), dtype, row_stride, _ptr(parents), _ptr(node_tokens),
+                                     B, N, V, max_depth, _ptr(accept_len), _ptr(accept_nodes),
+                                     _ptr(out_tokens), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def _check(status, what):
+    if status != SPECDEC_OK:
+        raise SpecdecError(status, what)
+
+
+# ---------------------------------------------------------------------------
+# torch layer
+# ---------------------------------------------------------------------------
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return SPECDEC_BF16
+    if t.dtype == torch.float32:
+        return SPECDEC_F32
+    raise TypeError("logits must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _row_stride(t, name):
+    """Row stride (elements) of a [B, R, V] tensor whose rows are evenly
+    spaced with a contiguous last dimension."""
+    if t.dim() != 3 or t.stride(2) != 1:
+        raise ValueError("%s must be a 3-D tensor with a contiguous last dimension" % name)
+    B, R, V = t.shape
+    if R > 1:
+        rs = t.stride(1)
+        if B > 1 and t.stride(0) != R * rs:
+            raise ValueError("%s: rows are not evenly spaced" % name)
+    elif B > 1:
+        rs = t.stride(0)
+    else:
+        rs = V
+    if rs < V:
+        raise ValueError("%s: overlapping rows" % name)
+    return int(rs)
+
+
+class Verifier:
+    """Speculative-decoding verifier bound to one CUDA device.
+
+    Owns a workspace that grows on demand (a new allocation happens outside
+    any CUDA-graph capture only if a call needs more than the last one) and is
+    zeroed once.  Calls are asynchronous on the given stream (default: the
+    current torch stream).  Calls on different streams that may overlap need
+    different Verifier objects.
+    """
+
+    def __init__(self, device=None):
+        import torch
+        self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self._ws = None
+        self._ws_bytes = 0
+
+    def workspace(self, nbytes: int, stream=None):
+        import torch
+        if nbytes > self._ws_bytes:
+            nbytes = max(nbytes, 2 * self._ws_bytes)
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+            _check(specdec_workspace_init(ws, nbytes, stream), "workspace_init")
+            self._ws, self._ws_bytes = ws, nbytes
+        return self._ws, self._ws_bytes
+
+    def greedy(self, logits, draft_tokens, topk: int = 0, stream=None, out=None):
+        """logits [B, k+1, V] (bf16/f32), draft_tokens [B, k] int32 ->
+        (accept_len [B], out_tokens [B, k+1][, topk_ids, topk_vals])."""
+        import torch
+        B, k1, V = logits.shape
+        k = k1 - 1
+        dt = _dtype_code(logits)
+        stride = _row_stride(logits, "logits")
+        d = draft_tokens
+        if k > 0 and (d.dtype != torch.int32 or not d.is_contiguous() or tuple(d.shape) != (B, k)):
+            raise ValueError("draft_tokens must be a contiguous int32 [B, k] tensor")
+        dev = logits.device
+        if out is None:
+            al = torch.empty(B, dtype=torch.int32, device=dev)
+            ot = torch.empty(B, k1, dtype=torch.int32, device=dev)
+            ids = torch.empty(B, k1, max(topk, 1), dtype=torch.int32, device=dev) if topk else None
+            vals = torch.empty(B, k1, max(topk, 1), dtype=torch.float32, device=dev) if topk else None
+        else:
+            al, ot, ids, vals = (tuple(out) + (None, None))[:4]
+        need = specdec_workspace_size(SPECDEC_MODE_GREEDY, B, k, V, dt)
+        ws, wsb = self.workspace(need, stream)
+        _check(specdec_verify_greedy(logits, dt, stride, d if k > 0 else None, B, k, V, al, ot, topk, ids, vals,
+                                     ws, wsb, stream), "verify_greedy")
+        return (al, ot, ids, vals) if topk else (al, ot)
+
+    def tree(self, logits, parents, node_tokens, max_depth: int, stream=None, out=None):
+        """logits [B, N+1, V], parents/node_tokens [B, N+1] int32 ->
+        (accept_len [B], accept_nodes [B, max_depth], out_tokens [B, max_depth+1])."""
+        import torch
+        B, n1, V = logits.shape
+        dt = _dtype_code(logits)
+        stride = _row_stride(logits, "logits")
+        for name, t in (("parents", parents), ("node_tokens", node_tokens)):
+            if t.dtype != torch.int32 or not t.is_contiguous() or tuple(t.shape) != (B, n1):
+                raise ValueError("%s must be a contiguous int32 [B, N+1] tensor" % name)
+        dev = logits.device
+        if out is None:
+            al = torch.empty(B, dtype=torch.int32, device=dev)
+            nodes = torch.empty(B, max_depth, dtype=torch.int32, device=dev)
+            ot = torch.empty(B, max_depth + 1, dtype=torch.int32, device=dev)
+        else:
+            al, nodes, ot = out
+        need = specdec_workspace_size(SPECDEC_MODE_TREE, B, n1 - 1, V, dt)
+        ws, wsb = self.workspace(need, stream)
+        _check(specdec_verify_tree(logits, dt, stride, parents, node_tokens, B, n1 - 1, V, max_depth, al, nodes, ot,
+                                   ws, wsb, stream), "verify_tree")
+        return al, nodes, ot
+
+    def rejection(self, target_logits, draft_probs, draft_tokens, temperature: float, seed: int, offset: int = 0,
+                  stream=None, out=None, want_p_draft: bool = True):
+        """target_logits [B, k+1, V], draft_probs [B, k, V] f32, draft_tokens
+        [B, k] int32 -> (accept_len [B], out_tokens [B, k+1], p_draft [B, k])."""
+        import torch
+        B, k1, V = target_logits.shape
+        k = k1 - 1
+        dt = _dtype_code(target_logits)
+        stride = _row_stride(target_logits, "target_logits")
+        q_stride = V
+        if k > 0:
+            if draft_probs.dtype != torch.float32 or tuple(draft_probs.shape) != (B, k, V):
+                raise ValueError("draft_probs must be a float32 [B, k, V] tensor")
+            q_stride = _row_stride(draft_probs, "draft_probs")
+            if draft_tokens.dtype != torch.int32 or not draft_tokens.is_contiguous():
+                raise ValueError("draft_tokens must be a contiguous int32 [B, k] tensor")
+        dev = target_logits.device
+        if out is None:
+            al = torch.empty(B, dtype=torch.int32, device=dev)
+            ot = torch.empty(B, k1, dtype=torch.int32, device=dev)
+            pd = torch.empty(B, max(k, 1), dtype=torch.float32, device=dev) if want_p_draft else None
+        else:
+            al, ot, pd = out
+        need = specdec_workspace_size(SPECDEC_MODE_REJECTION, B, k, V, dt)
+        ws, wsb = self.workspace(need, stream)
+        _check(specdec_verify_rejection(target_logits, dt, stride, draft_probs if k > 0 else None, q_stride,
+                                        draft_tokens if k > 0 else None, B, k, V, temperature, seed, offset,
+                                        al, ot, pd, ws, wsb, stream), "verify_rejection")
+        return al, ot, (pd[:, :k] if pd is not None else None)

@@ -1,0 +1,345 @@
+// specdec_api.cu — the C-ABI (include/specdec.h): argument checks, workspace
+// layout, grid sizing and kernel launches.
+//
+// Workspace layout (byte offsets; the ticket words are at fixed places so a
+// workspace initialised once serves calls of any shape):
+//   [0, 256 KiB)            pass-1 tickets, one 32-bit word per request
+//   [256 KiB, 512 KiB)      pass-2 tickets (rejection resample)
+//   [512 KiB, ...)          pass-1 partials: row r, slot s at (r*maxs + s)
+//   then (rejection only)   per-request RejState, pass-2 partials
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "../../include/specdec.h"
+#include "geometry.h"
+#include "verify_kernels.cuh"
+
+namespace specdec {
+namespace {
+
+constexpr size_t kTicketBytes = static_cast<size_t>(SPECDEC_MAX_B) * sizeof(unsigned);
+constexpr size_t kPartialBase = 2 * kTicketBytes;
+constexpr int64_t kMinVecsPerCta = 128;   // smallest piece worth a CTA
+constexpr int64_t kGridCap = 4096;        // largest grid any pass uses
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+    int64_t nv = 0, T1 = 0, G1max = 0, maxs1 = 0;
+    int64_t T2 = 0, G2max = 0, maxs2 = 0;
+    size_t partials1 = 0, state = 0, partials2 = 0, total = 0;
+};
+
+// Layout of one call.  `vec` = elements per vector (1 on the scalar path),
+// `slot1` = bytes per pass-1 partial.
+Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t slot1, bool rejection) {
+    Layout L;
+    L.total = kPartialBase;
+    if (rows <= 0 || V <= 0) return L;  // nothing streamed: only the ticket area
+    L.nv = (V + vec - 1) / vec;
+    L.T1 = rows * L.nv;
+    L.G1max = grid_upper(L.T1, kMinVecsPerCta, kGridCap);
+    L.maxs1 = slots_bound(L.nv, L.T1, L.G1max);
+    L.partials1 = kPartialBase;
+    size_t end = L.partials1 + static_cast<size_t>(rows) * L.maxs1 * slot1;
+    if (rejection) {
+        L.state = align_up(end, 256);
+        end = L.state + static_cast<size_t>(B) * sizeof(RejState);
+        L.T2 = static_cast<int64_t>(B) * L.nv;
+        L.G2max = grid_upper(L.T2, kMinVecsPerCta, kGridCap);
+        L.maxs2 = slots_bound(L.nv, L.T2, L.G2max);
+        L.partials2 = align_up(end, 256);
+        end = L.partials2 + static_cast<size_t>(B) * L.maxs2 * sizeof(ResamplePartial);
+    }
+    (void)rows_per_req;
+    L.total = align_up(end, 256);
+    return L;
+}
+
+int elem_size(specdec_dtype dt) { return dt == SPECDEC_BF16 ? 2 : 4; }
+int vec_elems(specdec_dtype dt) { return dt == SPECDEC_BF16 ? 8 : 4; }
+
+// Cached per (device, kernel) resident-CTA counts.
+constexpr int kMaxDevices = 64;
+constexpr int kNumKernels = 32;
+std::atomic<int> g_sms[kMaxDevices];
+std::atomic<int> g_occ[kMaxDevices][kNumKernels];
+
+cudaError_t grid_cap(const void* fn, int kernel_id, int64_t* cap) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) dev = kMaxDevices - 1;
+    int sms = g_sms[dev].load(std::memory_order_relaxed);
+    if (sms == 0) {
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        g_sms[dev].store(sms, std::memory_order_relaxed);
+    }
+    int occ = g_occ[dev][kernel_id].load(std::memory_order_relaxed);
+    if (occ == 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NT, 0);
+        if (e != cudaSuccess) return e;
+        if (occ < 1) occ = 1;
+        g_occ[dev][kernel_id].store(occ, std::memory_order_relaxed);
+    }
+    *cap = static_cast<int64_t>(sms) * occ;
+    if (*cap > kGridCap) *cap = kGridCap;
+    return cudaSuccess;
+}
+
+bool vector_path_ok(const void* p, int64_t stride, int esize) {
+    return (reinterpret_cast<uintptr_t>(p) % 16 == 0) && ((stride * esize) % 16 == 0);
+}
+
+bool rows_fit(int64_t rows, int64_t row_stride, int V) {
+    // Every element offset must fit comfortably in 63 bits.
+    return row_stride >= V && row_stride <= (int64_t(1) << 40) && rows * row_stride < (int64_t(1) << 52);
+}
+
+template <class Tag, int VEC, int MODE>
+specdec_status launch_pass1(Pass1Params P, cudaStream_t stream) {
+    auto fn = verify_pass1_kernel<Tag, VEC, MODE>;
+    const int kid = MODE * 4 + (VEC == 1 ? 0 : 1) * 2 + (sizeof(typename Tag::storage) == 2 ? 1 : 0);
+    int64_t cap = 0;
+    if (grid_cap(reinterpret_cast<const void*>(fn), kid, &cap) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    const int64_t G = grid_upper(P.T, kMinVecsPerCta, cap);
+    fn<<<static_cast<unsigned>(G), NT, 0, stream>>>(P);
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+template <class Tag, int VEC>
+specdec_status launch_pass2(Pass2Params P, cudaStream_t stream) {
+    auto fn = verify_resample_kernel<Tag, VEC>;
+    const int kid = 16 + (VEC == 1 ? 0 : 1) * 2 + (sizeof(typename Tag::storage) == 2 ? 1 : 0);
+    int64_t cap = 0;
+    if (grid_cap(reinterpret_cast<const void*>(fn), kid, &cap) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    const int64_t G = grid_upper(P.T, kMinVecsPerCta, cap);
+    fn<<<static_cast<unsigned>(G), NT, 0, stream>>>(P);
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+template <int MODE>
+specdec_status dispatch_pass1(specdec_dtype dt, bool vec, Pass1Params P, cudaStream_t s) {
+    if (dt == SPECDEC_BF16)
+        return vec ? launch_pass1<BF16Tag, 8, MODE>(P, s) : launch_pass1<BF16Tag, 1, MODE>(P, s);
+    return vec ? launch_pass1<F32Tag, 4, MODE>(P, s) : launch_pass1<F32Tag, 1, MODE>(P, s);
+}
+
+specdec_status dispatch_pass2(specdec_dtype dt, bool vec, Pass2Params P, cudaStream_t s) {
+    if (dt == SPECDEC_BF16) return vec ? launch_pass2<BF16Tag, 8>(P, s) : launch_pass2<BF16Tag, 1>(P, s);
+    return vec ? launch_pass2<F32Tag, 4>(P, s) : launch_pass2<F32Tag, 1>(P, s);
+}
+
+bool dtype_ok(specdec_dtype dt) { return dt == SPECDEC_F32 || dt == SPECDEC_BF16; }
+
+size_t slot_bytes(specdec_mode mode) {
+    if (mode == SPECDEC_MODE_GREEDY) return 8 * sizeof(uint64_t);  // room for top-8
+    if (mode == SPECDEC_MODE_REJECTION) return sizeof(SoftmaxPartial);
+    return sizeof(uint64_t);
+}
+
+specdec_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+    if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % 16 != 0) return SPECDEC_ERR_WORKSPACE;
+    if (ws_bytes < need) return SPECDEC_ERR_WORKSPACE;
+    return SPECDEC_OK;
+}
+
+void fill_common(Pass1Params& P, const void* logits, int64_t row_stride, int V, const Layout& L, int vec,
+                 int64_t rows, int rows_per_req, int B, void* ws) {
+    memset(&P, 0, sizeof(P));
+    P.logits = logits;
+    P.row_stride = row_stride;
+    P.V = V;
+    P.nv = static_cast<int>(L.nv);
+    P.nv_full = V / vec;
+    P.R = rows;
+    P.T = L.T1;
+    P.rows_per_req = rows_per_req;
+    P.B = B;
+    P.maxs = static_cast<int>(L.maxs1);
+    P.tickets = static_cast<unsigned*>(ws);
+    P.partials = static_cast<char*>(ws) + L.partials1;
+}
+
+}  // namespace
+}  // namespace specdec
+
+using namespace specdec;
+
+extern "C" {
+
+int specdec_abi_version(void) { return SPECDEC_ABI_VERSION; }
+
+const char* specdec_status_string(specdec_status s) {
+    switch (s) {
+        case SPECDEC_OK: return "ok";
+        case SPECDEC_ERR_INVALID_ARG: return "invalid argument";
+        case SPECDEC_ERR_UNSUPPORTED: return "unsupported dtype or mode";
+        case SPECDEC_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case SPECDEC_ERR_CUDA: return "CUDA runtime error";
+        case SPECDEC_ERR_TIMEOUT: return "timed out waiting on the device";
+    }
+    return "unknown status";
+}
+
+size_t specdec_workspace_size(specdec_mode mode, int B, int k_or_N, int V, specdec_dtype dtype) {
+    if (!dtype_ok(dtype) || B < 0 || B > SPECDEC_MAX_B || V < 1 || V > SPECDEC_MAX_V) return 0;
+    int rpr;
+    if (mode == SPECDEC_MODE_TREE) {
+        if (k_or_N < 0 || k_or_N + 1 > SPECDEC_MAX_TREE_NODES) return 0;
+        rpr = k_or_N + 1;
+    } else if (mode == SPECDEC_MODE_GREEDY || mode == SPECDEC_MODE_REJECTION) {
+        if (k_or_N < 0 || k_or_N > SPECDEC_MAX_K) return 0;
+        rpr = k_or_N + 1;
+    } else {
+        return 0;
+    }
+    const int64_t rows = static_cast<int64_t>(B) * rpr;
+    const bool rej = mode == SPECDEC_MODE_REJECTION;
+    // The larger of the vector and the scalar path's layouts.
+    const Layout a = make_layout(rows, rpr, B, V, vec_elems(dtype), slot_bytes(mode), rej);
+    const Layout b = make_layout(rows, rpr, B, V, 1, slot_bytes(mode), rej);
+    return a.total > b.total ? a.total : b.total;
+}
+
+specdec_status specdec_workspace_init(void* ws, size_t bytes, struct CUstream_st* stream) {
+    if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % 16 != 0) return SPECDEC_ERR_WORKSPACE;
+    if (bytes == 0) return SPECDEC_OK;
+    return cudaMemsetAsync(ws, 0, bytes, stream) == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+specdec_status specdec_verify_greedy(const void* logits, specdec_dtype dtype, int64_t row_stride,
+                                     const int32_t* draft_tokens, int B, int k, int V,
+                                     int32_t* accept_len, int32_t* out_tokens,
+                                     int topk, int32_t* topk_ids, float* topk_vals,
+                                     void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V < 1 || V > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (topk < 0 || topk > SPECDEC_MAX_TOPK) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    const int64_t rows = static_cast<int64_t>(B) * (k + 1);
+    if (!rows_fit(rows, row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
+    if (logits == nullptr || accept_len == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (k > 0 && draft_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (topk > 0 && (topk_ids == nullptr || topk_vals == nullptr)) return SPECDEC_ERR_INVALID_ARG;
+    const bool vec = vector_path_ok(logits, row_stride, elem_size(dtype));
+    const int ve = vec ? vec_elems(dtype) : 1;
+    const Layout L = make_layout(rows, k + 1, B, V, ve, topk > 0 ? 64 : 8, false);
+    specdec_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != SPECDEC_OK) return st;
+    Pass1Params P;
+    fill_common(P, logits, row_stride, V, L, ve, rows, k + 1, B, ws);
+    P.drafts = draft_tokens;
+    P.k = k;
+    P.accept_len = accept_len;
+    P.out_tokens = out_tokens;
+    P.topk = topk;
+    P.topk_ids = topk_ids;
+    P.topk_vals = topk_vals;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (topk > 0) return dispatch_pass1<MODE_TOP8>(dtype, vec, P, s);
+    return dispatch_pass1<MODE_ARGMAX>(dtype, vec, P, s);
+}
+
+specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int64_t row_stride,
+                                   const int32_t* parents, const int32_t* node_tokens,
+                                   int B, int N, int V, int max_depth,
+                                   int32_t* accept_len, int32_t* accept_nodes, int32_t* out_tokens,
+                                   void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || N < 0 || N + 1 > SPECDEC_MAX_TREE_NODES || V < 1 || V > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (max_depth < 1 || max_depth > SPECDEC_MAX_DEPTH) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    const int64_t rows = static_cast<int64_t>(B) * (N + 1);
+    if (!rows_fit(rows, row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
+    if (logits == nullptr || parents == nullptr || node_tokens == nullptr || accept_len == nullptr ||
+        accept_nodes == nullptr || out_tokens == nullptr)
+        return SPECDEC_ERR_INVALID_ARG;
+    const bool vec = vector_path_ok(logits, row_stride, elem_size(dtype));
+    const int ve = vec ? vec_elems(dtype) : 1;
+    const Layout L = make_layout(rows, N + 1, B, V, ve, 8, false);
+    specdec_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != SPECDEC_OK) return st;
+    Pass1Params P;
+    fill_common(P, logits, row_stride, V, L, ve, rows, N + 1, B, ws);
+    P.parents = parents;
+    P.node_tokens = node_tokens;
+    P.max_depth = max_depth;
+    P.accept_len = accept_len;
+    P.accept_nodes = accept_nodes;
+    P.out_tokens = out_tokens;
+    return dispatch_pass1<MODE_TREE>(dtype, vec, P, reinterpret_cast<cudaStream_t>(stream));
+}
+
+specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
+                                        const float* draft_probs, int64_t q_row_stride,
+                                        const int32_t* draft_tokens, int B, int k, int V,
+                                        float temperature, uint64_t seed, uint64_t offset,
+                                        int32_t* accept_len, int32_t* out_tokens, float* p_draft_out,
+                                        void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V < 1 || V > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    const int64_t rows = static_cast<int64_t>(B) * (k + 1);
+    if (!rows_fit(rows, row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
+    if (target_logits == nullptr || accept_len == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (k > 0 && (draft_tokens == nullptr || draft_probs == nullptr)) return SPECDEC_ERR_INVALID_ARG;
+    if (k > 0 && !rows_fit(static_cast<int64_t>(B) * k, q_row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
+    const bool vec = vector_path_ok(target_logits, row_stride, elem_size(dtype)) &&
+                     (k == 0 || vector_path_ok(draft_probs, q_row_stride, 4));
+    const int ve = vec ? vec_elems(dtype) : 1;
+    const Layout L = make_layout(rows, k + 1, B, V, ve, sizeof(SoftmaxPartial), true);
+    specdec_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != SPECDEC_OK) return st;
+    const double invT_d = 1.0 / static_cast<double>(temperature);
+    RejState* state = reinterpret_cast<RejState*>(static_cast<char*>(ws) + L.state);
+    Pass1Params P;
+    fill_common(P, target_logits, row_stride, V, L, ve, rows, k + 1, B, ws);
+    P.drafts = draft_tokens;
+    P.k = k;
+    P.accept_len = accept_len;
+    P.out_tokens = out_tokens;
+    P.q = draft_probs;
+    P.q_stride = q_row_stride;
+    P.invT = static_cast<float>(invT_d);
+    P.invT_d = invT_d;
+    P.seed = seed;
+    P.offset = offset;
+    P.p_draft_out = p_draft_out;
+    P.state = state;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
+    if (st != SPECDEC_OK) return st;
+    Pass2Params Q;
+    memset(&Q, 0, sizeof(Q));
+    Q.logits = target_logits;
+    Q.row_stride = row_stride;
+    Q.q = draft_probs;
+    Q.q_stride = q_row_stride;
+    Q.V = V;
+    Q.nv = static_cast<int>(L.nv);
+    Q.nv_full = V / ve;
+    Q.T = L.T2;
+    Q.B = B;
+    Q.k = k;
+    Q.maxs = static_cast<int>(L.maxs2);
+    Q.invT = static_cast<float>(invT_d);
+    Q.seed = seed;
+    Q.offset = offset;
+    Q.state = state;
+    Q.tickets = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kTicketBytes);
+    Q.partials = reinterpret_cast<ResamplePartial*>(static_cast<char*>(ws) + L.partials2);
+    Q.out_tokens = out_tokens;
+    return dispatch_pass2(dtype, vec, Q, s);
+}
+
+}  // extern "C"

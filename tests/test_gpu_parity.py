@@ -1,0 +1,435 @@
+"""CUDA verifier vs the CPU oracle, element by element, on the same seeded
+inputs.  Greedy and tree outputs must be bit-exact; rejection sampling must
+use the same Philox uniforms, give p_i(d_i) within 1e-6 relative, and agree
+on accepted lengths and tokens except in requests where a decision lies
+within 1e-6 of its boundary (and then in fewer than 1e-4 of requests)."""
+import math
+
+import numpy as np
+import pytest
+
+import gen
+import oracle
+import speculative_decoding_draft_decode_b200 as sd
+from gpu_util import dev_f32, dev_i32, dev_logits, host, require_cuda
+
+pytestmark = pytest.mark.gpu
+
+P_DRAFT_RTOL = 1e-6     # softmax probability tolerance
+MARGIN = 1e-6           # decisions closer than this to their boundary are exempt
+EXEMPT_FRACTION = 1e-4  # ... and may differ in fewer than this share of requests
+
+
+@pytest.fixture(scope="module")
+def V_():
+    torch = require_cuda()
+    return sd.Verifier(torch.device("cuda", 0))
+
+
+# ---------------------------------------------------------------------------
+# greedy
+# ---------------------------------------------------------------------------
+def run_greedy(ver, inp, topk=0):
+    x = dev_logits(inp.logits, inp.dtype)
+    d = dev_i32(inp.drafts)
+    res = ver.greedy(x, d, topk=topk)
+    return [host(t) for t in res]
+
+
+def check_greedy(ver, inp, topk=0, sample_topk_rows=None):
+    got = run_greedy(ver, inp, topk)
+    if topk == 0:
+        al, out = oracle.verify_greedy(inp.logits, inp.dtype, inp.drafts)
+        assert np.array_equal(got[0], al)
+        assert np.array_equal(got[1], out)
+        return got
+    al, out = oracle.verify_greedy(inp.logits, inp.dtype, inp.drafts)
+    assert np.array_equal(got[0], al)
+    assert np.array_equal(got[1], out)
+    rows = inp.logits.reshape(-1, inp.V)
+    R = rows.shape[0]
+    sel = np.arange(R) if sample_topk_rows is None else np.unique(
+        np.random.default_rng(0).integers(0, R, sample_topk_rows))
+    ids, vals = oracle.topk_rows(rows[sel], inp.dtype, topk)
+    gids = got[2].reshape(R, topk)[sel]
+    gvals = got[3].reshape(R, topk)[sel]
+    assert np.array_equal(gids, ids)
+    assert np.array_equal(gvals.view(np.uint32), vals.view(np.uint32))
+    return got
+
+
+def test_greedy_tiny(V_):
+    check_greedy(V_, gen.greedy_tiny())
+
+
+def test_worked_example(V_):
+    inp = gen.worked_example()
+    al, out = check_greedy(V_, inp)
+    assert al[0] == 2 and list(out[0, :3]) == [13, 578, 21747]
+
+
+def test_all_accept(V_):
+    inp = gen.all_accept_example()
+    al, out = check_greedy(V_, inp)
+    assert al[0] == 4
+
+
+def test_greedy_llama3_full(V_):
+    check_greedy(V_, gen.greedy_llama3())
+
+
+def test_greedy_large_batch_top8_full(V_):
+    check_greedy(V_, gen.greedy_large_batch(), topk=8, sample_topk_rows=160)
+
+
+@pytest.mark.parametrize("V", [1, 2, 7, 8, 9, 15, 17, 1003, 4099, 128256 + 5])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_greedy_ragged_vocab(V_, V, dtype):
+    inp = gen.greedy_synthetic(seed=V, B=5, k=3, V=V, alpha=0.6, sigma=2.0, dtype=dtype)
+    check_greedy(V_, inp)
+    check_greedy(V_, inp, topk=8)
+
+
+@pytest.mark.parametrize("k", [0, 1, 31, 32])
+def test_greedy_k_extremes(V_, k):
+    inp = gen.greedy_synthetic(seed=100 + k, B=7, k=k, V=3000, alpha=0.9, dtype="bf16")
+    check_greedy(V_, inp)
+    check_greedy(V_, inp, topk=5)
+
+
+@pytest.mark.parametrize("B,V", [(1, 64), (3000, 16), (20000, 3), (257, 517)])
+def test_greedy_many_small_requests(V_, B, V):
+    inp = gen.greedy_synthetic(seed=B + V, B=B, k=4, V=V, alpha=0.7, dtype="f32")
+    check_greedy(V_, inp)
+    check_greedy(V_, inp, topk=3)
+
+
+def special_rows(rng, shape):
+    pool = np.array([0.0, -0.0, 1.0, -1.0, np.inf, -np.inf, np.nan, 3.0, 3.0, -2.0], np.float32)
+    return rng.choice(pool, size=shape).astype(np.float32)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_greedy_nan_inf_ties(V_, dtype):
+    rng = np.random.default_rng(5)
+    B, k, V = 40, 3, 777
+    x = special_rows(rng, (B, k + 1, V))
+    x[0] = np.nan
+    x[1] = -np.inf
+    x[2] = -0.0
+    x[2, :, 400] = 0.0
+    x[3, :, :] = np.nan
+    x[3, :, 700] = -np.inf
+    x[4, :, :] = 5.0  # every element ties
+    x[5, :, :] = -np.inf
+    x[5, :, 3] = np.nan
+    x[5, :, 770] = 1.0
+    logits = gen.f32_to_bf16_bits(np.nan_to_num(x, nan=0.0)) if dtype == "bf16" else x
+    if dtype == "bf16":
+        logits[np.isnan(x)] = 0x7FC1  # NaN pattern with a payload
+    am = oracle.argmax_rows(logits.reshape(-1, V), dtype).reshape(B, k + 1)
+    drafts = np.where(rng.random((B, k)) < 0.7, am[:, :k], rng.integers(-2, V + 2, (B, k))).astype(np.int32)
+    inp = gen.GreedyInputs("special", dtype, logits, drafts, B, k, V)
+    check_greedy(V_, inp)
+    check_greedy(V_, inp, topk=8)
+
+
+def test_greedy_out_of_range_drafts(V_):
+    inp = gen.greedy_synthetic(seed=9, B=16, k=4, V=500, alpha=1.0)
+    inp.drafts[::2, 1] = -1
+    inp.drafts[1::4, 0] = 500
+    inp.drafts[3::4, 2] = 2**31 - 1
+    check_greedy(V_, inp)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("offset,pad", [(1, 0), (0, 3), (1, 5), (0, 8)])
+def test_greedy_strided_and_unaligned(V_, dtype, offset, pad):
+    """Rows with padding (row_stride > V) and base pointers off the 16-byte
+    grid (the scalar path)."""
+    import torch
+    B, k, V = 6, 4, 2051
+    inp = gen.greedy_synthetic(seed=offset * 10 + pad, B=B, k=k, V=V, alpha=0.7, dtype=dtype)
+    stride = V + pad
+    full = np.zeros((B * (k + 1) * stride + offset,), dtype=inp.logits.dtype)
+    view = full[offset:].reshape(B, k + 1, stride)
+    view[..., :V] = inp.logits
+    flat = dev_logits(full, dtype)
+    x = torch.as_strided(flat, (B, k + 1, V), (stride * (k + 1), stride, 1), storage_offset=offset)
+    for topk in (0, 8):
+        res = [host(t) for t in V_.greedy(x, dev_i32(inp.drafts), topk=topk)]
+        al, out = oracle.verify_greedy(inp.logits, dtype, inp.drafts)
+        assert np.array_equal(res[0], al) and np.array_equal(res[1], out)
+        if topk:
+            ids, vals = oracle.topk_rows(inp.logits.reshape(-1, V), dtype, 8)
+            assert np.array_equal(res[2].reshape(-1, 8), ids)
+            assert np.array_equal(res[3].reshape(-1, 8).view(np.uint32), vals.view(np.uint32))
+
+
+def test_greedy_deterministic_and_canaries(V_):
+    """Repeated calls give identical bits; nothing is written past the
+    outputs."""
+    import torch
+    inp = gen.greedy_synthetic(seed=3, B=33, k=6, V=32000, alpha=0.8, dtype="bf16")
+    x = dev_logits(inp.logits, "bf16")
+    d = dev_i32(inp.drafts)
+    B, k1 = 33, 7
+    canary = -123456789
+    al = torch.full((B + 8,), canary, dtype=torch.int32, device="cuda")
+    ot = torch.full((B * k1 + 8,), canary, dtype=torch.int32, device="cuda")
+    ids = torch.full((B * k1 * 8 + 8,), canary, dtype=torch.int32, device="cuda")
+    vals = torch.full((B * k1 * 8 + 8,), 7.0, dtype=torch.float32, device="cuda")
+    outs = (al[:B], ot[: B * k1].view(B, k1), ids[: B * k1 * 8].view(B, k1, 8), vals[: B * k1 * 8].view(B, k1, 8))
+    first = None
+    for rep in range(5):
+        V_.greedy(x, d, topk=8, out=outs)
+        now = [host(t).copy() for t in outs]
+        if first is None:
+            first = now
+        for a, b in zip(first, now):
+            assert np.array_equal(a.view(np.uint32) if a.dtype == np.float32 else a,
+                                  b.view(np.uint32) if b.dtype == np.float32 else b)
+    assert (host(al[B:]) == canary).all() and (host(ot[B * k1:]) == canary).all()
+    assert (host(ids[B * k1 * 8:]) == canary).all() and (host(vals[B * k1 * 8:]) == 7.0).all()
+    al_o, out_o = oracle.verify_greedy(inp.logits, "bf16", inp.drafts)
+    assert np.array_equal(first[0], al_o) and np.array_equal(first[1], out_o)
+
+
+def test_workspace_reuse_across_shapes(V_):
+    """One workspace serves calls of different modes and shapes in any order
+    (the per-request counters return to zero after every call)."""
+    import torch
+    ver = sd.Verifier(torch.device("cuda", 0))
+    ver.workspace(sd.specdec_workspace_size(sd.SPECDEC_MODE_REJECTION, 300, 8, 40000, sd.SPECDEC_F32) * 2)
+    cases = [gen.greedy_synthetic(seed=s, B=b, k=kk, V=v, alpha=0.7, dtype=dt)
+             for s, (b, kk, v, dt) in enumerate([(300, 8, 4000, "f32"), (5, 2, 40000, "bf16"), (120, 0, 77, "f32"),
+                                                  (7, 31, 1000, "bf16")])]
+    for rep in range(2):
+        for inp in cases:
+            got = [host(t) for t in ver.greedy(dev_logits(inp.logits, inp.dtype), dev_i32(inp.drafts))]
+            al, out = oracle.verify_greedy(inp.logits, inp.dtype, inp.drafts)
+            assert np.array_equal(got[0], al) and np.array_equal(got[1], out)
+        t = gen.tree_synthetic(seed=rep, B=9, parents=gen.complete_tree_parents((3, 2, 2)), V=900, dtype="f32")
+        got = [host(a) for a in ver.tree(dev_logits(t.logits, "f32"), dev_i32(t.parents), dev_i32(t.node_tokens),
+                                         t.max_depth)]
+        exp = oracle.verify_tree(t.logits, "f32", t.parents, t.node_tokens, t.max_depth)
+        for a, b in zip(got, exp):
+            assert np.array_equal(a, b)
+
+
+def test_cuda_graph_replay(V_):
+    """The greedy call captured once in a CUDA graph and replayed over new
+    inputs copied into the captured buffers."""
+    import torch
+    B, k, V = 16, 5, 50000
+    ver = sd.Verifier(torch.device("cuda", 0))
+    ver.workspace(sd.specdec_workspace_size(sd.SPECDEC_MODE_GREEDY, B, k, V, sd.SPECDEC_BF16))
+    x = torch.zeros(B, k + 1, V, dtype=torch.bfloat16, device="cuda")
+    d = torch.zeros(B, k, dtype=torch.int32, device="cuda")
+    al = torch.zeros(B, dtype=torch.int32, device="cuda")
+    ot = torch.zeros(B, k + 1, dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        ver.greedy(x, d, out=(al, ot))  # warm-up outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ver.greedy(x, d, out=(al, ot))
+    for seed in range(4):
+        inp = gen.greedy_synthetic(seed=50 + seed, B=B, k=k, V=V, alpha=0.8, dtype="bf16")
+        x.copy_(dev_logits(inp.logits, "bf16"))
+        d.copy_(dev_i32(inp.drafts))
+        g.replay()
+        a, o = oracle.verify_greedy(inp.logits, "bf16", inp.drafts)
+        assert np.array_equal(host(al), a) and np.array_equal(host(ot), o)
+
+
+def test_toy_lut_identity_on_gpu(V_):
+    """Draft-then-verify with the CUDA verifier equals plain greedy decoding
+    of the toy lookup-table target."""
+    from test_oracle_pins import plain_greedy_decode, speculative_greedy_decode
+    tbl, draft = gen.toy_lut()
+
+    def verify(rows, d):
+        res = V_.greedy(dev_logits(rows.astype(np.float32), "f32"), dev_i32(d))
+        return [host(t) for t in res]
+
+    for k in (1, 4, 8):
+        got, steps = speculative_greedy_decode(tbl, draft, 3, 128, k, verify)
+        assert got == plain_greedy_decode(tbl, 3, 128)
+
+
+# ---------------------------------------------------------------------------
+# tree
+# ---------------------------------------------------------------------------
+def run_tree(ver, t):
+    res = ver.tree(dev_logits(t.logits, t.dtype), dev_i32(t.parents), dev_i32(t.node_tokens), t.max_depth)
+    return [host(a) for a in res]
+
+
+def check_tree(ver, t):
+    got = run_tree(ver, t)
+    exp = oracle.verify_tree(t.logits, t.dtype, t.parents, t.node_tokens, t.max_depth)
+    for a, b in zip(got, exp):
+        assert np.array_equal(a, b)
+    return got
+
+
+def test_tree_medusa_full(V_):
+    got = check_tree(V_, gen.tree_medusa())
+    assert got[0].max() >= 1
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_tree_random_shapes(V_, seed):
+    rng = np.random.default_rng(seed)
+    B, n1, V = 13, int(rng.integers(1, 200)), int(rng.integers(2, 3000))
+    par = np.array([-1] + [int(rng.integers(max(0, c - 6), c)) for c in range(1, n1)], np.int32)
+    t = gen.tree_synthetic(seed=seed, B=B, parents=par, V=V, p_agree=0.8, max_depth=32,
+                           dtype=["f32", "bf16"][seed % 2])
+    # per-request variations: some invalid, some with duplicate-token siblings
+    t.parents[1, min(2, n1 - 1)] = n1 + 5 if n1 > 2 else 3
+    t.parents[2, 0] = 0
+    t.node_tokens[3, 1:] = t.node_tokens[3, 1]
+    check_tree(V_, t)
+
+
+def test_tree_max_size_and_depth(V_):
+    n1 = 1024
+    par = np.array([-1] + [max(0, c - 1) if c <= 32 else int(c % 32) for c in range(1, n1)], np.int32)
+    t = gen.tree_synthetic(seed=1, B=3, parents=par, V=4096, p_agree=0.95, max_depth=32, dtype="bf16")
+    check_tree(V_, t)
+    # one level too deep for max_depth = 31 -> invalid
+    t.max_depth = 31
+    got = check_tree(V_, t)
+    assert (got[0] == -1).all()
+
+
+def test_tree_single_node(V_):
+    t = gen.tree_synthetic(seed=2, B=4, parents=np.array([-1], np.int32), V=100, dtype="f32", max_depth=1)
+    got = check_tree(V_, t)
+    assert (got[0] == 0).all()
+
+
+def test_tree_chain_equals_greedy_on_gpu(V_):
+    inp = gen.greedy_synthetic(seed=77, B=20, k=6, V=5000, alpha=0.75, dtype="bf16")
+    par = np.tile(np.array([-1] + list(range(6)), np.int32), (20, 1))
+    tok = np.concatenate([np.zeros((20, 1), np.int32), inp.drafts], axis=1)
+    t = gen.TreeInputs("chain", "bf16", inp.logits, par, tok, 20, 6, 5000, 6)
+    got = run_tree(V_, t)
+    g = run_greedy(V_, inp)
+    assert np.array_equal(got[0], g[0]) and np.array_equal(got[2], g[1])
+
+
+# ---------------------------------------------------------------------------
+# rejection sampling
+# ---------------------------------------------------------------------------
+def run_rejection(ver, r, seed=None, offset=None):
+    res = ver.rejection(dev_logits(r.target, r.dtype), dev_f32(r.q), dev_i32(r.drafts), r.temperature,
+                        r.seed if seed is None else seed, r.offset if offset is None else offset)
+    return [host(a) for a in res]
+
+
+def compare_rejection(got, exp):
+    """Returns (requests, exempt mismatches); asserts everything else."""
+    al_g, out_g, pd_g = got
+    al_o, out_o, pd_o, mg = exp
+    valid = al_o >= 0
+    assert np.array_equal(al_g[~valid], al_o[~valid])
+    assert (out_g[~valid] == -1).all()
+    pv, pg = pd_o[valid], pd_g[valid].astype(np.float64)
+    pos = pv > 0
+    assert np.all(np.abs(pg[pos] - pv[pos]) <= P_DRAFT_RTOL * pv[pos]), np.max(np.abs(pg[pos] / pv[pos] - 1))
+    assert np.all(pg[~pos] == 0)
+    mism = (al_g != al_o) | np.any(out_g != out_o, axis=1)
+    exempt = mg < MARGIN
+    bad = mism & ~exempt & valid
+    assert not bad.any(), (np.nonzero(bad), al_g[bad], al_o[bad], out_g[bad], out_o[bad], mg[bad])
+    return int(valid.sum()), int((mism & exempt).sum())
+
+
+def test_rejection_qwen_full(V_):
+    r = gen.rejection_qwen()
+    n, ex = 0, 0
+    for off in range(8):
+        got = run_rejection(V_, r, offset=off)
+        exp = oracle.verify_rejection(r.target, r.dtype, r.q, r.drafts, r.temperature, r.seed, off)
+        a, b = compare_rejection(got, exp)
+        n, ex = n + a, ex + b
+    assert ex <= EXEMPT_FRACTION * n
+
+
+@pytest.mark.parametrize("V,k,T,dtype", [(16, 3, 1.0, "f32"), (1000, 4, 0.7, "bf16"), (4099, 2, 1.3, "f32"),
+                                         (7, 0, 1.0, "f32"), (33, 8, 0.5, "bf16"), (151936, 1, 2.0, "f32")])
+def test_rejection_small_cases(V_, V, k, T, dtype):
+    rng = np.random.default_rng(V + k)
+    B = 64 if V < 100000 else 8
+    tgt = rng.standard_normal((B, k + 1, V)).astype(np.float32) * np.float32(1.5)
+    noisy = tgt[:, :k].astype(np.float64) + rng.standard_normal((B, k, V))
+    q = np.exp(noisy - noisy.max(-1, keepdims=True))
+    q = (q / q.sum(-1, keepdims=True)).astype(np.float32)
+    drafts = np.empty((B, k), np.int32)
+    for b in range(B):
+        for i in range(k):
+            c = np.cumsum(q[b, i].astype(np.float64))
+            drafts[b, i] = min(int(np.searchsorted(c, rng.random() * c[-1], side="right")), V - 1)
+    target = gen.f32_to_bf16_bits(tgt) if dtype == "bf16" else tgt
+    r = gen.RejectionInputs("small", dtype, target, q, drafts, B, k, V, temperature=T, seed=99, offset=5)
+    n, ex = 0, 0
+    for off in (0, 1, 2**33 + 1):
+        got = run_rejection(V_, r, offset=off)
+        exp = oracle.verify_rejection(r.target, dtype, r.q, r.drafts, T, r.seed, off)
+        a, b = compare_rejection(got, exp)
+        n, ex = n + a, ex + b
+    assert ex <= EXEMPT_FRACTION * n
+
+
+def test_rejection_special_cases(V_):
+    V, k = 50, 3
+    B = 6
+    target = np.zeros((B, k + 1, V), np.float32)
+    q = np.full((B, k, V), 1.0 / V, np.float32)
+    drafts = np.tile(np.array([[1, 2, 3]], np.int32), (B, 1))
+    target[1, 2, 7] = np.nan           # invalid request
+    target[2, 0, :] = -np.inf          # invalid: row of only -inf
+    target[3, 3, 9] = np.inf           # invalid: +inf
+    target[4, :, :10] = -np.inf        # fine: probability 0 entries
+    drafts[5, 1] = V + 3               # out-of-range draft: rejected at 1
+    r = gen.RejectionInputs("special", "f32", target, q, drafts, B, k, V, seed=3)
+    got = run_rejection(V_, r)
+    exp = oracle.verify_rejection(target, "f32", q, drafts, 1.0, 3, 0)
+    compare_rejection(got, exp)
+    assert list(got[0][1:4]) == [-1, -1, -1]
+    assert got[0][0] == k  # q == p accepts everything
+    assert got[0][5] <= 1
+
+
+def test_rejection_worked_example_gpu(V_):
+    V = gen.LLAMA3_VOCAB
+    drafts = np.array([[13, 578, 7301]], np.int32)
+    target = np.full((1, 4, V), -1.0e4, np.float32)
+    target[0, 0, 13] = target[0, 1, 578] = target[0, 2, 21747] = target[0, 3, 5] = 0.0
+    q = np.zeros((1, 3, V), np.float32)
+    for i, d in enumerate(drafts[0]):
+        q[0, i, d] = 1.0
+    r = gen.RejectionInputs("worked", "f32", target, q, drafts, 1, 3, V)
+    for seed in (0, 1, 1234):
+        al, out, pd = run_rejection(V_, r, seed=seed)
+        assert al[0] == 2 and list(out[0, :3]) == [13, 578, 21747]
+
+
+def test_rejection_distribution_on_gpu(V_):
+    """The emitted tokens of the CUDA path follow p at every position
+    (chi-square, V = 8, k = 3, 40000 requests in one call)."""
+    from scipy.stats import chisquare
+    from test_oracle_pins import _rejection_trials, _softmax64
+    V, k, n = 8, 3, 40_000
+    tgt1, q1, target, q, drafts = _rejection_trials(V, k, n, seed=83)
+    r = gen.RejectionInputs("chi2", "f32", target, q, drafts, n, k, V, seed=2024)
+    al, out, pd = run_rejection(V_, r)
+    for j in range(k + 1):
+        sel = al >= j
+        obs = np.bincount(out[sel, j], minlength=V)
+        exp = _softmax64(tgt1[j]) * sel.sum()
+        assert chisquare(obs, exp).pvalue > 1e-4
