@@ -175,6 +175,30 @@ specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int6
                                    int32_t* accept_len, int32_t* accept_nodes, int32_t* out_tokens,
                                    void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
+/* Greedy verification without a caller workspace.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory (plug-ins and engine hooks handed only input and output
+ * pointers, or processes whose memory pool already owns the GPU).  Arguments
+ * and results are those of specdec_verify_greedy; the scratch is a fixed
+ * library-owned device array of SPECDEC_STATIC_SCRATCH_BYTES per GPU, held
+ * from library load until process exit, and nothing is allocated.
+ *   - The first call on each device looks up that device's scratch address
+ *     (cudaGetSymbolAddress, with the device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     each call clears the counters it needs on `stream` first.  Calls that
+ *     may overlap on the GPU (other streams, other threads) race: serialise
+ *     them or use specdec_verify_greedy with separate workspaces.
+ *   - A call whose workspace need (specdec_workspace_size) exceeds
+ *     SPECDEC_STATIC_SCRATCH_BYTES returns SPECDEC_ERR_WORKSPACE and launches
+ *     nothing. */
+#define SPECDEC_STATIC_SCRATCH_BYTES (8u << 20)
+specdec_status specdec_verify_greedy_static_scratch(const void* logits, specdec_dtype dtype, int64_t row_stride,
+                                                    const int32_t* draft_tokens, int B, int k, int V,
+                                                    int32_t* accept_len, int32_t* out_tokens,
+                                                    int topk, int32_t* topk_ids, float* topk_vals,
+                                                    struct CUstream_st* stream);
+
 /* Static text for a status code. */
 const char* specdec_status_string(specdec_status status);
 

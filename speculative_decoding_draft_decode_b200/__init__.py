@@ -297,3 +297,20 @@ class Verifier:
                                         draft_tokens if k > 0 else None, B, k, V, temperature, seed, offset,
                                         al, ot, pd, ws, wsb, stream), "verify_rejection")
         return al, ot, (pd[:, :k] if pd is not None else None)
+
+
+def specdec_verify_greedy_static_scratch(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len, out_tokens,
+                                         topk, topk_ids, topk_vals, stream=None) -> int:
+    """Greedy verification using the library's fixed device scratch instead of
+    a caller workspace (for callers that cannot allocate device memory).
+    Calls that may overlap on the GPU race on that scratch."""
+    fn = lib().specdec_verify_greedy_static_scratch
+    if fn.argtypes is None:  # declare the C signature once (64-bit pointers and strides)
+        P, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        fn.argtypes = [P, i32, i64, P, i32, i32, i32, P, P, i32, P, P, P]
+        fn.restype = i32
+    return fn(_ptr(logits), dtype, row_stride, _ptr(draft_tokens), B, k, V, _ptr(accept_len), _ptr(out_tokens),
+              topk, _ptr(topk_ids), _ptr(topk_vals), _stream(stream))
+
+
+SPECDEC_STATIC_SCRATCH_BYTES = 8 << 20

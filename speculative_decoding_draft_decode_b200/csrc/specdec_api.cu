@@ -343,3 +343,63 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Greedy verification with library-owned scratch (no allocation anywhere).
+//
+// Some callers cannot allocate device memory: plug-ins and engine hooks that
+// are handed only their input and output pointers and no allocator, or code
+// running in a process whose memory pool already owns the whole GPU (a
+// serving engine that reserved HBM for its KV cache up front), where a
+// cudaMalloc would fail or fragment the pool.  For them the scratch lives in
+// a fixed file-scope device array of SPECDEC_STATIC_SCRATCH_BYTES, which
+// every GPU that loads this library holds until the process exits.
+//
+// Host code must not pass `g_static_scratch` itself to a kernel: on the host
+// that name is only a stand-in for the device symbol.  The device address is
+// looked up once per device with cudaGetSymbolAddress, with that device
+// current, on the first call made on it.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_static_scratch[SPECDEC_STATIC_SCRATCH_BYTES];
+
+namespace specdec {
+namespace {
+std::atomic<void*> g_static_scratch_addr[kMaxDevices];
+
+// Device address of this device's copy of g_static_scratch (set-up on the
+// first call per device; later calls read the cached pointer).
+cudaError_t static_scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    void* p = g_static_scratch_addr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return e;
+        g_static_scratch_addr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return cudaSuccess;
+}
+}  // namespace
+}  // namespace specdec
+
+extern "C" specdec_status specdec_verify_greedy_static_scratch(
+    const void* logits, specdec_dtype dtype, int64_t row_stride, const int32_t* draft_tokens, int B, int k, int V,
+    int32_t* accept_len, int32_t* out_tokens, int topk, int32_t* topk_ids, float* topk_vals,
+    struct CUstream_st* stream) {
+    const size_t need = specdec_workspace_size(SPECDEC_MODE_GREEDY, B, k, V, dtype);
+    if (need > SPECDEC_STATIC_SCRATCH_BYTES) return SPECDEC_ERR_WORKSPACE;  // beyond the fixed scratch
+    void* scratch = nullptr;
+    if (B > 0 && need > 0) {
+        if (specdec::static_scratch_address(&scratch) != cudaSuccess) return SPECDEC_ERR_CUDA;
+        // The request counters must start at zero; the array keeps whatever
+        // the previous call left, so clear this call's counters first.
+        if (cudaMemsetAsync(scratch, 0, static_cast<size_t>(B) * sizeof(unsigned),
+                            reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return SPECDEC_ERR_CUDA;
+    }
+    return specdec_verify_greedy(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len, out_tokens, topk,
+                                 topk_ids, topk_vals, scratch, scratch ? SPECDEC_STATIC_SCRATCH_BYTES : 0, stream);
+}
