@@ -36,7 +36,9 @@ sys.path.insert(0, ROOT)
 import gen  # noqa: E402
 
 METRIC = "verified rows/s and achieved HBM GB/s (% of B200 peak) for B×(k+1)×V verify"
-KERNEL_SOURCES = ["speculative_decoding_draft_decode_b200/csrc/verify_kernels.cuh",
+KERNEL_SOURCES = ["speculative_decoding_draft_decode_b200/csrc/verify_pass1.cuh",
+                  "speculative_decoding_draft_decode_b200/csrc/verify_resample.cuh",
+                  "speculative_decoding_draft_decode_b200/csrc/verify_common.cuh",
                   "speculative_decoding_draft_decode_b200/csrc/device_utils.cuh",
                   "speculative_decoding_draft_decode_b200/csrc/specdec_api.cu",
                   "speculative_decoding_draft_decode_b200/csrc/geometry.h",

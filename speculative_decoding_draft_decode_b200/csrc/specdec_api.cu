@@ -1,12 +1,14 @@
 // specdec_api.cu — the C-ABI (include/specdec.h): argument checks, workspace
 // layout, grid sizing and kernel launches.
 //
-// Workspace layout (byte offsets; the ticket words are at fixed places so a
-// workspace initialised once serves calls of any shape):
+// Workspace layout (byte offsets).  Everything that must be zero when a call
+// starts sits at a fixed place, so a workspace initialised once serves calls
+// of any shape; each call returns those words to zero before it ends.
 //   [0, 256 KiB)            pass-1 tickets, one 32-bit word per request
 //   [256 KiB, 512 KiB)      pass-2 tickets (rejection resample)
-//   [512 KiB, ...)          pass-1 partials: row r, slot s at (r*maxs + s)
-//   then (rejection only)   per-request RejState, pass-2 partials
+//   [512 KiB, 768 KiB)      top-8 thresholds, one word per row (first 65536 rows)
+//   then                    pass-1 partials, one slot per (chunk, warp)
+//   then (rejection only)   per-request RejState, per-unit masses of row h
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -16,44 +18,45 @@
 
 #include "../../include/specdec.h"
 #include "geometry.h"
-#include "verify_kernels.cuh"
+#include "verify_pass1.cuh"
+#include "verify_resample.cuh"
 
 namespace specdec {
 namespace {
 
 constexpr size_t kTicketBytes = static_cast<size_t>(SPECDEC_MAX_B) * sizeof(unsigned);
-constexpr size_t kPartialBase = 2 * kTicketBytes;
-constexpr int64_t kMinVecsPerCta = 128;   // smallest piece worth a CTA
+constexpr size_t kThetaBase = 2 * kTicketBytes;
+constexpr size_t kPartialBase = kThetaBase + static_cast<size_t>(kThetaRows) * sizeof(unsigned);
+constexpr int64_t kMinUnitsPerCta = 4;    // resample pass: 32-vector units
 constexpr int64_t kGridCap = 4096;        // largest grid any pass uses
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-    int64_t nv = 0, T1 = 0, G1max = 0, maxs1 = 0;
-    int64_t T2 = 0, G2max = 0, maxs2 = 0;
-    size_t partials1 = 0, state = 0, partials2 = 0, total = 0;
+    int64_t nv = 0, nv_full = 0, cpr = 0, NC = 0;
+    int64_t nu = 0, T2 = 0;
+    size_t partials1 = 0, state = 0, units = 0, total = 0;
 };
 
 // Layout of one call.  `vec` = elements per vector (1 on the scalar path),
-// `slot1` = bytes per pass-1 partial.
+// `slot1` = bytes per pass-1 partial (one per chunk and warp).
 Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t slot1, bool rejection) {
     Layout L;
     L.total = kPartialBase;
-    if (rows <= 0 || V <= 0) return L;  // nothing streamed: only the ticket area
+    if (rows <= 0 || V <= 0) return L;  // nothing streamed: only the fixed area
     L.nv = (V + vec - 1) / vec;
-    L.T1 = rows * L.nv;
-    L.G1max = grid_upper(L.T1, kMinVecsPerCta, kGridCap);
-    L.maxs1 = slots_bound(L.nv, L.T1, L.G1max);
+    L.nv_full = V / vec;
+    L.cpr = chunks_per_row(L.nv_full, vec);
+    L.NC = rows * L.cpr;
     L.partials1 = kPartialBase;
-    size_t end = L.partials1 + static_cast<size_t>(rows) * L.maxs1 * slot1;
+    size_t end = L.partials1 + static_cast<size_t>(L.NC) * NWARPS * slot1;
     if (rejection) {
         L.state = align_up(end, 256);
         end = L.state + static_cast<size_t>(B) * sizeof(RejState);
-        L.T2 = static_cast<int64_t>(B) * L.nv;
-        L.G2max = grid_upper(L.T2, kMinVecsPerCta, kGridCap);
-        L.maxs2 = slots_bound(L.nv, L.T2, L.G2max);
-        L.partials2 = align_up(end, 256);
-        end = L.partials2 + static_cast<size_t>(B) * L.maxs2 * sizeof(ResamplePartial);
+        L.nu = (L.nv + kUnitVecs - 1) / kUnitVecs;
+        L.T2 = static_cast<int64_t>(B) * L.nu;
+        L.units = align_up(end, 256);
+        end = L.units + static_cast<size_t>(L.T2) * sizeof(double2);
     }
     (void)rows_per_req;
     L.total = align_up(end, 256);
@@ -69,7 +72,9 @@ constexpr int kNumKernels = 32;
 std::atomic<int> g_sms[kMaxDevices];
 std::atomic<int> g_occ[kMaxDevices][kNumKernels];
 
-cudaError_t grid_cap(const void* fn, int kernel_id, int64_t* cap) {
+// Resident CTAs of `fn` on the current device (cached), after allowing it
+// `dyn_smem` bytes of dynamic shared memory.
+cudaError_t grid_cap(const void* fn, int kernel_id, int dyn_smem, int64_t* cap) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -82,7 +87,13 @@ cudaError_t grid_cap(const void* fn, int kernel_id, int64_t* cap) {
     }
     int occ = g_occ[dev][kernel_id].load(std::memory_order_relaxed);
     if (occ == 0) {
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NT, 0);
+        if (dyn_smem > 0) {
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+            if (e != cudaSuccess) return e;
+        }
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NT, dyn_smem);
         if (e != cudaSuccess) return e;
         if (occ < 1) occ = 1;
         g_occ[dev][kernel_id].store(occ, std::memory_order_relaxed);
@@ -101,14 +112,29 @@ bool rows_fit(int64_t rows, int64_t row_stride, int V) {
     return row_stride >= V && row_stride <= (int64_t(1) << 40) && rows * row_stride < (int64_t(1) << 52);
 }
 
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel of the stream drains; it waits (griddepcontrol)
+// before touching global memory, so stream order is kept.
+template <class Kernel, class Params>
+cudaError_t launch_pdl(Kernel fn, int64_t G, int dyn, cudaStream_t stream, const Params& P) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(G));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = static_cast<size_t>(dyn);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fn, P);
+}
+
 template <class Tag, int VEC, int MODE>
 specdec_status launch_pass1(Pass1Params P, cudaStream_t stream) {
     auto fn = verify_pass1_kernel<Tag, VEC, MODE>;
-    const int kid = MODE * 4 + (VEC == 1 ? 0 : 1) * 2 + (sizeof(typename Tag::storage) == 2 ? 1 : 0);
-    int64_t cap = 0;
-    if (grid_cap(reinterpret_cast<const void*>(fn), kid, &cap) != cudaSuccess) return SPECDEC_ERR_CUDA;
-    const int64_t G = grid_upper(P.T, kMinVecsPerCta, cap);
-    fn<<<static_cast<unsigned>(G), NT, 0, stream>>>(P);
+    if (P.NC > 0x7fffffffull) return SPECDEC_ERR_UNSUPPORTED;  // one CTA per chunk: 1-D grid limit
+    if (launch_pdl(fn, static_cast<int64_t>(P.NC), 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 
@@ -117,9 +143,9 @@ specdec_status launch_pass2(Pass2Params P, cudaStream_t stream) {
     auto fn = verify_resample_kernel<Tag, VEC>;
     const int kid = 16 + (VEC == 1 ? 0 : 1) * 2 + (sizeof(typename Tag::storage) == 2 ? 1 : 0);
     int64_t cap = 0;
-    if (grid_cap(reinterpret_cast<const void*>(fn), kid, &cap) != cudaSuccess) return SPECDEC_ERR_CUDA;
-    const int64_t G = grid_upper(P.T, kMinVecsPerCta, cap);
-    fn<<<static_cast<unsigned>(G), NT, 0, stream>>>(P);
+    if (grid_cap(reinterpret_cast<const void*>(fn), kid, 0, &cap) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    const int64_t G = grid_upper(P.T, kMinUnitsPerCta, cap);
+    if (launch_pdl(fn, G, 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 
@@ -149,21 +175,22 @@ specdec_status check_ws(void* ws, size_t ws_bytes, size_t need) {
     return SPECDEC_OK;
 }
 
-void fill_common(Pass1Params& P, const void* logits, int64_t row_stride, int V, const Layout& L, int vec,
-                 int64_t rows, int rows_per_req, int B, void* ws) {
+void fill_common(Pass1Params& P, const void* logits, int64_t row_stride, int V, const Layout& L, int64_t rows,
+                 int rows_per_req, int B, void* ws) {
     memset(&P, 0, sizeof(P));
+    char* base = static_cast<char*>(ws);
     P.logits = logits;
     P.row_stride = row_stride;
     P.V = V;
-    P.nv = static_cast<int>(L.nv);
-    P.nv_full = V / vec;
+    P.nv_full = static_cast<int>(L.nv_full);
     P.R = rows;
-    P.T = L.T1;
+    P.cpr = static_cast<int>(L.cpr);
+    P.NC = static_cast<uint64_t>(L.NC);
     P.rows_per_req = rows_per_req;
     P.B = B;
-    P.maxs = static_cast<int>(L.maxs1);
-    P.tickets = static_cast<unsigned*>(ws);
-    P.partials = static_cast<char*>(ws) + L.partials1;
+    P.tickets = reinterpret_cast<unsigned*>(base);
+    P.theta_row = reinterpret_cast<unsigned*>(base + kThetaBase);
+    P.partials = base + L.partials1;
 }
 
 }  // namespace
@@ -234,7 +261,7 @@ specdec_status specdec_verify_greedy(const void* logits, specdec_dtype dtype, in
     specdec_status st = check_ws(ws, ws_bytes, L.total);
     if (st != SPECDEC_OK) return st;
     Pass1Params P;
-    fill_common(P, logits, row_stride, V, L, ve, rows, k + 1, B, ws);
+    fill_common(P, logits, row_stride, V, L, rows, k + 1, B, ws);
     P.drafts = draft_tokens;
     P.k = k;
     P.accept_len = accept_len;
@@ -268,7 +295,7 @@ specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int6
     specdec_status st = check_ws(ws, ws_bytes, L.total);
     if (st != SPECDEC_OK) return st;
     Pass1Params P;
-    fill_common(P, logits, row_stride, V, L, ve, rows, N + 1, B, ws);
+    fill_common(P, logits, row_stride, V, L, rows, N + 1, B, ws);
     P.parents = parents;
     P.node_tokens = node_tokens;
     P.max_depth = max_depth;
@@ -303,7 +330,7 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
     const double invT_d = 1.0 / static_cast<double>(temperature);
     RejState* state = reinterpret_cast<RejState*>(static_cast<char*>(ws) + L.state);
     Pass1Params P;
-    fill_common(P, target_logits, row_stride, V, L, ve, rows, k + 1, B, ws);
+    fill_common(P, target_logits, row_stride, V, L, rows, k + 1, B, ws);
     P.drafts = draft_tokens;
     P.k = k;
     P.accept_len = accept_len;
@@ -328,16 +355,16 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
     Q.V = V;
     Q.nv = static_cast<int>(L.nv);
     Q.nv_full = V / ve;
+    Q.nu = static_cast<int>(L.nu);
     Q.T = L.T2;
     Q.B = B;
     Q.k = k;
-    Q.maxs = static_cast<int>(L.maxs2);
     Q.invT = static_cast<float>(invT_d);
     Q.seed = seed;
     Q.offset = offset;
     Q.state = state;
     Q.tickets = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kTicketBytes);
-    Q.partials = reinterpret_cast<ResamplePartial*>(static_cast<char*>(ws) + L.partials2);
+    Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
     Q.out_tokens = out_tokens;
     return dispatch_pass2(dtype, vec, Q, s);
 }

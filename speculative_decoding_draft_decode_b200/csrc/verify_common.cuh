@@ -1,0 +1,41 @@
+// verify_common.cuh — pieces shared by the two verify kernels: the state the
+// rejection pass hands to the resample pass, the programmatic-launch
+// controls, and the ordered-atomic helpers.
+#pragma once
+
+#include <cuda/atomic>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace specdec {
+
+// Per-request state handed from the rejection statistics pass to the
+// resample pass.
+struct RejState {
+    int32_t h;       // accepted drafts
+    int32_t valid;   // 0: the request's target distribution is undefined
+    float M;         // max logit of row h
+    float pad;
+    double Z;        // sum exp((l - M)/T) of row h
+    double pad2;
+};
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel of the stream finishes;
+// griddepcontrol.wait blocks until that kernel has completed and its memory
+// is visible, so every global access comes after it.  launch_dependents lets
+// the next such kernel start its own launch early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+// Request counters: a release-acquire increment at device scope.  The
+// release publishes every write the CTA made before its preceding barrier;
+// the acquire lets the CTA that sees the final count read all of them.
+__device__ __forceinline__ unsigned ticket_add(unsigned* p) {
+    cuda::atomic_ref<unsigned, cuda::thread_scope_device> a(*p);
+    return a.fetch_add(1u, cuda::memory_order_acq_rel);
+}
+
+}  // namespace specdec

@@ -1,0 +1,805 @@
+// verify_pass1.cuh — the streaming verify pass (greedy, top-8, tree, and the
+// rejection statistics).
+//
+// Work unit: a chunk of kChunk 16-byte vectors of ONE logit row (rows are cut
+// into cpr chunks; the last one is shorter and carries the ragged row end).
+// One CTA per chunk; chunks are numbered sub-chunk-major (all rows' first
+// chunks, then all rows' second chunks, ...).  The grid is many times larger
+// than what the GPU keeps resident, so the hardware block scheduler hands
+// chunks to SMs as they free up and no SM waits for a slower one.  Every
+// thread issues all its loads of the chunk at once; each warp reduces its
+// part (argmax key, top-8 keys, or softmax max/sum) and stores one partial
+// per (chunk, warp).  The CTA then takes a ticket for its request; the CTA
+// that takes a request's last ticket merges that request's partials (one
+// warp per row) and runs the request epilogue:
+//
+//   greedy     accept-prefix scan and correction/bonus token (Arctic page,
+//              "Verifier optimisation"; handbook, "How does speculative
+//              decoding work"; vLLM page, section 1), optional top-k rows
+//              (Arctic page, "Whole-system optimisation");
+//   tree       accepted-node DP by pointer jumping, deepest accepted node,
+//              path and bonus (handbook, "Medusa" and "EAGLE");
+//   rejection  p_i(d_i), Philox accept test, accepted length h (vLLM page,
+//              section 1: rejection sampling keeps the target distribution);
+//              the resample of row h is the second kernel.
+//
+// No CTA ever waits for another: the last ticket holder does the merge and
+// resets what it used (its ticket, its rows' top-8 thresholds), so the next
+// call (or a graph replay) starts from zero.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <float.h>
+#include <limits.h>
+#include <stdint.h>
+
+#include "device_utils.cuh"
+#include "philox.cuh"
+#include "verify_common.cuh"
+
+namespace specdec {
+
+constexpr int kMaxRowsPerReq = 33;  // k + 1 with k <= 32
+constexpr int kTreeNodes = 1024;    // N + 1
+constexpr int kThetaRows = 65536;   // rows with a shared top-8 threshold
+
+enum Pass1Mode { MODE_ARGMAX = 0, MODE_TOP8 = 1, MODE_TREE = 2, MODE_SOFTMAX = 3 };
+
+// Chunk shape: kU 16-byte vectors per thread (vector path).
+#ifndef SPECDEC_PIPE_U
+#define SPECDEC_PIPE_U 8
+#endif
+constexpr int kU = SPECDEC_PIPE_U;
+constexpr int kChunk = kU * NT;  // vectors per chunk
+// Vectors per chunk: the scalar path (one element per "vector") takes 8x as
+// many so that a chunk covers as many elements as on the vector path.
+__host__ __device__ constexpr int chunk_vecs(int vec) { return vec > 1 ? kChunk : kChunk * 8; }
+// Chunks per row for rows of nv_full full vectors.
+__host__ __device__ inline int64_t chunks_per_row(int64_t nv_full, int vec) {
+    return nv_full > 0 ? (nv_full + chunk_vecs(vec) - 1) / chunk_vecs(vec) : 1;
+}
+constexpr int kCandBuf = 64;  // top-8 candidate buffer per warp
+
+struct SoftmaxPartial {
+    float M;
+    float pad;
+    double S;
+};
+
+struct Pass1Params {
+    // streamed rows
+    const void* logits;
+    int64_t row_stride;
+    int V;
+    int nv_full;        // full vectors per row
+    int64_t R;          // rows
+    int cpr;            // chunks per row
+    uint64_t NC;        // chunks in total (R * cpr)
+    int rows_per_req;
+    int B;
+    // workspace
+    unsigned* tickets;          // [B] per request
+    unsigned* theta_row;        // [kThetaRows] top-8 thresholds (ordered keys)
+    void* partials;             // [R * cpr * NWARPS] slots
+    // greedy / rejection
+    const int32_t* drafts;
+    int k;
+    int32_t* accept_len;
+    int32_t* out_tokens;
+    int topk;
+    int32_t* topk_ids;
+    float* topk_vals;
+    // tree
+    const int32_t* parents;
+    const int32_t* node_tokens;
+    int max_depth;
+    int32_t* accept_nodes;
+    // rejection
+    const float* q;
+    int64_t q_stride;
+    float invT;
+    double invT_d;
+    uint64_t seed;
+    uint64_t offset;
+    float* p_draft_out;
+    RejState* state;
+};
+
+// Static shared memory of the pass-1 kernel.
+struct Pass1Smem {
+    uint64_t red[NWARPS];
+    uint64_t stage[NWARPS * 8];
+    uint64_t wtop[NWARPS][8];          // top-8: per-warp best keys
+    uint64_t cand[NWARPS][kCandBuf];   // top-8: per-warp candidate buffers
+    int epi_req;                       // 1: this CTA completed its request
+    int am[kMaxRowsPerReq];
+    int drafts[kMaxRowsPerReq];
+    float rowM[kMaxRowsPerReq];
+    double rowZ[kMaxRowsPerReq];
+};
+struct TreeArrays {
+    int am[kTreeNodes];
+    int par[kTreeNodes];
+    int tok[kTreeNodes];
+    int anc[kTreeNodes];
+    int dep[kTreeNodes];
+    int ok[kTreeNodes];
+};
+struct Pass1SmemTree : Pass1Smem {
+    TreeArrays t;
+};
+template <int MODE> struct SmemFor { using type = Pass1Smem; };
+template <> struct SmemFor<MODE_TREE> { using type = Pass1SmemTree; };
+
+// ---------------------------------------------------------------------------
+// One 16-byte vector as loaded: its max (NaN ignored) and its elements.
+// bf16 vectors use packed bf16x2 max, three per 8 elements.
+// ---------------------------------------------------------------------------
+template <class Tag, int VEC>
+struct VecOps;
+
+template <class Tag>
+struct VecOps<Tag, 1> {  // scalar path: w.x holds the widened value
+    static __device__ __forceinline__ float vmax(const uint4& w) { return __uint_as_float(w.x); }
+    static __device__ __forceinline__ float elem(const uint4& w, int) { return __uint_as_float(w.x); }
+};
+
+template <>
+struct VecOps<F32Tag, 4> {
+    static __device__ __forceinline__ float vmax(const uint4& w) {
+        return fmaxf(fmaxf(__uint_as_float(w.x), __uint_as_float(w.y)),
+                     fmaxf(__uint_as_float(w.z), __uint_as_float(w.w)));
+    }
+    static __device__ __forceinline__ float elem(const uint4& w, int e) {
+        const uint32_t x = e == 0 ? w.x : e == 1 ? w.y : e == 2 ? w.z : w.w;
+        return __uint_as_float(x);
+    }
+};
+
+__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t x) {
+    __nv_bfloat162 r;
+    memcpy(&r, &x, 4);
+    return r;
+}
+
+template <>
+struct VecOps<BF16Tag, 8> {
+    static __device__ __forceinline__ float vmax(const uint4& w) {
+        const __nv_bfloat162 m =
+            __hmax2(__hmax2(as_bf162(w.x), as_bf162(w.y)), __hmax2(as_bf162(w.z), as_bf162(w.w)));
+        uint32_t u;
+        memcpy(&u, &m, 4);
+        return fmaxf(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    }
+    static __device__ __forceinline__ float elem(const uint4& w, int e) {
+        const uint32_t x = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
+        return __uint_as_float((e & 1) ? (x & 0xffff0000u) : (x << 16));
+    }
+};
+
+__device__ __forceinline__ int ord_i32(float x) {  // monotone for non-NaN x; -0 below +0
+    const int i = __float_as_int(x);
+    return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float from_ord_i32(int k) { return __int_as_float(k >= 0 ? k : k ^ 0x7fffffff); }
+
+__device__ __forceinline__ float key_value(uint64_t key) {
+    const uint32_t o = static_cast<uint32_t>(key >> 32);
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+// ---------------------------------------------------------------------------
+// Per-warp chunk reducers.  begin() starts a chunk of row r; vec() takes one
+// loaded vector whose first element has index `base` (ok = false: no data for
+// this lane); scalar() takes one element of the ragged row end; end() stores
+// the warp's partial for the chunk.  vec() and scalar() are warp-collective.
+// ---------------------------------------------------------------------------
+
+// Argmax with a warp-level running best: a warp looks at its lanes' vectors
+// only when some vector max beats the warp's best, then takes the new max and
+// the lowest index holding it.  Within a warp, later iterations hold higher
+// indices, so a later tie never wins.  NaN never beats anything and -inf
+// never beats the initial -inf (a row without an element above -inf is
+// rescanned exactly by the epilogue).
+struct ArgmaxBest {
+    float v;
+    int i;
+};
+
+template <class Tag, int VEC>
+__device__ __noinline__ ArgmaxBest argmax_raise(uint4 w, int base, bool up, float m) {
+    const float nm = from_ord_i32(__reduce_max_sync(FULL_MASK, up ? ord_i32(m) : ord_i32(-INFINITY)));
+    unsigned idx = 0xffffffffu;
+    if (up && m == nm) {
+#pragma unroll
+        for (int e = VEC - 1; e >= 0; --e)
+            if (VecOps<Tag, VEC>::elem(w, e) == nm) idx = static_cast<unsigned>(base + e);
+    }
+    ArgmaxBest r;
+    r.v = nm;
+    r.i = static_cast<int>(__reduce_min_sync(FULL_MASK, idx));
+    return r;
+}
+
+template <class Tag, int VEC>
+struct ArgmaxReducer {
+    ArgmaxBest best;  // warp-uniform; i = -1: none yet
+    __device__ __forceinline__ void begin(int64_t, const Pass1Params&, Pass1Smem&) {
+        best.v = -INFINITY;
+        best.i = -1;
+    }
+    __device__ __forceinline__ void vec(const uint4& w, int base, bool ok, Pass1Smem&) {
+        const float m = ok ? VecOps<Tag, VEC>::vmax(w) : -INFINITY;
+        const bool up = m > best.v;
+        if (__any_sync(FULL_MASK, up)) best = argmax_raise<Tag, VEC>(w, base, up, m);
+    }
+    __device__ __forceinline__ void scalar(float v, int idx, bool ok, Pass1Smem&) {
+        uint4 w = make_uint4(__float_as_uint(v), 0u, 0u, 0u);
+        const float m = ok ? v : -INFINITY;
+        const bool up = m > best.v;
+        if (__any_sync(FULL_MASK, up)) best = argmax_raise<Tag, 1>(w, idx, up, m);
+    }
+    __device__ __forceinline__ void end(int64_t, uint64_t slot, const Pass1Params& P, Pass1Smem&) {
+        if ((threadIdx.x & 31) == 0)
+            static_cast<uint64_t*>(P.partials)[slot] = best.i >= 0 ? make_key(best.v, best.i) : 0ull;
+    }
+};
+
+// Top-8 with thresholds: each warp keeps the 8 best keys of its part of the
+// chunk; theta is the value of its 8th best (-inf until it has 8), and the
+// row's shared threshold (published by the chunks of the row finished
+// earlier, as the largest 8th-best any warp has seen) is another lower bound
+// on the row's 8th best.  Only elements >= the larger of the two can matter;
+// a warp appends those to a small buffer (ballot compaction) and merges the
+// buffer into its 8 best when it fills.  The first chunk of a row seeds theta
+// from the 8th largest lane maximum.  NaN never passes (a row with fewer than
+// 8 elements above NaN is rescanned exactly by the epilogue).
+struct Top8State {
+    float theta;  // own 8th best
+    float th;     // threshold in force
+    int cnt;      // buffered candidates
+};
+
+// Warp-collective: new best 8 of (current best 8, buffered candidates).
+__device__ __noinline__ Top8State top8_merge(Top8State st, uint64_t* wtop, uint64_t* cand) {
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    uint64_t a = lane < st.cnt ? cand[lane] : 0ull;
+    uint64_t b = lane + 32 < st.cnt ? cand[lane + 32] : 0ull;
+    uint64_t c = lane < 8 ? wtop[lane] : 0ull;
+    uint64_t mine = 0ull;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        uint64_t lm = a > b ? a : b;
+        lm = lm > c ? lm : c;
+        const uint64_t m = warp_max_u64(lm);
+        if (m != 0ull) {
+            if (a == m) a = 0ull;
+            else if (b == m) b = 0ull;
+            else if (c == m) c = 0ull;
+        }
+        if (lane == r) mine = m;
+    }
+    __syncwarp();
+    if (lane < 8) wtop[lane] = mine;
+    __syncwarp();
+    st.cnt = 0;
+    const uint64_t k7 = __shfl_sync(FULL_MASK, mine, 7);
+    if (k7 != 0ull) {
+        st.theta = key_value(k7);
+        st.th = fmaxf(st.th, st.theta);
+    }
+    return st;
+}
+
+// Warp-collective: append the elements of mask cm (bit e = element e of this
+// lane's vector w) that still reach the threshold.
+template <class Tag, int VEC>
+__device__ __noinline__ Top8State top8_offer(Top8State st, uint4 w, unsigned cm, int base, uint64_t* wtop,
+                                             uint64_t* cand) {
+    const int lane = threadIdx.x & 31;
+    while (__any_sync(FULL_MASK, cm != 0u)) {
+        const bool c = cm != 0u;
+        const int e = c ? __ffs(cm) - 1 : 0;
+        const unsigned mask = __ballot_sync(FULL_MASK, c);
+        if (st.cnt + __popc(mask) > kCandBuf) {
+            st = top8_merge(st, wtop, cand);
+            unsigned keep = 0u;  // drop what the raised threshold now excludes
+#pragma unroll
+            for (int f = 0; f < VEC; ++f)
+                if (VecOps<Tag, VEC>::elem(w, f) >= st.th) keep |= 1u << f;
+            cm &= keep;
+            continue;
+        }
+        if (c) cand[st.cnt + __popc(mask & ((1u << lane) - 1u))] = make_key(VecOps<Tag, VEC>::elem(w, e), base + e);
+        st.cnt += __popc(mask);
+        cm &= cm - 1u;
+    }
+    return st;
+}
+
+// Warp-collective: the 8th largest lane maximum (lm = -inf: no data).
+__device__ __noinline__ float top8_seed(float lm) {
+    const int lane = threadIdx.x & 31;
+    uint64_t key = lm > -INFINITY ? ((static_cast<uint64_t>(ord32(lm)) << 32) | static_cast<uint32_t>(lane)) : 0ull;
+    uint64_t k8 = 0ull;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const uint64_t m = warp_max_u64(key);
+        if (key == m) key = 0ull;
+        k8 = m;
+    }
+    return k8 != 0ull ? key_value(k8) : -INFINITY;
+}
+
+template <class Tag, int VEC>
+struct Top8Reducer {
+    Top8State st;  // warp-uniform
+    bool seed;     // warp-uniform: the row has no shared threshold yet
+
+    __device__ __forceinline__ void begin(int64_t r, const Pass1Params& P, Pass1Smem& sm) {
+        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+        st.theta = -INFINITY;
+        st.cnt = 0;
+        const unsigned o = r < kThetaRows ? *reinterpret_cast<volatile unsigned*>(&P.theta_row[r]) : 0u;
+        st.th = o != 0u ? key_value(static_cast<uint64_t>(o) << 32) : -INFINITY;
+        seed = o == 0u;
+        if (lane < 8) sm.wtop[w][lane] = 0ull;
+        __syncwarp();
+    }
+    __device__ __forceinline__ void seed_from(float lm) {
+        const float t = top8_seed(lm);
+        st.theta = t;
+        st.th = fmaxf(st.th, t);
+    }
+    __device__ __forceinline__ void vec(const uint4& w, int base, bool ok, Pass1Smem& sm) {
+        const float m = ok ? VecOps<Tag, VEC>::vmax(w) : __uint_as_float(0x7fc00000u);
+        const bool hit = m >= st.th;
+        if (__any_sync(FULL_MASK, hit)) {
+            unsigned cm = 0u;
+            if (hit) {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    if (VecOps<Tag, VEC>::elem(w, e) >= st.th) cm |= 1u << e;
+            }
+            const int wp = threadIdx.x >> 5;
+            st = top8_offer<Tag, VEC>(st, w, cm, base, sm.wtop[wp], sm.cand[wp]);
+        }
+    }
+    __device__ __forceinline__ void scalar(float v, int idx, bool ok, Pass1Smem& sm) {
+        const bool hit = ok && v >= st.th;
+        if (__any_sync(FULL_MASK, hit)) {
+            const int wp = threadIdx.x >> 5;
+            st = top8_offer<Tag, 1>(st, make_uint4(__float_as_uint(v), 0u, 0u, 0u), hit ? 1u : 0u, idx, sm.wtop[wp],
+                                    sm.cand[wp]);
+        }
+    }
+    __device__ __forceinline__ void end(int64_t r, uint64_t slot, const Pass1Params& P, Pass1Smem& sm) {
+        const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+        if (st.cnt > 0) st = top8_merge(st, sm.wtop[wp], sm.cand[wp]);
+        __syncwarp();
+        if (lane < 8) static_cast<uint64_t*>(P.partials)[slot * 8 + lane] = sm.wtop[wp][lane];
+        const uint64_t k7 = sm.wtop[wp][7];
+        if (lane == 0 && k7 != 0ull && r < kThetaRows) atomicMax(&P.theta_row[r], static_cast<unsigned>(k7 >> 32));
+    }
+};
+
+// Softmax statistics: running max M of the raw logits and S = sum
+// exp((l - M)/T), fp32 exp and sum within a vector, fp64 across vectors; the
+// warp's lanes are merged at the end of the chunk.
+template <class Tag, int VEC>
+struct SoftmaxReducer {
+    float M;
+    double S;
+    float invT;
+    double invT_d;
+    __device__ __forceinline__ void begin(int64_t, const Pass1Params&, Pass1Smem&) {
+        M = -FLT_MAX;
+        S = 0.0;
+    }
+    __device__ __forceinline__ void vec(const uint4& w, int, bool ok, Pass1Smem&) {
+        if (!ok) return;
+        const float m = VecOps<Tag, VEC>::vmax(w);
+        if (m > M) {
+            S *= exp((static_cast<double>(M) - static_cast<double>(m)) * invT_d);
+            M = m;
+        }
+        float s = 0.0f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) s += expf((VecOps<Tag, VEC>::elem(w, e) - M) * invT);
+        S += static_cast<double>(s);
+    }
+    __device__ __forceinline__ void scalar(float v, int, bool ok, Pass1Smem&) {
+        if (!ok) return;
+        if (v > M) {
+            S *= exp((static_cast<double>(M) - static_cast<double>(v)) * invT_d);
+            M = v;
+        }
+        S += static_cast<double>(expf((v - M) * invT));
+    }
+    __device__ __forceinline__ void end(int64_t, uint64_t slot, const Pass1Params& P, Pass1Smem&) {
+        MaxSum acc;
+        acc.M = M;
+        acc.S = S;
+        acc = warp_maxsum(acc, invT_d);
+        if ((threadIdx.x & 31) == 0) {
+            SoftmaxPartial sp;
+            sp.M = acc.M;
+            sp.pad = 0.0f;
+            sp.S = acc.S;
+            static_cast<SoftmaxPartial*>(P.partials)[slot] = sp;
+        }
+    }
+};
+
+template <class Tag, int VEC, int MODE> struct ReducerFor;
+template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_ARGMAX> { using type = ArgmaxReducer<Tag, VEC>; };
+template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_TREE> { using type = ArgmaxReducer<Tag, VEC>; };
+template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_TOP8> { using type = Top8Reducer<Tag, VEC>; };
+template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_SOFTMAX> { using type = SoftmaxReducer<Tag, VEC>; };
+
+// ---------------------------------------------------------------------------
+// Row merges for the epilogues: warp-collective, over the row's cpr * NWARPS
+// partials.  A row whose partials hold no element above -inf (argmax) or
+// fewer than 8 elements above NaN (top-8) is rescanned exactly, element by
+// element, so NaN and -inf rank correctly.
+// ---------------------------------------------------------------------------
+template <class Tag>
+__device__ uint64_t row_argmax_key(const Pass1Params& P, int64_t r) {
+    const int lane = threadIdx.x & 31;
+    const int np = P.cpr * NWARPS;
+    const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r * np;
+    uint64_t best = 0ull;
+    for (int i = lane; i < np; i += 32) {
+        const uint64_t kk = __ldcg(p + i);
+        best = kk > best ? kk : best;
+    }
+    best = warp_max_u64(best);
+    if (best == 0ull) {
+        const typename Tag::storage* row = static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride;
+        for (int x = lane; x < P.V; x += 32) {
+            const uint64_t kk = make_key(load_scalar<Tag>(row + x), x);
+            best = kk > best ? kk : best;
+        }
+        best = warp_max_u64(best);
+    }
+    return best;
+}
+
+// Lane e (< 8) returns the row's e-th best key.
+template <class Tag>
+__device__ uint64_t row_top8_key(const Pass1Params& P, int64_t r) {
+    const int lane = threadIdx.x & 31;
+    const int nk = P.cpr * NWARPS * 8;
+    const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r * nk;
+    uint64_t l[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) l[s] = 0ull;
+    for (int i = lane; i < nk; i += 32) {
+        const uint64_t kk = __ldcg(p + i);
+        if (kk > l[7]) top8_insert(l, kk);
+    }
+    uint64_t mine = warp_top8(l);
+    if (__shfl_sync(FULL_MASK, mine, 7) == 0ull) {
+        const typename Tag::storage* row = static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) l[s] = 0ull;
+        for (int x = lane; x < P.V; x += 32) {
+            const uint64_t kk = make_key(load_scalar<Tag>(row + x), x);
+            if (kk > l[7]) top8_insert(l, kk);
+        }
+        mine = warp_top8(l);
+    }
+    return mine;
+}
+
+// ---------------------------------------------------------------------------
+// Request epilogues (every thread of the last-ticket CTA).
+// ---------------------------------------------------------------------------
+template <class Tag, int MODE>
+__device__ void epilogue_greedy(const Pass1Params& P, int64_t b, Pass1Smem& sm) {
+    const int k = P.k;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    if (threadIdx.x < k) sm.drafts[threadIdx.x] = P.drafts[b * k + threadIdx.x];
+    for (int t = wp; t <= k; t += NWARPS) {
+        const int64_t r = b * (k + 1) + t;
+        if constexpr (MODE == MODE_TOP8) {
+            const uint64_t mine = row_top8_key<Tag>(P, r);
+            const uint64_t k0 = __shfl_sync(FULL_MASK, mine, 0);
+            if (lane == 0) sm.am[t] = key_index(k0);
+            if (lane < P.topk) {
+                int id = -1;
+                float val = __uint_as_float(0x7fc00000u);
+                if (mine != 0ull) {
+                    id = key_index(mine);
+                    val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + id);
+                }
+                P.topk_ids[r * P.topk + lane] = id;
+                P.topk_vals[r * P.topk + lane] = val;
+            }
+            if (lane == 0 && r < kThetaRows) P.theta_row[r] = 0u;
+        } else {
+            const uint64_t key = row_argmax_key<Tag>(P, r);
+            if (lane == 0) sm.am[t] = key_index(key);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        bool match = false;
+        if (lane < k) {
+            const int d = sm.drafts[lane];
+            match = d >= 0 && d < P.V && d == sm.am[lane];
+        }
+        const unsigned miss = __ballot_sync(FULL_MASK, lane < k && !match);
+        const int h = miss ? __ffs(miss) - 1 : k;
+        for (int i = lane; i <= k; i += 32) {
+            int tokv = -1;
+            if (i < h) tokv = sm.drafts[i];
+            else if (i == h) tokv = sm.am[h];
+            P.out_tokens[b * (k + 1) + i] = tokv;
+        }
+        if (lane == 0) P.accept_len[b] = h;
+    }
+}
+
+template <class Tag>
+__device__ void epilogue_tree(const Pass1Params& P, int64_t b, Pass1SmemTree& sm) {
+    TreeArrays& ts = sm.t;
+    const int n1 = P.rows_per_req;
+    const int md = P.max_depth;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    for (int c = threadIdx.x; c < n1; c += NT) {
+        ts.par[c] = P.parents[b * n1 + c];
+        ts.tok[c] = P.node_tokens[b * n1 + c];
+    }
+    for (int c = wp; c < n1; c += NWARPS) {
+        const uint64_t key = row_argmax_key<Tag>(P, b * n1 + c);
+        if (lane == 0) ts.am[c] = key_index(key);
+    }
+    __syncthreads();
+    int bad = 0;
+    for (int c = threadIdx.x; c < n1; c += NT) {
+        const int p = ts.par[c];
+        if (c == 0 ? (p != -1) : (p < 0 || p >= c)) bad = 1;
+    }
+    bad = __syncthreads_or(bad);
+    int32_t* nodes_out = P.accept_nodes + b * md;
+    int32_t* out = P.out_tokens + b * (md + 1);
+    if (!bad) {
+        for (int c = threadIdx.x; c < n1; c += NT) {
+            const int p = ts.par[c];
+            ts.anc[c] = p;
+            ts.dep[c] = c == 0 ? 0 : 1;
+            const int t = ts.tok[c];
+            ts.ok[c] = c == 0 ? 1 : (t >= 0 && t < P.V && t == ts.am[p]);
+        }
+        __syncthreads();
+        // Pointer jumping: after each round every node has summed the depth and
+        // AND-ed the match flags of twice as many ancestors.
+        constexpr int PER = kTreeNodes / NT;
+        for (int span = 1; span < n1; span <<= 1) {
+            int na[PER], nd[PER], no[PER];
+#pragma unroll
+            for (int q = 0; q < PER; ++q) {
+                const int c = threadIdx.x + q * NT;
+                if (c < n1) {
+                    const int a = ts.anc[c];
+                    if (a >= 0) {
+                        na[q] = ts.anc[a];
+                        nd[q] = ts.dep[c] + ts.dep[a];
+                        no[q] = ts.ok[c] & ts.ok[a];
+                    } else {
+                        na[q] = a;
+                        nd[q] = ts.dep[c];
+                        no[q] = ts.ok[c];
+                    }
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int q = 0; q < PER; ++q) {
+                const int c = threadIdx.x + q * NT;
+                if (c < n1) { ts.anc[c] = na[q]; ts.dep[c] = nd[q]; ts.ok[c] = no[q]; }
+            }
+            __syncthreads();
+        }
+        int deep = 0;
+        for (int c = threadIdx.x; c < n1; c += NT)
+            if (ts.dep[c] > md) deep = 1;
+        bad = __syncthreads_or(deep);
+    }
+    if (bad) {
+        for (int i = threadIdx.x; i < md; i += NT) nodes_out[i] = -1;
+        for (int i = threadIdx.x; i <= md; i += NT) out[i] = -1;
+        if (threadIdx.x == 0) P.accept_len[b] = -1;
+        return;
+    }
+    uint64_t key = 0ull;
+    for (int c = threadIdx.x; c < n1; c += NT)
+        if (ts.ok[c]) {
+            const uint64_t kk =
+                (static_cast<uint64_t>(ts.dep[c]) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(c));
+            key = kk > key ? kk : key;
+        }
+    key = block_max_u64(key, sm.red);
+    const int best = key_index(key);
+    const int d = ts.dep[best];
+    for (int i = d + threadIdx.x; i < md; i += NT) nodes_out[i] = -1;
+    for (int i = d + 1 + threadIdx.x; i <= md; i += NT) out[i] = -1;
+    if (threadIdx.x == 0) {
+        int c = best;
+        for (int i = d - 1; i >= 0; --i) {
+            nodes_out[i] = c;
+            out[i] = ts.tok[c];
+            c = ts.par[c];
+        }
+        out[d] = ts.am[best];
+        P.accept_len[b] = d;
+    }
+}
+
+template <class Tag>
+__device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& sm) {
+    const int k = P.k;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    for (int t = wp; t <= k; t += NWARPS) {
+        const int64_t r = b * (k + 1) + t;
+        const int np = P.cpr * NWARPS;
+        const SoftmaxPartial* p = static_cast<const SoftmaxPartial*>(P.partials) + r * np;
+        MaxSum acc;
+        acc.M = -FLT_MAX;
+        acc.S = 0.0;
+        for (int i = lane; i < np; i += 32) {
+            MaxSum x;
+            x.M = __ldcg(&p[i].M);
+            x.S = __ldcg(&p[i].S);
+            acc = maxsum_merge(acc, x, P.invT_d);
+        }
+        acc = warp_maxsum(acc, P.invT_d);
+        if (lane == 0) {
+            sm.rowM[t] = acc.M;
+            sm.rowZ[t] = acc.S;
+        }
+    }
+    __syncthreads();
+    int bad = 0;
+    for (int t = threadIdx.x; t <= k; t += NT) {
+        const double z = sm.rowZ[t];
+        if (!(z > 0.0 && z <= DBL_MAX)) bad = 1;  // NaN, 0 or inf
+    }
+    bad = __syncthreads_or(bad);
+    if (bad) {
+        for (int i = threadIdx.x; i <= k; i += NT) P.out_tokens[b * (k + 1) + i] = -1;
+        if (P.p_draft_out)
+            for (int i = threadIdx.x; i < k; i += NT) P.p_draft_out[b * k + i] = __uint_as_float(0x7fc00000u);
+        if (threadIdx.x == 0) {
+            P.accept_len[b] = -1;
+            RejState st = {};
+            st.valid = 0;
+            P.state[b] = st;
+        }
+        return;
+    }
+    if (threadIdx.x < 32) {
+        bool accept = false;
+        if (lane < k) {
+            const int d = P.drafts[b * k + lane];
+            const bool in = d >= 0 && d < P.V;
+            double p = 0.0, qd = 0.0;
+            if (in) {
+                const int64_t r = b * (k + 1) + lane;
+                const float l =
+                    load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + d);
+                p = exp((static_cast<double>(l) - static_cast<double>(sm.rowM[lane])) * P.invT_d) / sm.rowZ[lane];
+                qd = static_cast<double>(__ldg(P.q + (b * k + lane) * P.q_stride + d));
+            }
+            if (P.p_draft_out) P.p_draft_out[b * k + lane] = static_cast<float>(p);
+            const double2 u = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(lane));
+            accept = in && (u.x * qd < p);
+        }
+        const unsigned rej = __ballot_sync(FULL_MASK, lane < k && !accept);
+        const int h = rej ? __ffs(rej) - 1 : k;
+        for (int i = lane; i <= k; i += 32) {
+            if (i < h) P.out_tokens[b * (k + 1) + i] = P.drafts[b * k + i];
+            else if (i > h) P.out_tokens[b * (k + 1) + i] = -1;
+        }
+        if (lane == 0) {
+            P.accept_len[b] = h;
+            RejState st = {};
+            st.h = h;
+            st.valid = 1;
+            st.M = sm.rowM[h];
+            st.Z = sm.rowZ[h];
+            P.state[b] = st;
+        }
+    }
+}
+
+template <class Tag, int MODE, class Smem>
+__device__ __forceinline__ void run_epilogue(const Pass1Params& P, int64_t b, Smem& sm) {
+    if constexpr (MODE == MODE_TREE) epilogue_tree<Tag>(P, b, sm);
+    else if constexpr (MODE == MODE_SOFTMAX) epilogue_rejection<Tag>(P, b, sm);
+    else epilogue_greedy<Tag, MODE>(P, b, sm);
+    if (threadIdx.x == 0) P.tickets[b] = 0u;
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// Pass-1 kernel: one CTA per chunk.  The grid holds many more CTAs than the
+// GPU keeps resident, so the hardware block scheduler hands chunks to SMs as
+// they free up (faster SMs take more chunks) and no counter is shared.  Every
+// thread issues all its loads of the chunk at once (kU x 16 bytes in flight
+// per thread), then its warp reduces.
+// ---------------------------------------------------------------------------
+template <class Tag, int VEC, int MODE>
+__global__ void __launch_bounds__(NT) verify_pass1_kernel(const Pass1Params P) {
+    __shared__ typename SmemFor<MODE>::type sm;
+    using Elem = typename Tag::storage;
+    constexpr int CH = chunk_vecs(VEC);  // vectors per chunk
+    constexpr int UPT = CH / NT;         // vectors per thread
+    constexpr int BATCH = UPT < kU ? UPT : kU;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    // Chunk c: row c % R, sub-chunk c / R (vectors [sub*CH, ...)).
+    const uint64_t c = blockIdx.x;
+    const uint64_t R = static_cast<uint64_t>(P.R);
+    const int64_t r = static_cast<int64_t>(c % R);
+    const int sub = static_cast<int>(c / R);
+    int cnt = P.nv_full - sub * CH;
+    cnt = cnt < CH ? cnt : CH;  // may be <= 0: only the ragged row end
+    const Elem* row = static_cast<const Elem*>(P.logits) + r * P.row_stride;
+
+    typename ReducerFor<Tag, VEC, MODE>::type red;
+    if constexpr (MODE == MODE_SOFTMAX) {
+        red.invT = P.invT;
+        red.invT_d = P.invT_d;
+    }
+    red.begin(r, P, sm);
+    for (int u0 = 0; u0 < UPT; u0 += BATCH) {
+        uint4 w[BATCH];
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int i = (u0 + u) * NT + static_cast<int>(threadIdx.x);
+            w[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < cnt) RowLoader<Tag, VEC>::raw(row, sub * CH + i, w[u]);
+        }
+        if constexpr (MODE == MODE_TOP8) {
+            if (u0 == 0 && red.seed) {
+                float lm = -INFINITY;
+#pragma unroll
+                for (int u = 0; u < BATCH; ++u)
+                    if (u * NT + static_cast<int>(threadIdx.x) < cnt) lm = fmaxf(lm, VecOps<Tag, VEC>::vmax(w[u]));
+                red.seed_from(lm);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int i = (u0 + u) * NT + static_cast<int>(threadIdx.x);
+            red.vec(w[u], (sub * CH + i) * VEC, i < cnt, sm);
+        }
+    }
+    if (sub == P.cpr - 1 && P.nv_full * VEC < P.V && wp == 0) {  // ragged row end: warp 0
+        for (int x0 = P.nv_full * VEC; x0 < P.V; x0 += 32) {
+            const int x = x0 + lane;
+            const bool ok = x < P.V;
+            red.scalar(ok ? load_scalar<Tag>(row + x) : 0.0f, x, ok, sm);
+        }
+    }
+    red.end(r, (static_cast<uint64_t>(r) * P.cpr + sub) * NWARPS + wp, P, sm);
+
+    // Ticket for the request; the CTA that completes it runs the epilogue.
+    __syncthreads();
+    const int64_t b = r / P.rows_per_req;
+    if (threadIdx.x == 0) {
+        const unsigned need = static_cast<unsigned>(P.rows_per_req * P.cpr);
+        sm.epi_req = ticket_add(&P.tickets[b]) + 1u == need ? 1 : 0;
+    }
+    __syncthreads();
+    if (sm.epi_req) run_epilogue<Tag, MODE>(P, b, sm);
+}
+
+}  // namespace specdec

@@ -134,6 +134,26 @@ def test_greedy_nan_inf_ties(V_, dtype):
     check_greedy(V_, inp, topk=8)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_top8_monotone_rows(V_, dtype):
+    """Worst cases for the per-warp top-8 filter: ascending rows (every element
+    beats the threshold), descending rows, constant rows and rows of a few
+    distinct values (many ties at the threshold)."""
+    B, k, V = 3, 3, 50001
+    x = np.empty((B, k + 1, V), np.float32)
+    x[0, 0] = np.linspace(-5, 5, V, dtype=np.float32)
+    x[0, 1] = np.linspace(5, -5, V, dtype=np.float32)
+    x[0, 2] = 1.5
+    x[0, 3] = np.arange(V, dtype=np.float32) % 3
+    rng = np.random.default_rng(12)
+    x[1] = np.floor(rng.random((k + 1, V)) * 4).astype(np.float32)
+    x[2] = np.sort(rng.standard_normal((k + 1, V)).astype(np.float32), axis=-1)
+    logits = gen.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    am = oracle.argmax_rows(logits.reshape(-1, V), dtype).reshape(B, k + 1)
+    inp = gen.GreedyInputs("monotone", dtype, logits, am[:, :k].copy(), B, k, V)
+    check_greedy(V_, inp, topk=8)
+
+
 def test_greedy_out_of_range_drafts(V_):
     inp = gen.greedy_synthetic(seed=9, B=16, k=4, V=500, alpha=1.0)
     inp.drafts[::2, 1] = -1
