@@ -39,7 +39,7 @@ struct Layout {
 };
 
 // Layout of one call.  `vec` = elements per vector (1 on the scalar path),
-// `slot1` = bytes per pass-1 partial (one per chunk and warp).
+// `slot1` = bytes of pass-1 partials per chunk.
 Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t slot1, bool rejection) {
     Layout L;
     L.total = kPartialBase;
@@ -49,7 +49,7 @@ Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t
     L.cpr = chunks_per_row(L.nv_full, vec);
     L.NC = rows * L.cpr;
     L.partials1 = kPartialBase;
-    size_t end = L.partials1 + static_cast<size_t>(L.NC) * NWARPS * slot1;
+    size_t end = L.partials1 + static_cast<size_t>(L.NC) * slot1;
     if (rejection) {
         L.state = align_up(end, 256);
         end = L.state + static_cast<size_t>(B) * sizeof(RejState);
@@ -116,9 +116,9 @@ bool rows_fit(int64_t rows, int64_t row_stride, int V) {
 // while the previous kernel of the stream drains; it waits (griddepcontrol)
 // before touching global memory, so stream order is kept.
 template <class Kernel, class Params>
-cudaError_t launch_pdl(Kernel fn, int64_t G, int dyn, cudaStream_t stream, const Params& P) {
+cudaError_t launch_pdl(Kernel fn, dim3 grid, int dyn, cudaStream_t stream, const Params& P) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(G));
+    cfg.gridDim = grid;
     cfg.blockDim = dim3(NT);
     cfg.dynamicSmemBytes = static_cast<size_t>(dyn);
     cfg.stream = stream;
@@ -130,11 +130,17 @@ cudaError_t launch_pdl(Kernel fn, int64_t G, int dyn, cudaStream_t stream, const
     return cudaLaunchKernelEx(&cfg, fn, P);
 }
 
+// The streaming pass (one CTA per chunk; trees stream like greedy argmax),
+// then the request epilogues (one CTA per request).
 template <class Tag, int VEC, int MODE>
 specdec_status launch_pass1(Pass1Params P, cudaStream_t stream) {
-    auto fn = verify_pass1_kernel<Tag, VEC, MODE>;
-    if (P.NC > 0x7fffffffull) return SPECDEC_ERR_UNSUPPORTED;  // one CTA per chunk: 1-D grid limit
-    if (launch_pdl(fn, static_cast<int64_t>(P.NC), 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    constexpr int STREAM_MODE = MODE == MODE_TREE ? MODE_ARGMAX : MODE;
+    if (P.R > 0x7fffffff || P.cpr > 65535) return SPECDEC_ERR_UNSUPPORTED;  // grid limits
+    const dim3 grid(static_cast<unsigned>(P.R), static_cast<unsigned>(P.cpr));
+    if (launch_pdl(verify_pass1_kernel<Tag, VEC, STREAM_MODE>, grid, 0, stream, P) != cudaSuccess)
+        return SPECDEC_ERR_CUDA;
+    if (launch_pdl(verify_epilogue_kernel<Tag, MODE>, dim3(static_cast<unsigned>(P.B)), 0, stream, P) != cudaSuccess)
+        return SPECDEC_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 
@@ -145,7 +151,7 @@ specdec_status launch_pass2(Pass2Params P, cudaStream_t stream) {
     int64_t cap = 0;
     if (grid_cap(reinterpret_cast<const void*>(fn), kid, 0, &cap) != cudaSuccess) return SPECDEC_ERR_CUDA;
     const int64_t G = grid_upper(P.T, kMinUnitsPerCta, cap);
-    if (launch_pdl(fn, G, 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    if (launch_pdl(fn, dim3(static_cast<unsigned>(G)), 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 
@@ -163,10 +169,15 @@ specdec_status dispatch_pass2(specdec_dtype dt, bool vec, Pass2Params P, cudaStr
 
 bool dtype_ok(specdec_dtype dt) { return dt == SPECDEC_F32 || dt == SPECDEC_BF16; }
 
+// Pass-1 partial bytes per chunk: one argmax key per warp, 8 keys per warp
+// (top-8), or the chunk's (max, sum) pair.
+constexpr size_t kArgmaxChunkBytes = NWARPS * sizeof(uint64_t);
+constexpr size_t kTop8ChunkBytes = NWARPS * 8 * sizeof(uint64_t);
+constexpr size_t kSoftmaxChunkBytes = sizeof(SoftmaxPartial);
 size_t slot_bytes(specdec_mode mode) {
-    if (mode == SPECDEC_MODE_GREEDY) return 8 * sizeof(uint64_t);  // room for top-8
-    if (mode == SPECDEC_MODE_REJECTION) return sizeof(SoftmaxPartial);
-    return sizeof(uint64_t);
+    if (mode == SPECDEC_MODE_GREEDY) return kArgmaxChunkBytes > kTop8ChunkBytes ? kArgmaxChunkBytes : kTop8ChunkBytes;
+    if (mode == SPECDEC_MODE_REJECTION) return kSoftmaxChunkBytes;
+    return kArgmaxChunkBytes;
 }
 
 specdec_status check_ws(void* ws, size_t ws_bytes, size_t need) {
@@ -188,7 +199,6 @@ void fill_common(Pass1Params& P, const void* logits, int64_t row_stride, int V, 
     P.NC = static_cast<uint64_t>(L.NC);
     P.rows_per_req = rows_per_req;
     P.B = B;
-    P.tickets = reinterpret_cast<unsigned*>(base);
     P.theta_row = reinterpret_cast<unsigned*>(base + kThetaBase);
     P.partials = base + L.partials1;
 }
@@ -257,7 +267,7 @@ specdec_status specdec_verify_greedy(const void* logits, specdec_dtype dtype, in
     if (topk > 0 && (topk_ids == nullptr || topk_vals == nullptr)) return SPECDEC_ERR_INVALID_ARG;
     const bool vec = vector_path_ok(logits, row_stride, elem_size(dtype));
     const int ve = vec ? vec_elems(dtype) : 1;
-    const Layout L = make_layout(rows, k + 1, B, V, ve, topk > 0 ? 64 : 8, false);
+    const Layout L = make_layout(rows, k + 1, B, V, ve, topk > 0 ? kTop8ChunkBytes : kArgmaxChunkBytes, false);
     specdec_status st = check_ws(ws, ws_bytes, L.total);
     if (st != SPECDEC_OK) return st;
     Pass1Params P;
@@ -291,7 +301,7 @@ specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int6
         return SPECDEC_ERR_INVALID_ARG;
     const bool vec = vector_path_ok(logits, row_stride, elem_size(dtype));
     const int ve = vec ? vec_elems(dtype) : 1;
-    const Layout L = make_layout(rows, N + 1, B, V, ve, 8, false);
+    const Layout L = make_layout(rows, N + 1, B, V, ve, kArgmaxChunkBytes, false);
     specdec_status st = check_ws(ws, ws_bytes, L.total);
     if (st != SPECDEC_OK) return st;
     Pass1Params P;
@@ -324,7 +334,7 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
     const bool vec = vector_path_ok(target_logits, row_stride, elem_size(dtype)) &&
                      (k == 0 || vector_path_ok(draft_probs, q_row_stride, 4));
     const int ve = vec ? vec_elems(dtype) : 1;
-    const Layout L = make_layout(rows, k + 1, B, V, ve, sizeof(SoftmaxPartial), true);
+    const Layout L = make_layout(rows, k + 1, B, V, ve, kSoftmaxChunkBytes, true);
     specdec_status st = check_ws(ws, ws_bytes, L.total);
     if (st != SPECDEC_OK) return st;
     const double invT_d = 1.0 / static_cast<double>(temperature);

@@ -3,8 +3,8 @@
 //
 // Work unit: a chunk of kChunk 16-byte vectors of ONE logit row (rows are cut
 // into cpr chunks; the last one is shorter and carries the ragged row end).
-// One CTA per chunk; chunks are numbered sub-chunk-major (all rows' first
-// chunks, then all rows' second chunks, ...).  The grid is many times larger
+// One CTA per chunk, on a (row, sub-chunk) grid scheduled sub-chunk-major
+// (all rows' first chunks, then all rows' second chunks, ...).  The grid is many times larger
 // than what the GPU keeps resident, so the hardware block scheduler hands
 // chunks to SMs as they free up and no SM waits for a slower one.  Every
 // thread issues all its loads of the chunk at once; each warp reduces its
@@ -79,7 +79,6 @@ struct Pass1Params {
     int rows_per_req;
     int B;
     // workspace
-    unsigned* tickets;          // [B] per request
     unsigned* theta_row;        // [kThetaRows] top-8 thresholds (ordered keys)
     void* partials;             // [R * cpr * NWARPS] slots
     // greedy / rejection
@@ -112,13 +111,16 @@ struct Pass1Smem {
     uint64_t stage[NWARPS * 8];
     uint64_t wtop[NWARPS][8];          // top-8: per-warp best keys
     uint64_t cand[NWARPS][kCandBuf];   // top-8: per-warp candidate buffers
-    int epi_req;                       // 1: this CTA completed its request
+    int wcnt[NWARPS];                  // top-8: candidates left in each buffer
+    float seed_theta;                  // top-8: CTA-wide seed threshold
+    uint64_t rowkey[kMaxRowsPerReq];   // epilogue: merged argmax key per row
     int am[kMaxRowsPerReq];
     int drafts[kMaxRowsPerReq];
     float rowM[kMaxRowsPerReq];
     double rowZ[kMaxRowsPerReq];
 };
 struct TreeArrays {
+    uint64_t key[kTreeNodes];
     int am[kTreeNodes];
     int par[kTreeNodes];
     int tok[kTreeNodes];
@@ -208,7 +210,7 @@ struct ArgmaxBest {
 };
 
 template <class Tag, int VEC>
-__device__ __noinline__ ArgmaxBest argmax_raise(uint4 w, int base, bool up, float m) {
+__device__ __forceinline__ ArgmaxBest argmax_raise(uint4 w, int base, bool up, float m) {
     const float nm = from_ord_i32(__reduce_max_sync(FULL_MASK, up ? ord_i32(m) : ord_i32(-INFINITY)));
     unsigned idx = 0xffffffffu;
     if (up && m == nm) {
@@ -225,7 +227,7 @@ __device__ __noinline__ ArgmaxBest argmax_raise(uint4 w, int base, bool up, floa
 template <class Tag, int VEC>
 struct ArgmaxReducer {
     ArgmaxBest best;  // warp-uniform; i = -1: none yet
-    __device__ __forceinline__ void begin(int64_t, const Pass1Params&, Pass1Smem&) {
+    __device__ __forceinline__ void begin(int64_t, int, const Pass1Params&, Pass1Smem&) {
         best.v = -INFINITY;
         best.i = -1;
     }
@@ -240,9 +242,10 @@ struct ArgmaxReducer {
         const bool up = m > best.v;
         if (__any_sync(FULL_MASK, up)) best = argmax_raise<Tag, 1>(w, idx, up, m);
     }
-    __device__ __forceinline__ void end(int64_t, uint64_t slot, const Pass1Params& P, Pass1Smem&) {
+    __device__ __forceinline__ void end(int64_t, int, uint64_t chunk, const Pass1Params& P, Pass1Smem&) {
         if ((threadIdx.x & 31) == 0)
-            static_cast<uint64_t*>(P.partials)[slot] = best.i >= 0 ? make_key(best.v, best.i) : 0ull;
+            static_cast<uint64_t*>(P.partials)[chunk * NWARPS + (threadIdx.x >> 5)] =
+                best.i >= 0 ? make_key(best.v, best.i) : 0ull;
     }
 };
 
@@ -259,6 +262,7 @@ struct Top8State {
     float theta;  // own 8th best
     float th;     // threshold in force
     int cnt;      // buffered candidates
+    int merged;   // the warp's best-8 list holds entries
 };
 
 // Warp-collective: new best 8 of (current best 8, buffered candidates).
@@ -285,6 +289,7 @@ __device__ __noinline__ Top8State top8_merge(Top8State st, uint64_t* wtop, uint6
     if (lane < 8) wtop[lane] = mine;
     __syncwarp();
     st.cnt = 0;
+    st.merged = 1;
     const uint64_t k7 = __shfl_sync(FULL_MASK, mine, 7);
     if (k7 != 0ull) {
         st.theta = key_value(k7);
@@ -296,7 +301,7 @@ __device__ __noinline__ Top8State top8_merge(Top8State st, uint64_t* wtop, uint6
 // Warp-collective: append the elements of mask cm (bit e = element e of this
 // lane's vector w) that still reach the threshold.
 template <class Tag, int VEC>
-__device__ __noinline__ Top8State top8_offer(Top8State st, uint4 w, unsigned cm, int base, uint64_t* wtop,
+__device__ __forceinline__ Top8State top8_offer(Top8State st, uint4 w, unsigned cm, int base, uint64_t* wtop,
                                              uint64_t* cand) {
     const int lane = threadIdx.x & 31;
     while (__any_sync(FULL_MASK, cm != 0u)) {
@@ -319,39 +324,50 @@ __device__ __noinline__ Top8State top8_offer(Top8State st, uint4 w, unsigned cm,
     return st;
 }
 
-// Warp-collective: the 8th largest lane maximum (lm = -inf: no data).
-__device__ __noinline__ float top8_seed(float lm) {
-    const int lane = threadIdx.x & 31;
-    uint64_t key = lm > -INFINITY ? ((static_cast<uint64_t>(ord32(lm)) << 32) | static_cast<uint32_t>(lane)) : 0ull;
-    uint64_t k8 = 0ull;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const uint64_t m = warp_max_u64(key);
-        if (key == m) key = 0ull;
-        k8 = m;
-    }
-    return k8 != 0ull ? key_value(k8) : -INFINITY;
-}
-
 template <class Tag, int VEC>
 struct Top8Reducer {
     Top8State st;  // warp-uniform
-    bool seed;     // warp-uniform: the row has no shared threshold yet
+    bool seed;     // CTA-uniform: the row has no shared threshold yet
 
-    __device__ __forceinline__ void begin(int64_t r, const Pass1Params& P, Pass1Smem& sm) {
+    // The first sub-chunk of a row seeds its own threshold (CTA-collective);
+    // later ones start from the row's shared threshold, read per warp.
+    __device__ __forceinline__ void begin(int64_t r, int sub, const Pass1Params& P, Pass1Smem& sm) {
         const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
         st.theta = -INFINITY;
         st.cnt = 0;
-        const unsigned o = r < kThetaRows ? *reinterpret_cast<volatile unsigned*>(&P.theta_row[r]) : 0u;
-        st.th = o != 0u ? key_value(static_cast<uint64_t>(o) << 32) : -INFINITY;
-        seed = o == 0u;
+        st.merged = 0;
+        st.th = -INFINITY;
         if (lane < 8) sm.wtop[w][lane] = 0ull;
+        seed = sub == 0;
+        if (!seed && r < kThetaRows) {
+            unsigned o = 0u;
+            if (lane == 0) o = *reinterpret_cast<volatile unsigned*>(&P.theta_row[r]);
+            o = __shfl_sync(FULL_MASK, o, 0);
+            if (o != 0u) st.th = key_value(static_cast<uint64_t>(o) << 32);
+        }
         __syncwarp();
     }
-    __device__ __forceinline__ void seed_from(float lm) {
-        const float t = top8_seed(lm);
-        st.theta = t;
-        st.th = fmaxf(st.th, t);
+    // CTA-collective: with lm the max of this thread's vectors, the 8th
+    // largest thread maximum is a value that 8 distinct elements reach, so
+    // nothing below it can be in the top 8.
+    __device__ __forceinline__ void seed_from(float lm, Pass1Smem& sm) {
+        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+        uint64_t l[8];
+        l[0] = lm > -INFINITY ? ((static_cast<uint64_t>(ord32(lm)) << 32) | threadIdx.x) : 0ull;
+#pragma unroll
+        for (int s2 = 1; s2 < 8; ++s2) l[s2] = 0ull;
+        const uint64_t wk = warp_top8(l);
+        if (lane < 8) sm.stage[w * 8 + lane] = wk;
+        __syncthreads();
+        if (w == 0) {
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) l[s2] = lane < NWARPS ? sm.stage[lane * 8 + s2] : 0ull;
+            const uint64_t k8 = __shfl_sync(FULL_MASK, warp_top8(l), 7);
+            if (lane == 0) sm.seed_theta = k8 != 0ull ? key_value(k8) : -INFINITY;
+        }
+        __syncthreads();
+        st.theta = sm.seed_theta;
+        st.th = fmaxf(st.th, st.theta);
     }
     __device__ __forceinline__ void vec(const uint4& w, int base, bool ok, Pass1Smem& sm) {
         const float m = ok ? VecOps<Tag, VEC>::vmax(w) : __uint_as_float(0x7fc00000u);
@@ -375,60 +391,75 @@ struct Top8Reducer {
                                     sm.cand[wp]);
         }
     }
-    __device__ __forceinline__ void end(int64_t r, uint64_t slot, const Pass1Params& P, Pass1Smem& sm) {
+    // Each warp stores 8 keys that include its best 8 of the chunk: its
+    // buffered candidates as they are when no more than 8 and never merged,
+    // else its merged best 8.  On a row's first sub-chunk the CTA also takes
+    // the chunk's 8th best (CTA-collective) to raise the row's shared
+    // threshold for the row's later chunks.
+    __device__ __forceinline__ void end(int64_t r, int sub, uint64_t chunk, const Pass1Params& P, Pass1Smem& sm) {
         const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-        if (st.cnt > 0) st = top8_merge(st, sm.wtop[wp], sm.cand[wp]);
+        if (st.merged || st.cnt > 8) st = top8_merge(st, sm.wtop[wp], sm.cand[wp]);
         __syncwarp();
-        if (lane < 8) static_cast<uint64_t*>(P.partials)[slot * 8 + lane] = sm.wtop[wp][lane];
-        const uint64_t k7 = sm.wtop[wp][7];
-        if (lane == 0 && k7 != 0ull && r < kThetaRows) atomicMax(&P.theta_row[r], static_cast<unsigned>(k7 >> 32));
+        uint64_t mine = 0ull;
+        if (lane < 8) mine = st.merged ? sm.wtop[wp][lane] : (lane < st.cnt ? sm.cand[wp][lane] : 0ull);
+        if (lane < 8) static_cast<uint64_t*>(P.partials)[(chunk * NWARPS + wp) * 8 + lane] = mine;
+        if (sub != 0 || r >= kThetaRows) return;
+        if (lane < 8) sm.stage[wp * 8 + lane] = mine;
+        __syncthreads();
+        if (wp == 0) {
+            uint64_t l[8];
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) l[s2] = 0ull;
+            for (int i = lane; i < NWARPS * 8; i += 32) {
+                const uint64_t kk = sm.stage[i];
+                if (kk > l[7]) top8_insert(l, kk);
+            }
+            const uint64_t k7 = __shfl_sync(FULL_MASK, warp_top8(l), 7);
+            if (lane == 0 && k7 != 0ull) atomicMax(&P.theta_row[r], static_cast<unsigned>(k7 >> 32));
+        }
     }
 };
 
-// Softmax statistics: running max M of the raw logits and S = sum
-// exp((l - M)/T), fp32 exp and sum within a vector, fp64 across vectors; the
-// warp's lanes are merged at the end of the chunk.
+// Softmax statistics of a chunk: its max M of the raw logits (NaN ignored),
+// then S = sum exp((l - M)/T) over the chunk, fp32 exp and sum within a
+// vector, fp64 across vectors and threads.  The chunk's elements are held in
+// registers, so the max is known before any exp is taken and no rescaling
+// is needed.  One (M, S) partial per chunk.
 template <class Tag, int VEC>
 struct SoftmaxReducer {
-    float M;
-    double S;
     float invT;
     double invT_d;
-    __device__ __forceinline__ void begin(int64_t, const Pass1Params&, Pass1Smem&) {
-        M = -FLT_MAX;
-        S = 0.0;
+    __device__ __forceinline__ void begin(int64_t, const Pass1Params&, Pass1Smem&) {}
+    // CTA-collective: max of the chunk.
+    __device__ __forceinline__ float chunk_max(float m, Pass1Smem& sm) {
+        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, o));
+        float* red = reinterpret_cast<float*>(sm.red);
+        if (lane == 0) red[w] = m;
+        __syncthreads();
+        float r = red[0];
+#pragma unroll
+        for (int i = 1; i < NWARPS; ++i) r = fmaxf(r, red[i]);
+        __syncthreads();
+        return r;
     }
-    __device__ __forceinline__ void vec(const uint4& w, int, bool ok, Pass1Smem&) {
-        if (!ok) return;
-        const float m = VecOps<Tag, VEC>::vmax(w);
-        if (m > M) {
-            S *= exp((static_cast<double>(M) - static_cast<double>(m)) * invT_d);
-            M = m;
-        }
+    __device__ __forceinline__ double vec_sum(const uint4& w, bool ok, float M) const {
+        if (!ok) return 0.0;
         float s = 0.0f;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) s += expf((VecOps<Tag, VEC>::elem(w, e) - M) * invT);
-        S += static_cast<double>(s);
+        return static_cast<double>(s);
     }
-    __device__ __forceinline__ void scalar(float v, int, bool ok, Pass1Smem&) {
-        if (!ok) return;
-        if (v > M) {
-            S *= exp((static_cast<double>(M) - static_cast<double>(v)) * invT_d);
-            M = v;
-        }
-        S += static_cast<double>(expf((v - M) * invT));
-    }
-    __device__ __forceinline__ void end(int64_t, uint64_t slot, const Pass1Params& P, Pass1Smem&) {
-        MaxSum acc;
-        acc.M = M;
-        acc.S = S;
-        acc = warp_maxsum(acc, invT_d);
-        if ((threadIdx.x & 31) == 0) {
+    // CTA-collective: store (M, S) of the chunk.
+    __device__ __forceinline__ void store(float M, double S, uint64_t chunk, const Pass1Params& P, Pass1Smem& sm) {
+        const double tot = block_sum_f64(S, reinterpret_cast<double*>(sm.red));
+        if (threadIdx.x == 0) {
             SoftmaxPartial sp;
-            sp.M = acc.M;
+            sp.M = M;
             sp.pad = 0.0f;
-            sp.S = acc.S;
-            static_cast<SoftmaxPartial*>(P.partials)[slot] = sp;
+            sp.S = tot;
+            static_cast<SoftmaxPartial*>(P.partials)[chunk] = sp;
         }
     }
 };
@@ -437,7 +468,6 @@ template <class Tag, int VEC, int MODE> struct ReducerFor;
 template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_ARGMAX> { using type = ArgmaxReducer<Tag, VEC>; };
 template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_TREE> { using type = ArgmaxReducer<Tag, VEC>; };
 template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_TOP8> { using type = Top8Reducer<Tag, VEC>; };
-template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_SOFTMAX> { using type = SoftmaxReducer<Tag, VEC>; };
 
 // ---------------------------------------------------------------------------
 // Row merges for the epilogues: warp-collective, over the row's cpr * NWARPS
@@ -445,26 +475,47 @@ template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_SOFTMAX> { using 
 // fewer than 8 elements above NaN (top-8) is rescanned exactly, element by
 // element, so NaN and -inf rank correctly.
 // ---------------------------------------------------------------------------
+// Merge the argmax partials of rows r0 .. r0+n-1 into keys[0..n) (shared
+// memory): warp w takes rows w, w+8, ..., four rows at a time with all their
+// loads in flight together.  Rows with no element above -inf are rescanned
+// exactly.  CTA-collective; keys are valid for every thread on return.
 template <class Tag>
-__device__ uint64_t row_argmax_key(const Pass1Params& P, int64_t r) {
-    const int lane = threadIdx.x & 31;
+__device__ void merge_argmax_rows(const Pass1Params& P, int64_t r0, int n, uint64_t* keys) {
+    constexpr int ROWB = 4;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const int np = P.cpr * NWARPS;
-    const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r * np;
-    uint64_t best = 0ull;
-    for (int i = lane; i < np; i += 32) {
-        const uint64_t kk = __ldcg(p + i);
-        best = kk > best ? kk : best;
-    }
-    best = warp_max_u64(best);
-    if (best == 0ull) {
-        const typename Tag::storage* row = static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride;
-        for (int x = lane; x < P.V; x += 32) {
-            const uint64_t kk = make_key(load_scalar<Tag>(row + x), x);
-            best = kk > best ? kk : best;
+    const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r0 * np;
+    for (int t0 = wp; t0 < n; t0 += NWARPS * ROWB) {
+        uint64_t best[ROWB];
+#pragma unroll
+        for (int q = 0; q < ROWB; ++q) best[q] = 0ull;
+        for (int i = lane; i < np; i += 32) {
+            uint64_t kk[ROWB];
+#pragma unroll
+            for (int q = 0; q < ROWB; ++q) {
+                const int t = t0 + q * NWARPS;
+                kk[q] = t < n ? __ldcg(p + static_cast<int64_t>(t) * np + i) : 0ull;
+            }
+#pragma unroll
+            for (int q = 0; q < ROWB; ++q) best[q] = kk[q] > best[q] ? kk[q] : best[q];
         }
-        best = warp_max_u64(best);
+#pragma unroll
+        for (int q = 0; q < ROWB; ++q) {
+            const int t = t0 + q * NWARPS;
+            uint64_t b = warp_max_u64(best[q]);
+            if (t < n && b == 0ull) {  // no element above -inf: exact rescan
+                const typename Tag::storage* row =
+                    static_cast<const typename Tag::storage*>(P.logits) + (r0 + t) * P.row_stride;
+                for (int x = lane; x < P.V; x += 32) {
+                    const uint64_t kx = make_key(load_scalar<Tag>(row + x), x);
+                    b = kx > b ? kx : b;
+                }
+                b = warp_max_u64(b);
+            }
+            if (t < n && lane == 0) keys[t] = b;
+        }
     }
-    return best;
+    __syncthreads();
 }
 
 // Lane e (< 8) returns the row's e-th best key.
@@ -502,7 +553,11 @@ __device__ void epilogue_greedy(const Pass1Params& P, int64_t b, Pass1Smem& sm) 
     const int k = P.k;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     if (threadIdx.x < k) sm.drafts[threadIdx.x] = P.drafts[b * k + threadIdx.x];
-    for (int t = wp; t <= k; t += NWARPS) {
+    if constexpr (MODE != MODE_TOP8) {
+        merge_argmax_rows<Tag>(P, b * (k + 1), k + 1, sm.rowkey);
+        if (threadIdx.x <= k) sm.am[threadIdx.x] = key_index(sm.rowkey[threadIdx.x]);
+    }
+    for (int t = wp; t <= k && MODE == MODE_TOP8; t += NWARPS) {
         const int64_t r = b * (k + 1) + t;
         if constexpr (MODE == MODE_TOP8) {
             const uint64_t mine = row_top8_key<Tag>(P, r);
@@ -519,9 +574,6 @@ __device__ void epilogue_greedy(const Pass1Params& P, int64_t b, Pass1Smem& sm) 
                 P.topk_vals[r * P.topk + lane] = val;
             }
             if (lane == 0 && r < kThetaRows) P.theta_row[r] = 0u;
-        } else {
-            const uint64_t key = row_argmax_key<Tag>(P, r);
-            if (lane == 0) sm.am[t] = key_index(key);
         }
     }
     __syncthreads();
@@ -548,15 +600,12 @@ __device__ void epilogue_tree(const Pass1Params& P, int64_t b, Pass1SmemTree& sm
     TreeArrays& ts = sm.t;
     const int n1 = P.rows_per_req;
     const int md = P.max_depth;
-    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     for (int c = threadIdx.x; c < n1; c += NT) {
         ts.par[c] = P.parents[b * n1 + c];
         ts.tok[c] = P.node_tokens[b * n1 + c];
     }
-    for (int c = wp; c < n1; c += NWARPS) {
-        const uint64_t key = row_argmax_key<Tag>(P, b * n1 + c);
-        if (lane == 0) ts.am[c] = key_index(key);
-    }
+    merge_argmax_rows<Tag>(P, b * n1, n1, ts.key);
+    for (int c = threadIdx.x; c < n1; c += NT) ts.am[c] = key_index(ts.key[c]);
     __syncthreads();
     int bad = 0;
     for (int c = threadIdx.x; c < n1; c += NT) {
@@ -645,7 +694,7 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     for (int t = wp; t <= k; t += NWARPS) {
         const int64_t r = b * (k + 1) + t;
-        const int np = P.cpr * NWARPS;
+        const int np = P.cpr;
         const SoftmaxPartial* p = static_cast<const SoftmaxPartial*>(P.partials) + r * np;
         MaxSum acc;
         acc.M = -FLT_MAX;
@@ -721,8 +770,55 @@ __device__ __forceinline__ void run_epilogue(const Pass1Params& P, int64_t b, Sm
     if constexpr (MODE == MODE_TREE) epilogue_tree<Tag>(P, b, sm);
     else if constexpr (MODE == MODE_SOFTMAX) epilogue_rejection<Tag>(P, b, sm);
     else epilogue_greedy<Tag, MODE>(P, b, sm);
-    if (threadIdx.x == 0) P.tickets[b] = 0u;
-    __syncthreads();
+}
+
+// Softmax statistics of one chunk (the rejection pass): the thread's vectors
+// stay in registers between the max and the exp-sum passes.
+template <class Tag, int VEC, int CH, int UPT>
+__device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typename Tag::storage* row, int64_t r,
+                                              int sub, int cnt, Pass1Smem& sm) {
+    SoftmaxReducer<Tag, VEC> red;
+    red.invT = P.invT;
+    red.invT_d = P.invT_d;
+    constexpr int KEEP = UPT <= 16 ? UPT : 16;  // vectors kept in registers per batch
+    float m = -FLT_MAX;
+    uint4 w[KEEP];
+    // The ragged row end (fewer than VEC elements) goes to lanes of warp 0.
+    const int tx = P.nv_full * VEC + static_cast<int>(threadIdx.x);
+    const bool has_tail = sub == P.cpr - 1 && threadIdx.x < 32 && tx < P.V;
+    const float tail = has_tail ? load_scalar<Tag>(row + tx) : -FLT_MAX;
+    if constexpr (UPT <= KEEP) {
+#pragma unroll
+        for (int u = 0; u < UPT; ++u) {
+            const int i = u * NT + static_cast<int>(threadIdx.x);
+            w[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < cnt) {
+                RowLoader<Tag, VEC>::raw(row, sub * CH + i, w[u]);
+                m = fmaxf(m, VecOps<Tag, VEC>::vmax(w[u]));
+            }
+        }
+    } else {
+        for (int i = static_cast<int>(threadIdx.x); i < cnt; i += NT) {
+            uint4 x;
+            RowLoader<Tag, VEC>::raw(row, sub * CH + i, x);
+            m = fmaxf(m, VecOps<Tag, VEC>::vmax(x));
+        }
+    }
+    if (has_tail) m = fmaxf(m, tail);
+    const float M = red.chunk_max(m, sm);
+    double S = 0.0;
+    if constexpr (UPT <= KEEP) {
+#pragma unroll
+        for (int u = 0; u < UPT; ++u) S += red.vec_sum(w[u], u * NT + static_cast<int>(threadIdx.x) < cnt, M);
+    } else {
+        for (int i = static_cast<int>(threadIdx.x); i < cnt; i += NT) {
+            uint4 x;
+            RowLoader<Tag, VEC>::raw(row, sub * CH + i, x);
+            S += red.vec_sum(x, true, M);
+        }
+    }
+    if (has_tail) S += static_cast<double>(expf((tail - M) * P.invT));
+    red.store(M, S, static_cast<uint64_t>(r) * P.cpr + sub, P, sm);
 }
 
 // ---------------------------------------------------------------------------
@@ -733,7 +829,7 @@ __device__ __forceinline__ void run_epilogue(const Pass1Params& P, int64_t b, Sm
 // per thread), then its warp reduces.
 // ---------------------------------------------------------------------------
 template <class Tag, int VEC, int MODE>
-__global__ void __launch_bounds__(NT) verify_pass1_kernel(const Pass1Params P) {
+__global__ void __launch_bounds__(NT, MODE == MODE_TOP8 ? 4 : 1) verify_pass1_kernel(const Pass1Params P) {
     __shared__ typename SmemFor<MODE>::type sm;
     using Elem = typename Tag::storage;
     constexpr int CH = chunk_vecs(VEC);  // vectors per chunk
@@ -744,21 +840,19 @@ __global__ void __launch_bounds__(NT) verify_pass1_kernel(const Pass1Params P) {
     grid_dependency_wait();
     grid_launch_dependents();
 
-    // Chunk c: row c % R, sub-chunk c / R (vectors [sub*CH, ...)).
-    const uint64_t c = blockIdx.x;
-    const uint64_t R = static_cast<uint64_t>(P.R);
-    const int64_t r = static_cast<int64_t>(c % R);
-    const int sub = static_cast<int>(c / R);
+    // Chunk (row blockIdx.x, sub-chunk blockIdx.y): vectors [sub*CH, ...) of
+    // the row.  x varies fastest, so all rows' first chunks are scheduled
+    // before their second ones.
+    const int64_t r = blockIdx.x;
+    const int sub = static_cast<int>(blockIdx.y);
     int cnt = P.nv_full - sub * CH;
     cnt = cnt < CH ? cnt : CH;  // may be <= 0: only the ragged row end
     const Elem* row = static_cast<const Elem*>(P.logits) + r * P.row_stride;
 
-    typename ReducerFor<Tag, VEC, MODE>::type red;
     if constexpr (MODE == MODE_SOFTMAX) {
-        red.invT = P.invT;
-        red.invT_d = P.invT_d;
-    }
-    red.begin(r, P, sm);
+        softmax_chunk<Tag, VEC, CH, UPT>(P, row, r, sub, cnt, sm);
+    } else {
+    typename ReducerFor<Tag, VEC, MODE>::type red;
     for (int u0 = 0; u0 < UPT; u0 += BATCH) {
         uint4 w[BATCH];
 #pragma unroll
@@ -767,13 +861,14 @@ __global__ void __launch_bounds__(NT) verify_pass1_kernel(const Pass1Params P) {
             w[u] = make_uint4(0u, 0u, 0u, 0u);
             if (i < cnt) RowLoader<Tag, VEC>::raw(row, sub * CH + i, w[u]);
         }
+        if (u0 == 0) red.begin(r, sub, P, sm);  // after the loads are in flight (top-8 reads the row threshold)
         if constexpr (MODE == MODE_TOP8) {
             if (u0 == 0 && red.seed) {
                 float lm = -INFINITY;
 #pragma unroll
                 for (int u = 0; u < BATCH; ++u)
                     if (u * NT + static_cast<int>(threadIdx.x) < cnt) lm = fmaxf(lm, VecOps<Tag, VEC>::vmax(w[u]));
-                red.seed_from(lm);
+                red.seed_from(lm, sm);
             }
         }
 #pragma unroll
@@ -789,17 +884,17 @@ __global__ void __launch_bounds__(NT) verify_pass1_kernel(const Pass1Params P) {
             red.scalar(ok ? load_scalar<Tag>(row + x) : 0.0f, x, ok, sm);
         }
     }
-    red.end(r, (static_cast<uint64_t>(r) * P.cpr + sub) * NWARPS + wp, P, sm);
-
-    // Ticket for the request; the CTA that completes it runs the epilogue.
-    __syncthreads();
-    const int64_t b = r / P.rows_per_req;
-    if (threadIdx.x == 0) {
-        const unsigned need = static_cast<unsigned>(P.rows_per_req * P.cpr);
-        sm.epi_req = ticket_add(&P.tickets[b]) + 1u == need ? 1 : 0;
+    red.end(r, sub, static_cast<uint64_t>(r) * P.cpr + sub, P, sm);
     }
-    __syncthreads();
-    if (sm.epi_req) run_epilogue<Tag, MODE>(P, b, sm);
+}
+
+// Request epilogues as their own kernel (one CTA per request), after the pass.
+template <class Tag, int MODE>
+__global__ void __launch_bounds__(NT) verify_epilogue_kernel(const Pass1Params P) {
+    __shared__ typename SmemFor<MODE>::type sm;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    run_epilogue<Tag, MODE>(P, blockIdx.x, sm);
 }
 
 }  // namespace specdec
