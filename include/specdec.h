@@ -46,9 +46,9 @@
  *     below -inf and -0 equals +0.  bf16 logits are widened exactly.
  *   - The workspace is caller-owned device memory of at least
  *     specdec_workspace_size() bytes, zeroed once by specdec_workspace_init().
- *     Every call leaves its counters at zero again, so one workspace serves
- *     any sequence of calls of any mode and shape that fits its size,
- *     including CUDA-graph replays.  Calls that may overlap on the GPU (other
+ *     Every call leaves its shared top-8 thresholds at zero again, so one
+ *     workspace serves any sequence of calls of any mode and shape that fits
+ *     its size, including CUDA-graph replays.  Calls that may overlap on the GPU (other
  *     streams) must use different workspaces.
  *
  * Limits: 0 <= B <= SPECDEC_MAX_B; 0 <= k <= SPECDEC_MAX_K; 1 <= V <=
@@ -186,7 +186,7 @@ specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int6
  *     (cudaGetSymbolAddress, with the device current); make that first call
  *     before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents;
- *     each call clears the counters it needs on `stream` first.  Calls that
+ *     a top-8 call clears its threshold words on `stream` first.  Calls that
  *     may overlap on the GPU (other streams, other threads) race: serialise
  *     them or use specdec_verify_greedy with separate workspaces.
  *   - A call whose workspace need (specdec_workspace_size) exceeds

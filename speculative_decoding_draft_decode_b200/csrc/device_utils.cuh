@@ -5,9 +5,11 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "geometry.h"
+
 namespace specdec {
 
-constexpr int NT = 256;               // threads per CTA
+constexpr int NT = kThreads;          // threads per CTA
 constexpr int NWARPS = NT / 32;
 constexpr unsigned FULL_MASK = 0xffffffffu;
 

@@ -1,13 +1,18 @@
-// geometry.h — how a verify pass splits its rows across CTAs.
+// geometry.h — how the verify kernels cut a logit row into chunks.
 //
-// Every logit row is cut into "vectors" (16 bytes: 8 bf16 or 4 fp32 values;
-// one element on the unaligned scalar path).  The rows of one call are laid
-// end to end into a flat vector space [0, T), T = rows * vectors_per_row, and
-// CTA c of G takes the contiguous range [c*T/G, (c+1)*T/G).  Every CTA
-// therefore streams the same number of bytes (within one vector), however
-// the rows fall; a CTA range may cover the tail of one row and the head of
-// the next.  The per-row pieces ("segments") are reduced per CTA and the
-// partial results stored in slot (row, c - first_cta(row)).
+// A row of V elements is read as nv_full = V / vec full 16-byte vectors
+// (vec = 8 bf16 or 4 fp32 values; vec = 1 on the unaligned scalar path) and
+// a ragged end of V - nv_full * vec < vec elements.  The vectors are grouped
+// into chunks of chunk_vecs(vec); chunk s of a row holds vectors
+// [s * CH, min((s + 1) * CH, nv_full)), and the row's last chunk also owns
+// the ragged end.  One CTA of kThreads threads handles one chunk.
+//
+// Two orders of the chunk's vectors over the CTA's threads:
+//   streaming  thread t takes vectors s*CH + u*kThreads + t, u = 0..UPT-1, so
+//              each load instruction of a warp covers 32 consecutive vectors;
+//   rescan     thread t takes vectors s*CH + t*UPT + u, so that each thread's
+//              elements are consecutive and thread order is index order (the
+//              inverse-CDF search of the resample needs index order).
 //
 // Plain C++ so that the host launcher, the device code and a CPU test share
 // the same definition.
@@ -21,30 +26,39 @@
 #define SPECDEC_HD inline
 #endif
 
+#ifndef SPECDEC_PIPE_U
+#define SPECDEC_PIPE_U 8
+#endif
+
 namespace specdec {
 
-// First vector of CTA c (c = G gives T).
-SPECDEC_HD int64_t part_begin(int64_t c, int64_t T, int64_t G) { return (c * T) / G; }
+constexpr int kThreads = 256;                  // threads per CTA
+constexpr int kU = SPECDEC_PIPE_U;             // 16-byte loads in flight per thread
+constexpr int kChunk = kU * kThreads;          // vectors per chunk (vector path)
 
-// The CTA whose range holds vector v: the largest c with part_begin(c) <= v.
-SPECDEC_HD int64_t cta_of(int64_t v, int64_t T, int64_t G) { return ((v + 1) * G - 1) / T; }
+// Vectors per chunk: the scalar path (one element per "vector") takes 8x as
+// many, so that a chunk covers as many elements as on the vector path.
+SPECDEC_HD constexpr int chunk_vecs(int vec) { return vec > 1 ? kChunk : kChunk * 8; }
 
-// Upper bound on the CTAs whose ranges meet one run of `len` consecutive
-// vectors, when every range holds at least floor(T/G) vectors.
-SPECDEC_HD int64_t slots_bound(int64_t len, int64_t T, int64_t G) {
-    int64_t lmin = G > 0 ? T / G : T;
-    if (lmin < 1) lmin = 1;
-    return (len + lmin - 1) / lmin + 1;
+// Vectors of a chunk per thread.
+SPECDEC_HD constexpr int chunk_upt(int vec) { return chunk_vecs(vec) / kThreads; }
+
+// Chunks per row for rows of nv_full full vectors (at least one: a row
+// shorter than one vector is all ragged end).
+SPECDEC_HD int64_t chunks_per_row(int64_t nv_full, int vec) {
+    return nv_full > 0 ? (nv_full + chunk_vecs(vec) - 1) / chunk_vecs(vec) : 1;
 }
 
-// Largest grid a pass over T vectors may use: at least `min_vecs` vectors per
-// CTA, at most `g_cap` CTAs, never more CTAs than vectors.
-SPECDEC_HD int64_t grid_upper(int64_t T, int64_t min_vecs, int64_t g_cap) {
-    int64_t g = T / min_vecs;
-    if (g < 1) g = 1;
-    if (g > g_cap) g = g_cap;
-    if (g > T) g = T;
-    return g;
+// Full vectors in chunk `sub` (0 for a chunk that holds only the ragged end).
+SPECDEC_HD int chunk_count(int nv_full, int sub, int vec) {
+    const int c = nv_full - sub * chunk_vecs(vec);
+    return c < 0 ? 0 : (c < chunk_vecs(vec) ? c : chunk_vecs(vec));
 }
+
+// Position within the chunk of thread t's u-th vector, streaming order.
+SPECDEC_HD int stream_pos(int u, int t) { return u * kThreads + t; }
+
+// Position within the chunk of thread t's u-th vector, rescan order.
+SPECDEC_HD int rescan_pos(int u, int t, int vec) { return t * chunk_upt(vec) + u; }
 
 }  // namespace specdec

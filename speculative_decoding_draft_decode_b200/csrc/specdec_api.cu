@@ -1,14 +1,12 @@
 // specdec_api.cu — the C-ABI (include/specdec.h): argument checks, workspace
 // layout, grid sizing and kernel launches.
 //
-// Workspace layout (byte offsets).  Everything that must be zero when a call
-// starts sits at a fixed place, so a workspace initialised once serves calls
+// Workspace layout (byte offsets).  The words that must be zero when a call
+// starts sit at a fixed place, so a workspace initialised once serves calls
 // of any shape; each call returns those words to zero before it ends.
-//   [0, 256 KiB)            pass-1 tickets, one 32-bit word per request
-//   [256 KiB, 512 KiB)      pass-2 tickets (rejection resample)
-//   [512 KiB, 768 KiB)      top-8 thresholds, one word per row (first 65536 rows)
-//   then                    pass-1 partials, one slot per (chunk, warp)
-//   then (rejection only)   per-request RejState, per-unit masses of row h
+//   [0, 256 KiB)            top-8 thresholds, one word per row (first 65536 rows)
+//   then                    streaming-pass partials, one slot per chunk
+//   then (rejection only)   per-request RejState, per-chunk masses of row h
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -17,25 +15,20 @@
 #include <atomic>
 
 #include "../../include/specdec.h"
-#include "geometry.h"
 #include "verify_pass1.cuh"
 #include "verify_resample.cuh"
 
 namespace specdec {
 namespace {
 
-constexpr size_t kTicketBytes = static_cast<size_t>(SPECDEC_MAX_B) * sizeof(unsigned);
-constexpr size_t kThetaBase = 2 * kTicketBytes;
+constexpr size_t kThetaBase = 0;
 constexpr size_t kPartialBase = kThetaBase + static_cast<size_t>(kThetaRows) * sizeof(unsigned);
-constexpr int64_t kMinUnitsPerCta = 4;    // resample pass: 32-vector units
-constexpr int64_t kGridCap = 4096;        // largest grid any pass uses
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
     int64_t nv = 0, nv_full = 0, cpr = 0, NC = 0;
-    int64_t nu = 0, T2 = 0;
-    size_t partials1 = 0, state = 0, units = 0, total = 0;
+    size_t partials1 = 0, state = 0, masses = 0, total = 0;
 };
 
 // Layout of one call.  `vec` = elements per vector (1 on the scalar path),
@@ -53,10 +46,8 @@ Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t
     if (rejection) {
         L.state = align_up(end, 256);
         end = L.state + static_cast<size_t>(B) * sizeof(RejState);
-        L.nu = (L.nv + kUnitVecs - 1) / kUnitVecs;
-        L.T2 = static_cast<int64_t>(B) * L.nu;
-        L.units = align_up(end, 256);
-        end = L.units + static_cast<size_t>(L.T2) * sizeof(double2);
+        L.masses = align_up(end, 256);
+        end = L.masses + static_cast<size_t>(B) * static_cast<size_t>(L.cpr) * sizeof(double2);
     }
     (void)rows_per_req;
     L.total = align_up(end, 256);
@@ -66,42 +57,7 @@ Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t
 int elem_size(specdec_dtype dt) { return dt == SPECDEC_BF16 ? 2 : 4; }
 int vec_elems(specdec_dtype dt) { return dt == SPECDEC_BF16 ? 8 : 4; }
 
-// Cached per (device, kernel) resident-CTA counts.
 constexpr int kMaxDevices = 64;
-constexpr int kNumKernels = 32;
-std::atomic<int> g_sms[kMaxDevices];
-std::atomic<int> g_occ[kMaxDevices][kNumKernels];
-
-// Resident CTAs of `fn` on the current device (cached), after allowing it
-// `dyn_smem` bytes of dynamic shared memory.
-cudaError_t grid_cap(const void* fn, int kernel_id, int dyn_smem, int64_t* cap) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) dev = kMaxDevices - 1;
-    int sms = g_sms[dev].load(std::memory_order_relaxed);
-    if (sms == 0) {
-        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-        g_sms[dev].store(sms, std::memory_order_relaxed);
-    }
-    int occ = g_occ[dev][kernel_id].load(std::memory_order_relaxed);
-    if (occ == 0) {
-        if (dyn_smem > 0) {
-            e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
-            if (e != cudaSuccess) return e;
-        }
-        e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, NT, dyn_smem);
-        if (e != cudaSuccess) return e;
-        if (occ < 1) occ = 1;
-        g_occ[dev][kernel_id].store(occ, std::memory_order_relaxed);
-    }
-    *cap = static_cast<int64_t>(sms) * occ;
-    if (*cap > kGridCap) *cap = kGridCap;
-    return cudaSuccess;
-}
 
 bool vector_path_ok(const void* p, int64_t stride, int esize) {
     return (reinterpret_cast<uintptr_t>(p) % 16 == 0) && ((stride * esize) % 16 == 0);
@@ -144,14 +100,16 @@ specdec_status launch_pass1(Pass1Params P, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 
+// The chunk masses of row h (one CTA per chunk), then the token search (one
+// CTA per request).
 template <class Tag, int VEC>
 specdec_status launch_pass2(Pass2Params P, cudaStream_t stream) {
-    auto fn = verify_resample_kernel<Tag, VEC>;
-    const int kid = 16 + (VEC == 1 ? 0 : 1) * 2 + (sizeof(typename Tag::storage) == 2 ? 1 : 0);
-    int64_t cap = 0;
-    if (grid_cap(reinterpret_cast<const void*>(fn), kid, 0, &cap) != cudaSuccess) return SPECDEC_ERR_CUDA;
-    const int64_t G = grid_upper(P.T, kMinUnitsPerCta, cap);
-    if (launch_pdl(fn, dim3(static_cast<unsigned>(G)), 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    if (P.cpr > 65535) return SPECDEC_ERR_UNSUPPORTED;  // grid limit
+    const dim3 grid(static_cast<unsigned>(P.B), static_cast<unsigned>(P.cpr));
+    if (launch_pdl(verify_resample_kernel<Tag, VEC>, grid, 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    if (launch_pdl(verify_resample_epilogue_kernel<Tag, VEC>, dim3(static_cast<unsigned>(P.B)), 0, stream, P) !=
+        cudaSuccess)
+        return SPECDEC_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 
@@ -363,18 +321,15 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
     Q.q = draft_probs;
     Q.q_stride = q_row_stride;
     Q.V = V;
-    Q.nv = static_cast<int>(L.nv);
-    Q.nv_full = V / ve;
-    Q.nu = static_cast<int>(L.nu);
-    Q.T = L.T2;
+    Q.nv_full = static_cast<int>(L.nv_full);
+    Q.cpr = static_cast<int>(L.cpr);
     Q.B = B;
     Q.k = k;
     Q.invT = static_cast<float>(invT_d);
     Q.seed = seed;
     Q.offset = offset;
     Q.state = state;
-    Q.tickets = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kTicketBytes);
-    Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
+    Q.chunk_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.masses);
     Q.out_tokens = out_tokens;
     return dispatch_pass2(dtype, vec, Q, s);
 }
@@ -431,11 +386,17 @@ extern "C" specdec_status specdec_verify_greedy_static_scratch(
     void* scratch = nullptr;
     if (B > 0 && need > 0) {
         if (specdec::static_scratch_address(&scratch) != cudaSuccess) return SPECDEC_ERR_CUDA;
-        // The request counters must start at zero; the array keeps whatever
-        // the previous call left, so clear this call's counters first.
-        if (cudaMemsetAsync(scratch, 0, static_cast<size_t>(B) * sizeof(unsigned),
-                            reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-            return SPECDEC_ERR_CUDA;
+        // The top-8 row thresholds must start at zero.  Every completed call
+        // leaves them so, but the array keeps whatever a call that failed
+        // half-way left: clear this call's words first.
+        if (topk > 0 && k >= 0 && k <= SPECDEC_MAX_K) {
+            int64_t rows = static_cast<int64_t>(B) * (k + 1);
+            if (rows > specdec::kThetaRows) rows = specdec::kThetaRows;
+            if (cudaMemsetAsync(static_cast<char*>(scratch) + specdec::kThetaBase, 0,
+                                static_cast<size_t>(rows) * sizeof(unsigned),
+                                reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+                return SPECDEC_ERR_CUDA;
+        }
     }
     return specdec_verify_greedy(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len, out_tokens, topk,
                                  topk_ids, topk_vals, scratch, scratch ? SPECDEC_STATIC_SCRATCH_BYTES : 0, stream);

@@ -46,19 +46,6 @@ constexpr int kThetaRows = 65536;   // rows with a shared top-8 threshold
 
 enum Pass1Mode { MODE_ARGMAX = 0, MODE_TOP8 = 1, MODE_TREE = 2, MODE_SOFTMAX = 3 };
 
-// Chunk shape: kU 16-byte vectors per thread (vector path).
-#ifndef SPECDEC_PIPE_U
-#define SPECDEC_PIPE_U 8
-#endif
-constexpr int kU = SPECDEC_PIPE_U;
-constexpr int kChunk = kU * NT;  // vectors per chunk
-// Vectors per chunk: the scalar path (one element per "vector") takes 8x as
-// many so that a chunk covers as many elements as on the vector path.
-__host__ __device__ constexpr int chunk_vecs(int vec) { return vec > 1 ? kChunk : kChunk * 8; }
-// Chunks per row for rows of nv_full full vectors.
-__host__ __device__ inline int64_t chunks_per_row(int64_t nv_full, int vec) {
-    return nv_full > 0 ? (nv_full + chunk_vecs(vec) - 1) / chunk_vecs(vec) : 1;
-}
 constexpr int kCandBuf = 64;  // top-8 candidate buffer per warp
 
 struct SoftmaxPartial {

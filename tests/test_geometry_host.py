@@ -1,8 +1,9 @@
-"""The even split of the flattened row space over CTAs (csrc/geometry.h),
-compiled for the host and checked exhaustively on small cases: the ranges
-tile [0, T) without gaps or overlaps, every CTA gets floor(T/G) or
-ceil(T/G) vectors, cta_of inverts the split, and slots_bound bounds the CTAs
-meeting any row."""
+"""The chunk geometry of the verify kernels (csrc/geometry.h), compiled for
+the host and checked exhaustively on small rows and at the largest ones: the
+chunks of a row, in streaming order and in rescan order, cover every full
+vector exactly once and nothing past the row; the ragged end (fewer than one
+vector) belongs to the last chunk; rescan order is index order over the
+threads; and no index overflows 32 bits at SPECDEC_MAX_V."""
 import os
 import subprocess
 
@@ -11,54 +12,66 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 DRIVER = r"""
 #include "geometry.h"
 #include <cstdio>
+#include <vector>
 #include <initializer_list>
 using namespace specdec;
+static long fails = 0, checks = 0;
+static void row_case(int V, int vec) {
+  const int nv_full = V / vec;
+  const int64_t cpr = chunks_per_row(nv_full, vec);
+  const int CH = chunk_vecs(vec), UPT = chunk_upt(vec);
+  if (UPT * kThreads != CH) ++fails;
+  std::vector<int> seen_s(nv_full, 0), seen_r(nv_full, 0);
+  int total = 0;
+  for (int sub = 0; sub < cpr; ++sub) {
+    const int cnt = chunk_count(nv_full, sub, vec);
+    if (cnt < 0 || cnt > CH) ++fails;
+    if (sub < cpr - 1 && cnt != CH) ++fails;   // only the last chunk is short
+    total += cnt;
+    int prev = -1;
+    for (int t = 0; t < kThreads; ++t)
+      for (int u = 0; u < UPT; ++u) {
+        const int is = stream_pos(u, t), ir = rescan_pos(u, t, vec);
+        if (is < 0 || is >= CH || ir < 0 || ir >= CH) ++fails;
+        if (is < cnt) { const int j = sub * CH + is; if (j >= nv_full) ++fails; else ++seen_s[j]; }
+        if (ir < cnt) {
+          const int j = sub * CH + ir;
+          if (j >= nv_full) ++fails; else ++seen_r[j];
+          if (j <= prev) ++fails;                  // thread-major order is index order
+          prev = j;
+        }
+      }
+  }
+  if (total != nv_full) ++fails;
+  for (int j = 0; j < nv_full; ++j) { ++checks; if (seen_s[j] != 1 || seen_r[j] != 1) ++fails; }
+  // the ragged end: fewer than one vector, one warp's lanes cover it
+  const int tail = V - nv_full * vec;
+  if (tail < 0 || tail >= vec + (vec == 1)) ++fails;
+  if (tail > 32) ++fails;
+}
 int main() {
-  long fails = 0, checks = 0;
-  for (int64_t nv = 1; nv <= 40; ++nv)
-  for (int64_t rows = 1; rows <= 30; ++rows) {
-    const int64_t T = rows * nv;
-    for (int64_t G = 1; G <= T && G <= 64; ++G) {
-      int64_t prev_end = 0;
-      for (int64_t c = 0; c < G; ++c) {
-        int64_t b = part_begin(c, T, G), e = part_begin(c + 1, T, G);
-        ++checks;
-        if (b != prev_end) ++fails;
-        if (e - b != T / G && e - b != (T + G - 1) / G) ++fails;
-        for (int64_t v = b; v < e; ++v) if (cta_of(v, T, G) != c) ++fails;
-        prev_end = e;
-      }
-      if (prev_end != T) ++fails;
-      const int64_t bound = slots_bound(nv, T, G);
-      for (int64_t r = 0; r < rows; ++r) {
-        int64_t n = cta_of(r * nv + nv - 1, T, G) - cta_of(r * nv, T, G) + 1;
-        if (n > bound) ++fails;
-      }
-      // a larger grid never needs fewer slots
-      if (G > 1 && slots_bound(nv, T, G - 1) > bound) ++fails;
-    }
+  for (int vec : {1, 4, 8}) {
+    for (int V = 1; V <= 3 * chunk_vecs(vec) * vec + 20; V += (V < 300 ? 1 : 997)) row_case(V, vec);
+    for (int V : {32000, 128256, 151936, 152064, 256000}) row_case(V, vec);
+    // the largest row: every element index stays below 2^31
+    const int64_t V = 1 << 24, nv_full = V / vec, cpr = chunks_per_row(nv_full, vec);
+    const int64_t last = ((cpr - 1) * chunk_vecs(vec) + chunk_vecs(vec) - 1) * vec + vec;
+    if (last >= (int64_t(1) << 31)) ++fails;
+    if (cpr > 65535) ++fails;                      // fits a grid dimension
   }
-  // large values do not overflow
-  const int64_t T = (int64_t)65536 * 33 * (1 << 21);
-  for (int64_t G : {1, 148, 4096}) {
-    if (part_begin(G, T, G) != T) ++fails;
-    if (cta_of(T - 1, T, G) != G - 1) ++fails;
-    if (cta_of(0, T, G) != 0) ++fails;
-  }
-  if (grid_upper(5000, 128, 4096) != 39 || grid_upper(10, 128, 4096) != 1 || grid_upper(1 << 30, 128, 1184) != 1184) ++fails;
   std::printf("%ld %ld\n", checks, fails);
   return fails != 0;
 }
 """
 
 
-def test_partition_properties(tmp_path):
+def test_chunk_geometry(tmp_path):
     src = tmp_path / "geom.cpp"
     src.write_text(DRIVER)
     exe = tmp_path / "geom"
     inc = os.path.join(ROOT, "speculative_decoding_draft_decode_b200", "csrc")
-    subprocess.run(["g++", "-std=c++17", "-O1", "-I", inc, str(src), "-o", str(exe)], check=True)
-    res = subprocess.run([str(exe)], capture_output=True, text=True)
+    subprocess.run(["g++", "-std=c++17", "-O2", "-I", inc, str(src), "-o", str(exe)], check=True)
+    res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
     checks, fails = map(int, res.stdout.split())
-    assert checks > 10000
+    assert checks > 100000
     assert fails == 0 and res.returncode == 0
