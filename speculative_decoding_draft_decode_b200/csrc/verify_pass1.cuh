@@ -505,18 +505,30 @@ __device__ void merge_argmax_rows(const Pass1Params& P, int64_t r0, int n, uint6
     __syncthreads();
 }
 
-// Lane e (< 8) returns the row's e-th best key.
+// Lane e (< 8) returns the row's e-th best key.  The row's shared threshold
+// (the largest 8th-best value any of its chunks published) bounds the row's
+// 8th best from below, so keys under it are skipped; each lane issues its
+// loads of a batch together.
 template <class Tag>
 __device__ uint64_t row_top8_key(const Pass1Params& P, int64_t r) {
+    constexpr int KB = 16;  // keys per lane per batch
     const int lane = threadIdx.x & 31;
     const int nk = P.cpr * NWARPS * 8;
     const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r * nk;
+    const uint64_t floor_key = r < kThetaRows ? static_cast<uint64_t>(__ldcg(&P.theta_row[r])) << 32 : 0ull;
     uint64_t l[8];
 #pragma unroll
     for (int s = 0; s < 8; ++s) l[s] = 0ull;
-    for (int i = lane; i < nk; i += 32) {
-        const uint64_t kk = __ldcg(p + i);
-        if (kk > l[7]) top8_insert(l, kk);
+    for (int i0 = 0; i0 < nk; i0 += 32 * KB) {
+        uint64_t kk[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            const int i = i0 + j * 32 + lane;
+            kk[j] = i < nk ? __ldcg(p + i) : 0ull;
+        }
+#pragma unroll
+        for (int j = 0; j < KB; ++j)
+            if (kk[j] >= floor_key && kk[j] > l[7]) top8_insert(l, kk[j]);
     }
     uint64_t mine = warp_top8(l);
     if (__shfl_sync(FULL_MASK, mine, 7) == 0ull) {
