@@ -121,6 +121,18 @@ struct Pass1SmemTree : Pass1Smem {
 template <int MODE> struct SmemFor { using type = Pass1Smem; };
 template <> struct SmemFor<MODE_TREE> { using type = Pass1SmemTree; };
 
+// The top-8 epilogue's shared lists: per row, the partial keys at or above
+// the row threshold (kSurv at most) and the merged 8 best.
+constexpr int kSurv = 64;
+struct Top8EpiSmem : Pass1Smem {
+    unsigned floor_ord[kMaxRowsPerReq];
+    int cnt[kMaxRowsPerReq];
+    uint64_t surv[kMaxRowsPerReq][kSurv];
+    uint64_t top[kMaxRowsPerReq][8];
+};
+template <int MODE> struct EpiSmemFor { using type = typename SmemFor<MODE>::type; };
+template <> struct EpiSmemFor<MODE_TOP8> { using type = Top8EpiSmem; };
+
 // ---------------------------------------------------------------------------
 // One 16-byte vector as loaded: its max (NaN ignored) and its elements.
 // bf16 vectors use packed bf16x2 max, three per 8 elements.
@@ -463,34 +475,43 @@ template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_TOP8> { using typ
 // element, so NaN and -inf rank correctly.
 // ---------------------------------------------------------------------------
 // Merge the argmax partials of rows r0 .. r0+n-1 into keys[0..n) (shared
-// memory): warp w takes rows w, w+8, ..., four rows at a time with all their
-// loads in flight together.  Rows with no element above -inf are rescanned
-// exactly.  CTA-collective; keys are valid for every thread on return.
+// memory): warp w takes rows w, w+8, ..., up to kRowB rows at a time, and
+// each lane issues the loads of all of them (kJB keys per row) before any
+// compare, so a request of up to 72 rows of up to 96 partials costs one
+// round trip.  Rows with no element above -inf are rescanned exactly.
+// CTA-collective; keys are valid for every thread on return.
 template <class Tag>
 __device__ void merge_argmax_rows(const Pass1Params& P, int64_t r0, int n, uint64_t* keys) {
-    constexpr int ROWB = 4;
+    constexpr int kRowB = 9, kJB = 3;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const int np = P.cpr * NWARPS;
     const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r0 * np;
-    for (int t0 = wp; t0 < n; t0 += NWARPS * ROWB) {
-        uint64_t best[ROWB];
+    for (int t0 = wp; t0 < n; t0 += NWARPS * kRowB) {
+        uint64_t best[kRowB];
 #pragma unroll
-        for (int q = 0; q < ROWB; ++q) best[q] = 0ull;
-        for (int i = lane; i < np; i += 32) {
-            uint64_t kk[ROWB];
+        for (int q = 0; q < kRowB; ++q) best[q] = 0ull;
+        for (int i0 = lane; i0 < np; i0 += 32 * kJB) {
+            uint64_t kk[kRowB][kJB];
 #pragma unroll
-            for (int q = 0; q < ROWB; ++q) {
+            for (int q = 0; q < kRowB; ++q) {
                 const int t = t0 + q * NWARPS;
-                kk[q] = t < n ? __ldcg(p + static_cast<int64_t>(t) * np + i) : 0ull;
+#pragma unroll
+                for (int j = 0; j < kJB; ++j) {
+                    const int i = i0 + 32 * j;
+                    kk[q][j] = (t < n && i < np) ? __ldcg(p + static_cast<int64_t>(t) * np + i) : 0ull;
+                }
             }
 #pragma unroll
-            for (int q = 0; q < ROWB; ++q) best[q] = kk[q] > best[q] ? kk[q] : best[q];
+            for (int q = 0; q < kRowB; ++q)
+#pragma unroll
+                for (int j = 0; j < kJB; ++j) best[q] = kk[q][j] > best[q] ? kk[q][j] : best[q];
         }
 #pragma unroll
-        for (int q = 0; q < ROWB; ++q) {
+        for (int q = 0; q < kRowB; ++q) {
             const int t = t0 + q * NWARPS;
+            if (t >= n) break;  // warp-uniform
             uint64_t b = warp_max_u64(best[q]);
-            if (t < n && b == 0ull) {  // no element above -inf: exact rescan
+            if (b == 0ull) {  // no element above -inf: exact rescan
                 const typename Tag::storage* row =
                     static_cast<const typename Tag::storage*>(P.logits) + (r0 + t) * P.row_stride;
                 for (int x = lane; x < P.V; x += 32) {
@@ -499,7 +520,7 @@ __device__ void merge_argmax_rows(const Pass1Params& P, int64_t r0, int n, uint6
                 }
                 b = warp_max_u64(b);
             }
-            if (t < n && lane == 0) keys[t] = b;
+            if (lane == 0) keys[t] = b;
         }
     }
     __syncthreads();
@@ -544,38 +565,104 @@ __device__ uint64_t row_top8_key(const Pass1Params& P, int64_t r) {
     return mine;
 }
 
-// ---------------------------------------------------------------------------
-// Request epilogues (every thread of the last-ticket CTA).
-// ---------------------------------------------------------------------------
-template <class Tag, int MODE>
-__device__ void epilogue_greedy(const Pass1Params& P, int64_t b, Pass1Smem& sm) {
-    const int k = P.k;
+// The 8 best keys of rows r0 .. r0+n-1 into sm.top (CTA-collective).  Every
+// thread loads kKPT partial keys at a time, all issued before any compare;
+// keys at or above their row's threshold go to the row's survivor list
+// (shared-memory counter), and one warp per row takes the 8 best of the
+// survivors.  A row with more than kSurv survivors (no threshold, or many
+// equal values) falls back to the warp merge of all its keys.
+template <class Tag>
+__device__ void merge_top8_rows(const Pass1Params& P, int64_t r0, int n, Top8EpiSmem& sm) {
+    constexpr int kKPT = 20;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    if (threadIdx.x < k) sm.drafts[threadIdx.x] = P.drafts[b * k + threadIdx.x];
-    if constexpr (MODE != MODE_TOP8) {
-        merge_argmax_rows<Tag>(P, b * (k + 1), k + 1, sm.rowkey);
-        if (threadIdx.x <= k) sm.am[threadIdx.x] = key_index(sm.rowkey[threadIdx.x]);
+    const int t = static_cast<int>(threadIdx.x);
+    const int nk = P.cpr * NWARPS * 8;
+    const int total = n * nk;
+    const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r0 * nk;
+    if (t < n) {
+        sm.floor_ord[t] = r0 + t < kThetaRows ? __ldcg(&P.theta_row[r0 + t]) : 0u;
+        sm.cnt[t] = 0;
     }
-    for (int t = wp; t <= k && MODE == MODE_TOP8; t += NWARPS) {
-        const int64_t r = b * (k + 1) + t;
-        if constexpr (MODE == MODE_TOP8) {
-            const uint64_t mine = row_top8_key<Tag>(P, r);
-            const uint64_t k0 = __shfl_sync(FULL_MASK, mine, 0);
-            if (lane == 0) sm.am[t] = key_index(k0);
-            if (lane < P.topk) {
-                int id = -1;
-                float val = __uint_as_float(0x7fc00000u);
-                if (mine != 0ull) {
-                    id = key_index(mine);
-                    val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + id);
+    for (int i0 = 0; i0 < total; i0 += NT * kKPT) {  // same trip count in every thread
+        uint64_t kk[kKPT];
+#pragma unroll
+        for (int j = 0; j < kKPT; ++j) {
+            const int i = i0 + j * NT + t;
+            kk[j] = i < total ? __ldcg(p + i) : 0ull;
+        }
+        __syncthreads();  // thresholds and counters are set
+#pragma unroll
+        for (int j = 0; j < kKPT; ++j) {
+            if (kk[j] != 0ull) {
+                const int row = (i0 + j * NT + t) / nk;
+                if (static_cast<uint32_t>(kk[j] >> 32) >= sm.floor_ord[row]) {
+                    const int pos = atomicAdd(&sm.cnt[row], 1);
+                    if (pos < kSurv) sm.surv[row][pos] = kk[j];
                 }
-                P.topk_ids[r * P.topk + lane] = id;
-                P.topk_vals[r * P.topk + lane] = val;
             }
-            if (lane == 0 && r < kThetaRows) P.theta_row[r] = 0u;
         }
     }
     __syncthreads();
+    for (int r = wp; r < n; r += NWARPS) {
+        const int c = sm.cnt[r];
+        uint64_t mine;
+        if (c <= kSurv) {
+            uint64_t l[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) l[e] = 0ull;
+            for (int i = lane; i < c; i += 32) {
+                const uint64_t kx = sm.surv[r][i];
+                if (kx > l[7]) top8_insert(l, kx);
+            }
+            mine = warp_top8(l);
+            if (__shfl_sync(FULL_MASK, mine, 7) == 0ull) mine = row_top8_key<Tag>(P, r0 + r);  // < 8 keys: exact
+        } else {
+            mine = row_top8_key<Tag>(P, r0 + r);
+        }
+        if (lane < 8) sm.top[r][lane] = mine;
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// Request epilogues (every thread of the last-ticket CTA).
+// ---------------------------------------------------------------------------
+template <class Tag, int MODE, class Smem>
+__device__ void epilogue_greedy(const Pass1Params& P, int64_t b, Smem& sm) {
+    const int k = P.k;
+    // The drafts are loaded into registers first and stored after the merge
+    // has issued its loads, so the two round trips overlap.
+    const int dr = threadIdx.x < k ? P.drafts[b * k + threadIdx.x] : 0;
+    if constexpr (MODE != MODE_TOP8) {
+        merge_argmax_rows<Tag>(P, b * (k + 1), k + 1, sm.rowkey);
+        if (threadIdx.x <= k) sm.am[threadIdx.x] = key_index(sm.rowkey[threadIdx.x]);
+        if (threadIdx.x < k) sm.drafts[threadIdx.x] = dr;
+    } else {
+        merge_top8_rows<Tag>(P, b * (k + 1), k + 1, sm);
+        if (threadIdx.x < k) sm.drafts[threadIdx.x] = dr;
+        // One thread per (row, rank): the argmax, the top-k outputs (values
+        // re-read at the winning indices, so they are the stored bits), and
+        // the row threshold back to zero.
+        for (int o = threadIdx.x; o < (k + 1) * 8; o += NT) {
+            const int t = o >> 3, e = o & 7;
+            const int64_t r = b * (k + 1) + t;
+            const uint64_t key = sm.top[t][e];
+            if (e == 0) sm.am[t] = key_index(key);
+            if (e < P.topk) {
+                int id = -1;
+                float val = __uint_as_float(0x7fc00000u);
+                if (key != 0ull) {
+                    id = key_index(key);
+                    val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + id);
+                }
+                P.topk_ids[r * P.topk + e] = id;
+                P.topk_vals[r * P.topk + e] = val;
+            }
+            if (e == 0 && r < kThetaRows) P.theta_row[r] = 0u;
+        }
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
     if (threadIdx.x < 32) {
         bool match = false;
         if (lane < k) {
@@ -599,12 +686,26 @@ __device__ void epilogue_tree(const Pass1Params& P, int64_t b, Pass1SmemTree& sm
     TreeArrays& ts = sm.t;
     const int n1 = P.rows_per_req;
     const int md = P.max_depth;
-    for (int c = threadIdx.x; c < n1; c += NT) {
-        ts.par[c] = P.parents[b * n1 + c];
-        ts.tok[c] = P.node_tokens[b * n1 + c];
+    // Parents and node tokens go to registers first and to shared memory
+    // after the merge has issued its loads, so the two round trips overlap.
+    constexpr int PER = kTreeNodes / NT;
+    int pr[PER], tr[PER];
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+        const int c = static_cast<int>(threadIdx.x) + q * NT;
+        pr[q] = c < n1 ? P.parents[b * n1 + c] : 0;
+        tr[q] = c < n1 ? P.node_tokens[b * n1 + c] : 0;
     }
     merge_argmax_rows<Tag>(P, b * n1, n1, ts.key);
-    for (int c = threadIdx.x; c < n1; c += NT) ts.am[c] = key_index(ts.key[c]);
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+        const int c = static_cast<int>(threadIdx.x) + q * NT;
+        if (c < n1) {
+            ts.par[c] = pr[q];
+            ts.tok[c] = tr[q];
+            ts.am[c] = key_index(ts.key[c]);
+        }
+    }
     __syncthreads();
     int bad = 0;
     for (int c = threadIdx.x; c < n1; c += NT) {
@@ -625,7 +726,6 @@ __device__ void epilogue_tree(const Pass1Params& P, int64_t b, Pass1SmemTree& sm
         __syncthreads();
         // Pointer jumping: after each round every node has summed the depth and
         // AND-ed the match flags of twice as many ancestors.
-        constexpr int PER = kTreeNodes / NT;
         for (int span = 1; span < n1; span <<= 1) {
             int na[PER], nd[PER], no[PER];
 #pragma unroll
@@ -691,6 +791,19 @@ template <class Tag>
 __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& sm) {
     const int k = P.k;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    constexpr int kGatherWarp = NWARPS - 1;
+    // The last warp fetches the drafts and their logits and q values first;
+    // those two dependent round trips overlap the merge of the partials.
+    int d = -1;
+    float ld = 0.0f, qf = 0.0f;
+    if (wp == kGatherWarp && lane < k) {
+        d = P.drafts[b * k + lane];
+        if (d >= 0 && d < P.V) {
+            const int64_t r = b * (k + 1) + lane;
+            ld = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + d);
+            qf = __ldg(P.q + (b * k + lane) * P.q_stride + d);
+        }
+    }
     for (int t = wp; t <= k; t += NWARPS) {
         const int64_t r = b * (k + 1) + t;
         const int np = P.cpr;
@@ -729,18 +842,14 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
         }
         return;
     }
-    if (threadIdx.x < 32) {
+    if (wp == kGatherWarp) {
         bool accept = false;
         if (lane < k) {
-            const int d = P.drafts[b * k + lane];
             const bool in = d >= 0 && d < P.V;
             double p = 0.0, qd = 0.0;
             if (in) {
-                const int64_t r = b * (k + 1) + lane;
-                const float l =
-                    load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + d);
-                p = exp((static_cast<double>(l) - static_cast<double>(sm.rowM[lane])) * P.invT_d) / sm.rowZ[lane];
-                qd = static_cast<double>(__ldg(P.q + (b * k + lane) * P.q_stride + d));
+                p = exp((static_cast<double>(ld) - static_cast<double>(sm.rowM[lane])) * P.invT_d) / sm.rowZ[lane];
+                qd = static_cast<double>(qf);
             }
             if (P.p_draft_out) P.p_draft_out[b * k + lane] = static_cast<float>(p);
             const double2 u = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(lane));
@@ -748,10 +857,10 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
         }
         const unsigned rej = __ballot_sync(FULL_MASK, lane < k && !accept);
         const int h = rej ? __ffs(rej) - 1 : k;
-        for (int i = lane; i <= k; i += 32) {
-            if (i < h) P.out_tokens[b * (k + 1) + i] = P.drafts[b * k + i];
-            else if (i > h) P.out_tokens[b * (k + 1) + i] = -1;
-        }
+        // out_tokens[i] = d_i for i < h, -1 after h; slot h is the resample's.
+        if (lane < h) P.out_tokens[b * (k + 1) + lane] = d;
+        else if (lane > h && lane <= k) P.out_tokens[b * (k + 1) + lane] = -1;
+        if (k == 32 && lane == 0 && h < 32) P.out_tokens[b * (k + 1) + 32] = -1;
         if (lane == 0) {
             P.accept_len[b] = h;
             RejState st = {};
@@ -890,7 +999,7 @@ __global__ void __launch_bounds__(NT, MODE == MODE_TOP8 ? 4 : 1) verify_pass1_ke
 // Request epilogues as their own kernel (one CTA per request), after the pass.
 template <class Tag, int MODE>
 __global__ void __launch_bounds__(NT) verify_epilogue_kernel(const Pass1Params P) {
-    __shared__ typename SmemFor<MODE>::type sm;
+    __shared__ typename EpiSmemFor<MODE>::type sm;
     grid_dependency_wait();
     grid_launch_dependents();
     run_epilogue<Tag, MODE>(P, blockIdx.x, sm);

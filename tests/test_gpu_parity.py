@@ -381,7 +381,8 @@ def test_rejection_qwen_full(V_):
 
 
 @pytest.mark.parametrize("V,k,T,dtype", [(16, 3, 1.0, "f32"), (1000, 4, 0.7, "bf16"), (4099, 2, 1.3, "f32"),
-                                         (7, 0, 1.0, "f32"), (33, 8, 0.5, "bf16"), (151936, 1, 2.0, "f32")])
+                                         (7, 0, 1.0, "f32"), (33, 8, 0.5, "bf16"), (151936, 1, 2.0, "f32"),
+                                         (300, 32, 0.9, "f32")])
 def test_rejection_small_cases(V_, V, k, T, dtype):
     rng = np.random.default_rng(V + k)
     B = 64 if V < 100000 else 8
