@@ -128,10 +128,10 @@ specdec_status dispatch_pass2(specdec_dtype dt, bool vec, Pass2Params P, cudaStr
 bool dtype_ok(specdec_dtype dt) { return dt == SPECDEC_F32 || dt == SPECDEC_BF16; }
 
 // Pass-1 partial bytes per chunk: one argmax key per warp, 8 keys per warp
-// (top-8), or the chunk's (max, sum) pair.
+// (top-8), or one (max, sum) pair per warp (softmax).
 constexpr size_t kArgmaxChunkBytes = NWARPS * sizeof(uint64_t);
 constexpr size_t kTop8ChunkBytes = NWARPS * 8 * sizeof(uint64_t);
-constexpr size_t kSoftmaxChunkBytes = sizeof(SoftmaxPartial);
+constexpr size_t kSoftmaxChunkBytes = NWARPS * sizeof(SoftmaxPartial);
 size_t slot_bytes(specdec_mode mode) {
     if (mode == SPECDEC_MODE_GREEDY) return kArgmaxChunkBytes > kTop8ChunkBytes ? kArgmaxChunkBytes : kTop8ChunkBytes;
     if (mode == SPECDEC_MODE_REJECTION) return kSoftmaxChunkBytes;

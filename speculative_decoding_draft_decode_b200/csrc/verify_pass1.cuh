@@ -123,7 +123,7 @@ template <> struct SmemFor<MODE_TREE> { using type = Pass1SmemTree; };
 
 // The top-8 epilogue's shared lists: per row, the partial keys at or above
 // the row threshold (kSurv at most) and the merged 8 best.
-constexpr int kSurv = 64;
+constexpr int kSurv = 128;
 struct Top8EpiSmem : Pass1Smem {
     unsigned floor_ord[kMaxRowsPerReq];
     int cnt[kMaxRowsPerReq];
@@ -419,29 +419,22 @@ struct Top8Reducer {
     }
 };
 
-// Softmax statistics of a chunk: its max M of the raw logits (NaN ignored),
-// then S = sum exp((l - M)/T) over the chunk, fp32 exp and sum within a
-// vector, fp64 across vectors and threads.  The chunk's elements are held in
-// registers, so the max is known before any exp is taken and no rescaling
-// is needed.  One (M, S) partial per chunk.
+// Softmax statistics of each warp's part of a chunk: its max M of the raw
+// logits (NaN ignored), then S = sum exp((l - M)/T) over the part, fp32 exp
+// and sum within a vector, fp64 across vectors and lanes.  The part's
+// elements are held in registers, so the max is known before any exp is
+// taken and no rescaling is needed; no CTA barrier is involved.  One (M, S)
+// partial per (chunk, warp).
 template <class Tag, int VEC>
 struct SoftmaxReducer {
     float invT;
     double invT_d;
     __device__ __forceinline__ void begin(int64_t, const Pass1Params&, Pass1Smem&) {}
-    // CTA-collective: max of the chunk.
-    __device__ __forceinline__ float chunk_max(float m, Pass1Smem& sm) {
-        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    // Warp-collective: max over the warp's part of the chunk.
+    __device__ __forceinline__ float part_max(float m) const {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, o));
-        float* red = reinterpret_cast<float*>(sm.red);
-        if (lane == 0) red[w] = m;
-        __syncthreads();
-        float r = red[0];
-#pragma unroll
-        for (int i = 1; i < NWARPS; ++i) r = fmaxf(r, red[i]);
-        __syncthreads();
-        return r;
+        return m;
     }
     __device__ __forceinline__ double vec_sum(const uint4& w, bool ok, float M) const {
         if (!ok) return 0.0;
@@ -450,15 +443,16 @@ struct SoftmaxReducer {
         for (int e = 0; e < VEC; ++e) s += expf((VecOps<Tag, VEC>::elem(w, e) - M) * invT);
         return static_cast<double>(s);
     }
-    // CTA-collective: store (M, S) of the chunk.
-    __device__ __forceinline__ void store(float M, double S, uint64_t chunk, const Pass1Params& P, Pass1Smem& sm) {
-        const double tot = block_sum_f64(S, reinterpret_cast<double*>(sm.red));
-        if (threadIdx.x == 0) {
+    // Warp-collective: store (M, S) of the warp's part of the chunk.
+    __device__ __forceinline__ void store(float M, double S, uint64_t chunk, const Pass1Params& P) const {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(FULL_MASK, S, o);
+        if ((threadIdx.x & 31) == 0) {
             SoftmaxPartial sp;
             sp.M = M;
             sp.pad = 0.0f;
-            sp.S = tot;
-            static_cast<SoftmaxPartial*>(P.partials)[chunk] = sp;
+            sp.S = S;
+            static_cast<SoftmaxPartial*>(P.partials)[chunk * NWARPS + (threadIdx.x >> 5)] = sp;
         }
     }
 };
@@ -565,18 +559,22 @@ __device__ uint64_t row_top8_key(const Pass1Params& P, int64_t r) {
     return mine;
 }
 
-// The 8 best keys of rows r0 .. r0+n-1 into sm.top (CTA-collective).  Every
-// thread loads kKPT partial keys at a time, all issued before any compare;
-// keys at or above their row's threshold go to the row's survivor list
-// (shared-memory counter), and one warp per row takes the 8 best of the
-// survivors.  A row with more than kSurv survivors (no threshold, or many
-// equal values) falls back to the warp merge of all its keys.
+// The 8 best keys of rows r0 .. r0+n-1 into sm.top (CTA-collective).
+//   1. Every thread loads kKPT partial keys at a time, all issued before any
+//      compare; keys at or above their row's threshold go to the row's
+//      survivor list (shared-memory counter).
+//   2. Every survivor's rank in its row is the number of the row's survivors
+//      above it (keys are distinct); ranks 0..7 are the row's 8 best.  The
+//      survivors of all rows are spread over all threads.
+// A row with more than kSurv survivors (no threshold, or many equal values)
+// or fewer than 8 falls back to the warp merge of all its keys, which also
+// rescans the row exactly when its partials hold fewer than 8 keys.
 template <class Tag>
 __device__ void merge_top8_rows(const Pass1Params& P, int64_t r0, int n, Top8EpiSmem& sm) {
     constexpr int kKPT = 20;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const int t = static_cast<int>(threadIdx.x);
-    const int nk = P.cpr * NWARPS * 8;
+    const int nk = P.cpr * NWARPS * 8;  // keys per row, a multiple of 64
     const int total = n * nk;
     const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r0 * nk;
     if (t < n) {
@@ -591,35 +589,46 @@ __device__ void merge_top8_rows(const Pass1Params& P, int64_t r0, int n, Top8Epi
             kk[j] = i < total ? __ldcg(p + i) : 0ull;
         }
         __syncthreads();  // thresholds and counters are set
+        // The row of key i, tracked as i grows by NT per step.
+        int row = (i0 + t) / nk, row_end = (row + 1) * nk;
 #pragma unroll
         for (int j = 0; j < kKPT; ++j) {
-            if (kk[j] != 0ull) {
-                const int row = (i0 + j * NT + t) / nk;
-                if (static_cast<uint32_t>(kk[j] >> 32) >= sm.floor_ord[row]) {
-                    const int pos = atomicAdd(&sm.cnt[row], 1);
-                    if (pos < kSurv) sm.surv[row][pos] = kk[j];
-                }
+            const int i = i0 + j * NT + t;
+            while (i >= row_end) {
+                ++row;
+                row_end += nk;
+            }
+            if (kk[j] != 0ull && static_cast<uint32_t>(kk[j] >> 32) >= sm.floor_ord[row]) {
+                const int pos = atomicAdd(&sm.cnt[row], 1);
+                if (pos < kSurv) sm.surv[row][pos] = kk[j];
             }
         }
     }
     __syncthreads();
+    // 2. Ranks.  Survivor (row, s) for rows with 8 <= count <= kSurv, taken
+    // in row order over a running index.
+    int base = 0;
+    for (int r = 0; r < n; ++r) {
+        const int c = sm.cnt[r];
+        const bool ok = c >= 8 && c <= kSurv;
+        if (ok) {
+            for (int s2 = t - base; s2 < c; s2 += NT) {
+                if (s2 < 0) continue;
+                const uint64_t key = sm.surv[r][s2];
+                int rank = 0;
+                for (int x = 0; x < c; ++x) rank += sm.surv[r][x] > key ? 1 : 0;
+                if (rank < 8) sm.top[r][rank] = key;
+            }
+            base = (base + c) % NT;
+        }
+    }
+    // Rows outside the fast case: one warp each.
     for (int r = wp; r < n; r += NWARPS) {
         const int c = sm.cnt[r];
-        uint64_t mine;
-        if (c <= kSurv) {
-            uint64_t l[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) l[e] = 0ull;
-            for (int i = lane; i < c; i += 32) {
-                const uint64_t kx = sm.surv[r][i];
-                if (kx > l[7]) top8_insert(l, kx);
-            }
-            mine = warp_top8(l);
-            if (__shfl_sync(FULL_MASK, mine, 7) == 0ull) mine = row_top8_key<Tag>(P, r0 + r);  // < 8 keys: exact
-        } else {
-            mine = row_top8_key<Tag>(P, r0 + r);
+        if (c < 8 || c > kSurv) {
+            const uint64_t mine = row_top8_key<Tag>(P, r0 + r);
+            if (lane < 8) sm.top[r][lane] = mine;
         }
-        if (lane < 8) sm.top[r][lane] = mine;
     }
     __syncthreads();
 }
@@ -806,16 +815,22 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
     }
     for (int t = wp; t <= k; t += NWARPS) {
         const int64_t r = b * (k + 1) + t;
-        const int np = P.cpr;
+        const int np = P.cpr * NWARPS;
         const SoftmaxPartial* p = static_cast<const SoftmaxPartial*>(P.partials) + r * np;
         MaxSum acc;
         acc.M = -FLT_MAX;
         acc.S = 0.0;
-        for (int i = lane; i < np; i += 32) {
-            MaxSum x;
-            x.M = __ldcg(&p[i].M);
-            x.S = __ldcg(&p[i].S);
-            acc = maxsum_merge(acc, x, P.invT_d);
+        constexpr int kPB = 8;  // partials per lane per batch, loaded together
+        for (int i0 = lane; i0 < np; i0 += 32 * kPB) {
+            MaxSum x[kPB];
+#pragma unroll
+            for (int j = 0; j < kPB; ++j) {
+                const int i = i0 + 32 * j;
+                x[j].M = i < np ? __ldcg(&p[i].M) : -FLT_MAX;
+                x[j].S = i < np ? __ldcg(&p[i].S) : 0.0;
+            }
+#pragma unroll
+            for (int j = 0; j < kPB; ++j) acc = maxsum_merge(acc, x[j], P.invT_d);
         }
         acc = warp_maxsum(acc, P.invT_d);
         if (lane == 0) {
@@ -913,7 +928,7 @@ __device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typena
         }
     }
     if (has_tail) m = fmaxf(m, tail);
-    const float M = red.chunk_max(m, sm);
+    const float M = red.part_max(m);
     double S = 0.0;
     if constexpr (UPT <= KEEP) {
 #pragma unroll
@@ -926,7 +941,7 @@ __device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typena
         }
     }
     if (has_tail) S += static_cast<double>(expf((tail - M) * P.invT));
-    red.store(M, S, static_cast<uint64_t>(r) * P.cpr + sub, P, sm);
+    red.store(M, S, static_cast<uint64_t>(r) * P.cpr + sub, P);
 }
 
 // ---------------------------------------------------------------------------
