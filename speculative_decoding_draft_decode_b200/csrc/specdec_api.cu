@@ -6,7 +6,8 @@
 // of any shape; each call returns those words to zero before it ends.
 //   [0, 256 KiB)            top-8 thresholds, one word per row (first 65536 rows)
 //   then                    streaming-pass partials, one slot per chunk
-//   then (rejection only)   per-request RejState, per-chunk masses of row h
+//   then (rejection only)   per-request RejState, per-chunk and per-unit masses
+//                           of row h
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -28,7 +29,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
     int64_t nv = 0, nv_full = 0, cpr = 0, NC = 0;
-    size_t partials1 = 0, state = 0, masses = 0, total = 0;
+    size_t partials1 = 0, state = 0, masses = 0, units = 0, total = 0;
 };
 
 // Layout of one call.  `vec` = elements per vector (1 on the scalar path),
@@ -48,6 +49,9 @@ Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t
         end = L.state + static_cast<size_t>(B) * sizeof(RejState);
         L.masses = align_up(end, 256);
         end = L.masses + static_cast<size_t>(B) * static_cast<size_t>(L.cpr) * sizeof(double2);
+        L.units = align_up(end, 256);
+        end = L.units + static_cast<size_t>(B) * static_cast<size_t>(L.cpr) *
+                            static_cast<size_t>(units_per_chunk(vec)) * sizeof(double2);
     }
     (void)rows_per_req;
     L.total = align_up(end, 256);
@@ -107,8 +111,8 @@ specdec_status launch_pass2(Pass2Params P, cudaStream_t stream) {
     if (P.cpr > 65535) return SPECDEC_ERR_UNSUPPORTED;  // grid limit
     const dim3 grid(static_cast<unsigned>(P.B), static_cast<unsigned>(P.cpr));
     if (launch_pdl(verify_resample_kernel<Tag, VEC>, grid, 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
-    if (launch_pdl(verify_resample_epilogue_kernel<Tag, VEC>, dim3(static_cast<unsigned>(P.B)), 0, stream, P) !=
-        cudaSuccess)
+    const unsigned search_ctas = static_cast<unsigned>((P.B + NWARPS - 1) / NWARPS);  // a warp per request
+    if (launch_pdl(verify_resample_epilogue_kernel<Tag, VEC>, dim3(search_ctas), 0, stream, P) != cudaSuccess)
         return SPECDEC_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
@@ -330,6 +334,7 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
     Q.offset = offset;
     Q.state = state;
     Q.chunk_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.masses);
+    Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
     Q.out_tokens = out_tokens;
     return dispatch_pass2(dtype, vec, Q, s);
 }

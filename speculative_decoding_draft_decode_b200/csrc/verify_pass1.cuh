@@ -734,8 +734,11 @@ __device__ void epilogue_tree(const Pass1Params& P, int64_t b, Pass1SmemTree& sm
         }
         __syncthreads();
         // Pointer jumping: after each round every node has summed the depth and
-        // AND-ed the match flags of twice as many ancestors.
-        for (int span = 1; span < n1; span <<= 1) {
+        // AND-ed the match flags of twice as many ancestors.  After the rounds
+        // with span <= max_depth, a node has covered min(depth, 2 * last span)
+        // > max_depth edges, so every node within max_depth of the root is
+        // complete and every deeper node shows a depth above max_depth.
+        for (int span = 1; span <= md && span < n1; span <<= 1) {
             int na[PER], nd[PER], no[PER];
 #pragma unroll
             for (int q = 0; q < PER; ++q) {

@@ -9,12 +9,16 @@
 //
 // Two kernels, both launched with programmatic stream serialisation:
 //   verify_resample_kernel            one CTA per (request, chunk of row h):
-//                                     the chunk's mass of r and of p (fp64);
-//   verify_resample_epilogue_kernel   one CTA per request: scans the chunk
-//                                     masses in index order for the chunk
-//                                     where the cumulative mass first exceeds
-//                                     u_res * S, rescans that chunk in index
-//                                     order and writes the token.
+//                                     the mass of r and of p (fp64) of the
+//                                     chunk and of each of its units (the 32
+//                                     consecutive vectors one warp load
+//                                     instruction covers), plus the ragged
+//                                     row end as one more unit of the last
+//                                     chunk;
+//   verify_resample_epilogue_kernel   one warp per request: finds, in index
+//                                     order, the chunk, then the unit, then
+//                                     the element where the running mass
+//                                     first exceeds u_res * S.
 // No CTA waits for another and nothing needs resetting between calls.
 #pragma once
 
@@ -29,6 +33,9 @@
 #include "verify_common.cuh"
 
 namespace specdec {
+
+// Units per chunk, plus one slot for the ragged row end (last chunk only).
+__host__ __device__ constexpr int units_per_chunk(int vec) { return chunk_upt(vec) * NWARPS + 1; }
 
 struct Pass2Params {
     const void* logits;
@@ -45,6 +52,7 @@ struct Pass2Params {
     uint64_t offset;
     const RejState* state;
     double2* chunk_mass;  // [B, cpr] (residual mass, target mass) of row h
+    double2* unit_mass;   // [B, cpr, units_per_chunk] likewise per unit
     int32_t* out_tokens;
 };
 
@@ -116,9 +124,41 @@ __device__ __forceinline__ Pass2Row pass2_row(const Pass2Params& P, int64_t b, c
     return R;
 }
 
+// Warp-collective transpose-reduce of 16 values per lane: lane L returns the
+// warp total of value (L >> 1) & 15 (each total lands in two lanes).  Four
+// halving exchanges and one full one: 16 shuffles instead of 16 x 5.
+__device__ __forceinline__ double warp_sum16(double (&v)[16]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool hi = (lane & 16) != 0;
+        const double send = hi ? v[i] : v[i + 8];
+        v[i] = (hi ? v[i + 8] : v[i]) + __shfl_xor_sync(FULL_MASK, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool hi = (lane & 8) != 0;
+        const double send = hi ? v[i] : v[i + 4];
+        v[i] = (hi ? v[i + 4] : v[i]) + __shfl_xor_sync(FULL_MASK, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool hi = (lane & 4) != 0;
+        const double send = hi ? v[i] : v[i + 2];
+        v[i] = (hi ? v[i + 2] : v[i]) + __shfl_xor_sync(FULL_MASK, send, 4);
+    }
+    {
+        const bool hi = (lane & 2) != 0;
+        const double send = hi ? v[0] : v[1];
+        v[0] = (hi ? v[1] : v[0]) + __shfl_xor_sync(FULL_MASK, send, 2);
+    }
+    return v[0] + __shfl_xor_sync(FULL_MASK, v[0], 1);
+}
+
 // ---------------------------------------------------------------------------
-// Chunk masses: CTA (b, sub) sums r and p over chunk `sub` of request b's row
-// h.  Every thread issues all its loads of the chunk before any arithmetic.
+// Chunk and unit masses: CTA (b, sub) sums r and p over chunk `sub` of
+// request b's row h, and over each unit of it.  Every thread issues all its
+// loads of a batch of kU vectors before any arithmetic.
 // ---------------------------------------------------------------------------
 template <class Tag, int VEC>
 __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P) {
@@ -126,7 +166,8 @@ __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P
     using Elem = typename Tag::storage;
     constexpr int CH = chunk_vecs(VEC);
     constexpr int UPT = chunk_upt(VEC);
-    constexpr int BATCH = UPT < kU ? UPT : kU;
+    constexpr int UPC = units_per_chunk(VEC);
+    static_assert(kU == 8, "the unit transpose-reduce takes 8 vectors per thread per batch");
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const int t = static_cast<int>(threadIdx.x);
 
@@ -140,36 +181,63 @@ __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P
     const Pass2Row R = pass2_row<Tag>(P, b, st);
     const Elem* row = static_cast<const Elem*>(R.row);
     const int cnt = chunk_count(P.nv_full, sub, VEC);
+    double2* um = P.unit_mass + (b * P.cpr + sub) * UPC;
 
     double sr = 0.0, sp = 0.0;
-    for (int u0 = 0; u0 < UPT; u0 += BATCH) {
-        ResidualVec<Tag, VEC> v[BATCH];
+    for (int u0 = 0; u0 < UPT; u0 += kU) {
+        ResidualVec<Tag, VEC> v[kU];
 #pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
+        for (int u = 0; u < kU; ++u) {
             const int i = stream_pos(u0 + u, t);
             if (i < cnt) v[u].load(row, R.qrow, sub * CH + i, R.has_q);
         }
+        double m[16];
 #pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
+        for (int u = 0; u < kU; ++u) {
+            double ar = 0.0, ap = 0.0;
             if (stream_pos(u0 + u, t) < cnt) {
                 float p[VEC], r[VEC];
                 v[u].values(R.has_q, st.M, P.invT, R.invZ, p, r);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) {
-                    sr += static_cast<double>(r[e]);
-                    sp += static_cast<double>(p[e]);
+                    ar += static_cast<double>(r[e]);
+                    ap += static_cast<double>(p[e]);
                 }
             }
+            m[u] = ar;
+            m[kU + u] = ap;
+            sr += ar;
+            sp += ap;
+        }
+        // Unit (u, warp) is the 32 vectors u*NT + warp*32 + [0, 32); its index
+        // in the chunk is u*NWARPS + warp, which is index order.
+        const double tot = warp_sum16(m);
+        const int which = (lane >> 1) & 15;
+        if ((lane & 1) == 0) {
+            double* dst = reinterpret_cast<double*>(&um[(u0 + (which & 7)) * NWARPS + wp]);
+            dst[which >> 3] = tot;
         }
     }
-    // The ragged row end (fewer than VEC elements) goes to lanes of warp 0.
+    // The ragged row end (fewer than VEC elements): lanes of warp 0, stored
+    // as the last unit slot of the last chunk.
     if (sub == P.cpr - 1 && wp == 0) {
         const int x = P.nv_full * VEC + lane;
+        double tr = 0.0, tp = 0.0;
         if (x < P.V) {
             float p, r;
             residual_scalar<Tag>(row, R.qrow, x, R.has_q, st.M, P.invT, R.invZ, p, r);
-            sr += static_cast<double>(r);
-            sp += static_cast<double>(p);
+            tr = static_cast<double>(r);
+            tp = static_cast<double>(p);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            tr += __shfl_xor_sync(FULL_MASK, tr, o);
+            tp += __shfl_xor_sync(FULL_MASK, tp, o);
+        }
+        if (lane == 0) {
+            um[UPC - 1] = make_double2(tr, tp);
+            sr += tr;
+            sp += tp;
         }
     }
 #pragma unroll
@@ -194,131 +262,189 @@ __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P
 }
 
 // ---------------------------------------------------------------------------
-// Token search of request b (one CTA).
+// Token search, one warp per request.
 // ---------------------------------------------------------------------------
-struct ResampleSmem {
-    double dred[NWARPS];
-    int ired[NWARPS];
-    double before;
-};
+// One level of the search over masses m[0, n) in index order (component .x
+// = residual, .y = target; `use_p` picks .y), lane L owning the contiguous
+// range [L * per, ...).  With `found`, returns the first index whose running
+// mass, starting from `start`, exceeds `target` and sets *before to the mass
+// before it; with no crossing (rounding put the target past the end) or
+// without `found`, returns the last index with positive mass and clears
+// `found`; -1 if there is none.  Warp-collective.
+__device__ __forceinline__ int warp_find_level(const double2* m, int n, bool use_p, double start, double target,
+                                               bool& found, double& before) {
+    constexpr int kKeep = 4;  // masses per lane kept in registers for the walk
+    const int lane = threadIdx.x & 31;
+    const int per = (n + 31) / 32;
+    const int i0 = min(lane * per, n), i1 = min(i0 + per, n);
+    double ls = 0.0, keep[kKeep];
+#pragma unroll
+    for (int j = 0; j < kKeep; ++j) {
+        keep[j] = 0.0;
+        if (i0 + j < i1) {
+            const double2 x = __ldcg(&m[i0 + j]);
+            keep[j] = use_p ? x.y : x.x;
+        }
+    }
+    for (int i = i0; i < i1; ++i) {
+        double v;
+        if (i - i0 < kKeep) {
+            v = 0.0;
+#pragma unroll
+            for (int j = 0; j < kKeep; ++j)
+                if (i - i0 == j) v = keep[j];
+        } else {
+            const double2 x = __ldcg(&m[i]);
+            v = use_p ? x.y : x.x;
+        }
+        ls += v;
+    }
+    double incl = ls;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double w = __shfl_up_sync(FULL_MASK, incl, o);
+        if (lane >= o) incl += w;
+    }
+    double run = start + (incl - ls);
+    int hit = INT_MAX, last = -1;
+    double hit_before = 0.0;
+    for (int i = i0; i < i1; ++i) {
+        double v;
+        if (i - i0 < kKeep) {
+            v = 0.0;
+#pragma unroll
+            for (int j = 0; j < kKeep; ++j)
+                if (i - i0 == j) v = keep[j];
+        } else {
+            const double2 x = __ldcg(&m[i]);
+            v = use_p ? x.y : x.x;
+        }
+        if (v > 0.0) {
+            last = i;
+            if (found && hit == INT_MAX && run + v > target) {
+                hit = i;
+                hit_before = run;
+            }
+        }
+        run += v;
+    }
+    const unsigned hits = __ballot_sync(FULL_MASK, hit != INT_MAX);
+    if (hits) {
+        const int src = __ffs(hits) - 1;
+        before = __shfl_sync(FULL_MASK, hit_before, src);
+        return __shfl_sync(FULL_MASK, hit, src);
+    }
+    found = false;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(FULL_MASK, last, o));
+    return last;
+}
 
 template <class Tag, int VEC>
 __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass2Params P) {
-    __shared__ ResampleSmem sm;
     using Elem = typename Tag::storage;
     constexpr int CH = chunk_vecs(VEC);
-    constexpr int UPT = chunk_upt(VEC);
-    const int t = static_cast<int>(threadIdx.x);
+    constexpr int UPC = units_per_chunk(VEC);
+    const int lane = threadIdx.x & 31;
 
     grid_dependency_wait();
     grid_launch_dependents();
 
-    const int64_t b = blockIdx.x;
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * NWARPS + (threadIdx.x >> 5);
+    if (b >= P.B) return;  // warp-uniform
     const RejState st = P.state[b];
     if (!st.valid) return;  // the statistics pass already wrote -1 everywhere
+    const int64_t out_at = b * (P.k + 1) + st.h;
 
-    // 1. The chunk where the cumulative mass first exceeds u_res * S; thread
-    //    t owns chunks [c0, c1), in index order.
+    // Totals of r and p over the chunk masses, then u_res * S.
     const double2* cm = P.chunk_mass + b * P.cpr;
-    const int per = (P.cpr + NT - 1) / NT;
-    const int c0 = min(t * per, P.cpr), c1 = min(c0 + per, P.cpr);
     double tr = 0.0, tp = 0.0;
-    for (int c = c0; c < c1; ++c) {
-        const double2 m = __ldcg(&cm[c]);
-        tr += m.x;
-        tp += m.y;
+    for (int c = lane; c < P.cpr; c += 32) {
+        const double2 x = __ldcg(&cm[c]);
+        tr += x.x;
+        tp += x.y;
     }
-    double Sr, Sp;
-    const double pre_r = block_exclusive_scan_f64(tr, sm.dred, &Sr);
-    const double pre_p = block_exclusive_scan_f64(tp, sm.dred, &Sp);
-    const bool use_p = !(Sr > 0.0);
-    const double S = use_p ? Sp : Sr;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tr += __shfl_xor_sync(FULL_MASK, tr, o);
+        tp += __shfl_xor_sync(FULL_MASK, tp, o);
+    }
+    const bool use_p = !(tr > 0.0);
+    const double S = use_p ? tp : tr;
     const double2 uu = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(st.h));
     const double target = uu.y * S;
-    int cand = INT_MAX, last_pos = -1;
-    double run = use_p ? pre_p : pre_r, cand_before = 0.0;
-    for (int c = c0; c < c1; ++c) {
-        const double2 m2 = __ldcg(&cm[c]);
-        const double m = use_p ? m2.y : m2.x;
-        if (m > 0.0) last_pos = c;
-        if (cand == INT_MAX && run + m > target) {
-            cand = c;
-            cand_before = run;
-        }
-        run += m;
-    }
-    int chunk = block_min_int(cand, sm.ired);
-    const bool found = chunk != INT_MAX;
-    if (found && cand == chunk) sm.before = cand_before;
-    if (!found) chunk = block_max_int(last_pos, sm.ired);  // rounding put the target past the end
-    __syncthreads();
-    const int64_t out_at = b * (P.k + 1) + st.h;
+
+    // 1. the chunk, 2. the unit within it, 3. the element within the unit.
+    bool found = true;
+    double before = 0.0;
+    const int chunk = warp_find_level(cm, P.cpr, use_p, 0.0, target, found, before);
     if (chunk < 0) {  // no mass anywhere (cannot happen for a valid row)
-        if (t == 0) P.out_tokens[out_at] = P.V - 1;
+        if (lane == 0) P.out_tokens[out_at] = P.V - 1;
         return;
     }
-
-    // 2. Rescan that chunk in index order: thread t holds UPT consecutive
-    //    vectors, and the last thread also the ragged row end.
-    const Pass2Row R = pass2_row<Tag>(P, b, st);
-    const Elem* row = static_cast<const Elem*>(R.row);
-    const int cnt = chunk_count(P.nv_full, chunk, VEC);
-    ResidualVec<Tag, VEC> v[UPT];
+    const bool has_tail = chunk == P.cpr - 1 && P.nv_full * VEC < P.V;
+    const double2* um = P.unit_mass + (b * P.cpr + chunk) * UPC;
+    const int unit = warp_find_level(um, has_tail ? UPC : UPC - 1, use_p, before, target, found, before);
+    int token = P.V - 1;
+    if (unit >= 0) {
+        const Pass2Row R = pass2_row<Tag>(P, b, st);
+        const Elem* row = static_cast<const Elem*>(R.row);
+        float m[VEC];
+        int x0 = 0, nx = 0;  // first element of the lane and how many it holds
+        if (unit == UPC - 1) {  // the ragged row end, one element per lane
+            x0 = P.nv_full * VEC + lane;
+            nx = x0 < P.V ? 1 : 0;
+            if (nx) {
+                float p, r;
+                residual_scalar<Tag>(row, R.qrow, x0, R.has_q, st.M, P.invT, R.invZ, p, r);
+                m[0] = use_p ? p : r;
+            }
+        } else {
+            const int u = unit / NWARPS, w = unit % NWARPS;
+            const int pos = stream_pos(u, w * 32 + lane);
+            const int j = chunk * CH + pos;
+            x0 = j * VEC;
+            if (pos < chunk_count(P.nv_full, chunk, VEC)) {
+                nx = VEC;
+                ResidualVec<Tag, VEC> v;
+                v.load(row, R.qrow, j, R.has_q);
+                float p[VEC], r[VEC];
+                v.values(R.has_q, st.M, P.invT, R.invZ, p, r);
 #pragma unroll
-    for (int u = 0; u < UPT; ++u) {
-        const int i = rescan_pos(u, t, VEC);
-        if (i < cnt) v[u].load(row, R.qrow, chunk * CH + i, R.has_q);
-    }
-    constexpr int kTail = VEC > 1 ? VEC - 1 : 1;
-    const bool has_tail = t == NT - 1 && chunk == P.cpr - 1;
-    const int tail0 = P.nv_full * VEC;
-    float mv[UPT][VEC], mt[kTail];
-    double ls = 0.0;
+                for (int e = 0; e < VEC; ++e) m[e] = use_p ? p[e] : r[e];
+            }
+        }
+        double ls = 0.0;
 #pragma unroll
-    for (int u = 0; u < UPT; ++u) {
-        const bool in = rescan_pos(u, t, VEC) < cnt;
-        float p[VEC], r[VEC];
-        v[u].values(R.has_q, st.M, P.invT, R.invZ, p, r);
+        for (int e = 0; e < VEC; ++e)
+            if (e < nx) ls += static_cast<double>(m[e]);
+        double incl = ls;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double w = __shfl_up_sync(FULL_MASK, incl, o);
+            if (lane >= o) incl += w;
+        }
+        double run = before + (incl - ls);
+        int hit = INT_MAX, last = -1;
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-            mv[u][e] = in ? (use_p ? p[e] : r[e]) : 0.0f;
-            ls += static_cast<double>(mv[u][e]);
+            if (e < nx) {
+                const double v = static_cast<double>(m[e]);
+                if (v > 0.0) {
+                    last = x0 + e;
+                    if (found && hit == INT_MAX && run + v > target) hit = x0 + e;
+                }
+                run += v;
+            }
         }
-    }
 #pragma unroll
-    for (int e = 0; e < kTail; ++e) {
-        mt[e] = 0.0f;
-        if (has_tail && tail0 + e < P.V) {
-            float p, r;
-            residual_scalar<Tag>(row, R.qrow, tail0 + e, R.has_q, st.M, P.invT, R.invZ, p, r);
-            mt[e] = use_p ? p : r;
-            ls += static_cast<double>(mt[e]);
+        for (int o = 16; o > 0; o >>= 1) {
+            hit = min(hit, __shfl_xor_sync(FULL_MASK, hit, o));
+            last = max(last, __shfl_xor_sync(FULL_MASK, last, o));
         }
+        token = hit != INT_MAX ? hit : (last >= 0 ? last : P.V - 1);
     }
-    double dummy;
-    double run2 = block_exclusive_scan_f64(ls, sm.dred, &dummy) + (found ? sm.before : 0.0);
-    int hit = INT_MAX, lastp = -1;
-#pragma unroll
-    for (int u = 0; u < UPT; ++u) {
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            const int x = (chunk * CH + rescan_pos(u, t, VEC)) * VEC + e;
-            const double m = static_cast<double>(mv[u][e]);
-            if (m > 0.0) lastp = x;
-            run2 += m;
-            if (found && hit == INT_MAX && m > 0.0 && run2 > target) hit = x;
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < kTail; ++e) {
-        const double m = static_cast<double>(mt[e]);
-        if (m > 0.0) lastp = tail0 + e;
-        run2 += m;
-        if (found && hit == INT_MAX && m > 0.0 && run2 > target) hit = tail0 + e;
-    }
-    hit = block_min_int(hit, sm.ired);
-    lastp = block_max_int(lastp, sm.ired);
-    if (t == 0) P.out_tokens[out_at] = hit != INT_MAX ? hit : (lastp >= 0 ? lastp : P.V - 1);
+    if (lane == 0) P.out_tokens[out_at] = token;
 }
 
 }  // namespace specdec

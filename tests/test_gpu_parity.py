@@ -326,6 +326,21 @@ def test_tree_max_size_and_depth(V_):
     assert (got[0] == -1).all()
 
 
+@pytest.mark.parametrize("md", [1, 2, 3, 4, 5, 7, 8])
+def test_tree_depth_bound_small(V_, md):
+    """Chains and brooms around the depth bound: depth md is valid, md + 1 is
+    not, for bounds that are and are not one less than a power of two."""
+    for n1 in (md, md + 1, md + 2, 2 * md + 3):
+        chain = np.array([-1] + list(range(n1 - 1)), np.int32)
+        t = gen.tree_synthetic(seed=md * 10 + n1, B=3, parents=chain, V=300, p_agree=1.0, max_depth=md,
+                               dtype="f32")
+        got = check_tree(V_, t)
+        assert (got[0] == (n1 - 1 if n1 - 1 <= md else -1)).all()
+        broom = np.array([-1] + [max(0, c - 1) if c <= md else 0 for c in range(1, n1 + 4)], np.int32)
+        check_tree(V_, gen.tree_synthetic(seed=md + n1, B=3, parents=broom, V=300, p_agree=0.9, max_depth=md,
+                                          dtype="bf16"))
+
+
 def test_tree_single_node(V_):
     t = gen.tree_synthetic(seed=2, B=4, parents=np.array([-1], np.int32), V=100, dtype="f32", max_depth=1)
     got = check_tree(V_, t)
