@@ -76,10 +76,10 @@ bool rows_fit(int64_t rows, int64_t row_stride, int V) {
 // while the previous kernel of the stream drains; it waits (griddepcontrol)
 // before touching global memory, so stream order is kept.
 template <class Kernel, class Params>
-cudaError_t launch_pdl(Kernel fn, dim3 grid, int dyn, cudaStream_t stream, const Params& P) {
+cudaError_t launch_pdl(Kernel fn, dim3 grid, int dyn, cudaStream_t stream, const Params& P, int block = NT) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(NT);
+    cfg.blockDim = dim3(static_cast<unsigned>(block));
     cfg.dynamicSmemBytes = static_cast<size_t>(dyn);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -99,8 +99,16 @@ specdec_status launch_pass1(Pass1Params P, cudaStream_t stream) {
     const dim3 grid(static_cast<unsigned>(P.R), static_cast<unsigned>(P.cpr));
     if (launch_pdl(verify_pass1_kernel<Tag, VEC, STREAM_MODE>, grid, 0, stream, P) != cudaSuccess)
         return SPECDEC_ERR_CUDA;
-    if (launch_pdl(verify_epilogue_kernel<Tag, MODE>, dim3(static_cast<unsigned>(P.B)), 0, stream, P) != cudaSuccess)
-        return SPECDEC_ERR_CUDA;
+    if constexpr (MODE == MODE_TOP8) {
+        const int rows = P.k + 1 < kTop8EpiWarps ? P.k + 1 : kTop8EpiWarps;  // a warp per row
+        if (launch_pdl(verify_top8_epilogue_kernel<Tag>, dim3(static_cast<unsigned>(P.B)), 0, stream, P, 32 * rows) !=
+            cudaSuccess)
+            return SPECDEC_ERR_CUDA;
+    } else {
+        if (launch_pdl(verify_epilogue_kernel<Tag, MODE>, dim3(static_cast<unsigned>(P.B)), 0, stream, P) !=
+            cudaSuccess)
+            return SPECDEC_ERR_CUDA;
+    }
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 

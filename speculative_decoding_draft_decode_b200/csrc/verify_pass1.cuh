@@ -121,17 +121,6 @@ struct Pass1SmemTree : Pass1Smem {
 template <int MODE> struct SmemFor { using type = Pass1Smem; };
 template <> struct SmemFor<MODE_TREE> { using type = Pass1SmemTree; };
 
-// The top-8 epilogue's shared lists: per row, the partial keys at or above
-// the row threshold (kSurv at most) and the merged 8 best.
-constexpr int kSurv = 128;
-struct Top8EpiSmem : Pass1Smem {
-    unsigned floor_ord[kMaxRowsPerReq];
-    int cnt[kMaxRowsPerReq];
-    uint64_t surv[kMaxRowsPerReq][kSurv];
-    uint64_t top[kMaxRowsPerReq][8];
-};
-template <int MODE> struct EpiSmemFor { using type = typename SmemFor<MODE>::type; };
-template <> struct EpiSmemFor<MODE_TOP8> { using type = Top8EpiSmem; };
 
 // ---------------------------------------------------------------------------
 // One 16-byte vector as loaded: its max (NaN ignored) and its elements.
@@ -559,135 +548,106 @@ __device__ uint64_t row_top8_key(const Pass1Params& P, int64_t r) {
     return mine;
 }
 
-// The 8 best keys of rows r0 .. r0+n-1 into sm.top (CTA-collective).
-//   1. Every thread loads kKPT partial keys at a time, all issued before any
-//      compare; keys at or above their row's threshold go to the row's
-//      survivor list (shared-memory counter).
-//   2. Every survivor's rank in its row is the number of the row's survivors
-//      above it (keys are distinct); ranks 0..7 are the row's 8 best.  The
-//      survivors of all rows are spread over all threads.
-// A row with more than kSurv survivors (no threshold, or many equal values)
-// or fewer than 8 falls back to the warp merge of all its keys, which also
-// rescans the row exactly when its partials hold fewer than 8 keys.
+// The top-8 epilogue's shared memory: per warp a survivor list, per row the
+// merged 8 best, and the request's drafts and argmaxes.
+constexpr int kSurv = 128;
+constexpr int kTop8EpiWarps = 16;
+struct Top8EpiSmem {
+    uint64_t surv[kTop8EpiWarps][kSurv];
+    uint64_t top[kMaxRowsPerReq][8];
+    int am[kMaxRowsPerReq];
+    int drafts[kMaxRowsPerReq];
+};
+
+// The 8 best keys of row r into top[0..8) (warp-collective).  Each lane
+// issues its loads of a batch together; keys at or above the row threshold
+// (the largest 8th best any chunk of the row published, a lower bound on the
+// row's own 8th best) are ballot-compacted into the warp's survivor list,
+// and the warp takes the 8 best of the survivors.  A row with more than
+// kSurv survivors or fewer than 8 falls back to the merge of all its keys,
+// which rescans the row exactly when its partials hold fewer than 8 keys.
 template <class Tag>
-__device__ void merge_top8_rows(const Pass1Params& P, int64_t r0, int n, Top8EpiSmem& sm) {
-    constexpr int kKPT = 20;
-    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    const int t = static_cast<int>(threadIdx.x);
-    const int nk = P.cpr * NWARPS * 8;  // keys per row, a multiple of 64
-    const int total = n * nk;
-    const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r0 * nk;
-    if (t < n) {
-        sm.floor_ord[t] = r0 + t < kThetaRows ? __ldcg(&P.theta_row[r0 + t]) : 0u;
-        sm.cnt[t] = 0;
-    }
-    for (int i0 = 0; i0 < total; i0 += NT * kKPT) {  // same trip count in every thread
-        uint64_t kk[kKPT];
+__device__ void row_top8_warp(const Pass1Params& P, int64_t r, uint64_t* surv, uint64_t* top) {
+    constexpr int KB = 16;  // keys per lane per batch
+    const int lane = threadIdx.x & 31;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    const int nk = P.cpr * NWARPS * 8;
+    const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r * nk;
+    unsigned fl = 0u;
+    if (lane == 0 && r < kThetaRows) fl = __ldcg(&P.theta_row[r]);
+    int cnt = 0;  // warp-uniform
+    for (int i0 = 0; i0 < nk; i0 += 32 * KB) {
+        uint64_t kk[KB];
 #pragma unroll
-        for (int j = 0; j < kKPT; ++j) {
-            const int i = i0 + j * NT + t;
-            kk[j] = i < total ? __ldcg(p + i) : 0ull;
+        for (int j = 0; j < KB; ++j) {
+            const int i = i0 + j * 32 + lane;
+            kk[j] = i < nk ? __ldcg(p + i) : 0ull;
         }
-        __syncthreads();  // thresholds and counters are set
-        // The row of key i, tracked as i grows by NT per step.
-        int row = (i0 + t) / nk, row_end = (row + 1) * nk;
+        fl = __shfl_sync(FULL_MASK, fl, 0);
 #pragma unroll
-        for (int j = 0; j < kKPT; ++j) {
-            const int i = i0 + j * NT + t;
-            while (i >= row_end) {
-                ++row;
-                row_end += nk;
-            }
-            if (kk[j] != 0ull && static_cast<uint32_t>(kk[j] >> 32) >= sm.floor_ord[row]) {
-                const int pos = atomicAdd(&sm.cnt[row], 1);
-                if (pos < kSurv) sm.surv[row][pos] = kk[j];
-            }
+        for (int j = 0; j < KB; ++j) {
+            const bool pass = kk[j] != 0ull && static_cast<uint32_t>(kk[j] >> 32) >= fl;
+            const unsigned mask = __ballot_sync(FULL_MASK, pass);
+            const int pos = cnt + __popc(mask & lt_mask);
+            if (pass && pos < kSurv) surv[pos] = kk[j];
+            cnt += __popc(mask);
         }
     }
-    __syncthreads();
-    // 2. Ranks.  Survivor (row, s) for rows with 8 <= count <= kSurv, taken
-    // in row order over a running index.
-    int base = 0;
-    for (int r = 0; r < n; ++r) {
-        const int c = sm.cnt[r];
-        const bool ok = c >= 8 && c <= kSurv;
-        if (ok) {
-            for (int s2 = t - base; s2 < c; s2 += NT) {
-                if (s2 < 0) continue;
-                const uint64_t key = sm.surv[r][s2];
-                int rank = 0;
-                for (int x = 0; x < c; ++x) rank += sm.surv[r][x] > key ? 1 : 0;
-                if (rank < 8) sm.top[r][rank] = key;
-            }
-            base = (base + c) % NT;
+    __syncwarp();
+    uint64_t mine;
+    if (cnt >= 8 && cnt <= kSurv) {
+        uint64_t l[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) l[e] = 0ull;
+        for (int i = lane; i < cnt; i += 32) {
+            const uint64_t kx = surv[i];
+            if (kx > l[7]) top8_insert(l, kx);
         }
+        mine = warp_top8(l);
+    } else {
+        mine = row_top8_key<Tag>(P, r);
     }
-    // Rows outside the fast case: one warp each.
-    for (int r = wp; r < n; r += NWARPS) {
-        const int c = sm.cnt[r];
-        if (c < 8 || c > kSurv) {
-            const uint64_t mine = row_top8_key<Tag>(P, r0 + r);
-            if (lane < 8) sm.top[r][lane] = mine;
-        }
-    }
-    __syncthreads();
+    if (lane < 8) top[lane] = mine;
+    __syncwarp();
 }
 
 // ---------------------------------------------------------------------------
 // Request epilogues (every thread of the last-ticket CTA).
 // ---------------------------------------------------------------------------
-template <class Tag, int MODE, class Smem>
-__device__ void epilogue_greedy(const Pass1Params& P, int64_t b, Smem& sm) {
+// Greedy accept scan of request b (warp 0): h = the number of leading drafts
+// equal to their row's argmax; out = d_0..d_{h-1}, argmax_h, then -1.
+__device__ __forceinline__ void greedy_accept(const Pass1Params& P, int64_t b, const int* drafts, const int* am) {
     const int k = P.k;
-    // The drafts are loaded into registers first and stored after the merge
-    // has issued its loads, so the two round trips overlap.
-    const int dr = threadIdx.x < k ? P.drafts[b * k + threadIdx.x] : 0;
-    if constexpr (MODE != MODE_TOP8) {
-        merge_argmax_rows<Tag>(P, b * (k + 1), k + 1, sm.rowkey);
-        if (threadIdx.x <= k) sm.am[threadIdx.x] = key_index(sm.rowkey[threadIdx.x]);
-        if (threadIdx.x < k) sm.drafts[threadIdx.x] = dr;
-    } else {
-        merge_top8_rows<Tag>(P, b * (k + 1), k + 1, sm);
-        if (threadIdx.x < k) sm.drafts[threadIdx.x] = dr;
-        // One thread per (row, rank): the argmax, the top-k outputs (values
-        // re-read at the winning indices, so they are the stored bits), and
-        // the row threshold back to zero.
-        for (int o = threadIdx.x; o < (k + 1) * 8; o += NT) {
-            const int t = o >> 3, e = o & 7;
-            const int64_t r = b * (k + 1) + t;
-            const uint64_t key = sm.top[t][e];
-            if (e == 0) sm.am[t] = key_index(key);
-            if (e < P.topk) {
-                int id = -1;
-                float val = __uint_as_float(0x7fc00000u);
-                if (key != 0ull) {
-                    id = key_index(key);
-                    val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + id);
-                }
-                P.topk_ids[r * P.topk + e] = id;
-                P.topk_vals[r * P.topk + e] = val;
-            }
-            if (e == 0 && r < kThetaRows) P.theta_row[r] = 0u;
-        }
-    }
-    __syncthreads();
     const int lane = threadIdx.x & 31;
     if (threadIdx.x < 32) {
         bool match = false;
         if (lane < k) {
-            const int d = sm.drafts[lane];
-            match = d >= 0 && d < P.V && d == sm.am[lane];
+            const int d = drafts[lane];
+            match = d >= 0 && d < P.V && d == am[lane];
         }
         const unsigned miss = __ballot_sync(FULL_MASK, lane < k && !match);
         const int h = miss ? __ffs(miss) - 1 : k;
         for (int i = lane; i <= k; i += 32) {
             int tokv = -1;
-            if (i < h) tokv = sm.drafts[i];
-            else if (i == h) tokv = sm.am[h];
+            if (i < h) tokv = drafts[i];
+            else if (i == h) tokv = am[h];
             P.out_tokens[b * (k + 1) + i] = tokv;
         }
         if (lane == 0) P.accept_len[b] = h;
     }
+}
+
+template <class Tag, class Smem>
+__device__ void epilogue_greedy(const Pass1Params& P, int64_t b, Smem& sm) {
+    const int k = P.k;
+    // The drafts are loaded into registers first and stored after the merge
+    // has issued its loads, so the two round trips overlap.
+    const int dr = threadIdx.x < k ? P.drafts[b * k + threadIdx.x] : 0;
+    merge_argmax_rows<Tag>(P, b * (k + 1), k + 1, sm.rowkey);
+    if (threadIdx.x <= k) sm.am[threadIdx.x] = key_index(sm.rowkey[threadIdx.x]);
+    if (threadIdx.x < k) sm.drafts[threadIdx.x] = dr;
+    __syncthreads();
+    greedy_accept(P, b, sm.drafts, sm.am);
 }
 
 template <class Tag>
@@ -895,7 +855,7 @@ template <class Tag, int MODE, class Smem>
 __device__ __forceinline__ void run_epilogue(const Pass1Params& P, int64_t b, Smem& sm) {
     if constexpr (MODE == MODE_TREE) epilogue_tree<Tag>(P, b, sm);
     else if constexpr (MODE == MODE_SOFTMAX) epilogue_rejection<Tag>(P, b, sm);
-    else epilogue_greedy<Tag, MODE>(P, b, sm);
+    else epilogue_greedy<Tag>(P, b, sm);
 }
 
 // Softmax statistics of one chunk (the rejection pass): the thread's vectors
@@ -1017,10 +977,48 @@ __global__ void __launch_bounds__(NT, MODE == MODE_TOP8 ? 4 : 1) verify_pass1_ke
 // Request epilogues as their own kernel (one CTA per request), after the pass.
 template <class Tag, int MODE>
 __global__ void __launch_bounds__(NT) verify_epilogue_kernel(const Pass1Params P) {
-    __shared__ typename EpiSmemFor<MODE>::type sm;
+    __shared__ typename SmemFor<MODE>::type sm;
     grid_dependency_wait();
     grid_launch_dependents();
     run_epilogue<Tag, MODE>(P, blockIdx.x, sm);
+}
+
+// Greedy top-8 request epilogue, one CTA per request of 32 * min(k + 1, 16)
+// threads: one warp per row (rows beyond 16 take a second turn), then the
+// top-k outputs (values re-read at the winning indices, so they are the
+// stored bits), the row thresholds back to zero, and the accept scan.
+template <class Tag>
+__global__ void __launch_bounds__(32 * kTop8EpiWarps) verify_top8_epilogue_kernel(const Pass1Params P) {
+    __shared__ Top8EpiSmem sm;
+    const int k = P.k, n = k + 1;
+    const int nthreads = static_cast<int>(blockDim.x), nw = nthreads >> 5;
+    const int wp = threadIdx.x >> 5;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int64_t b = blockIdx.x;
+    const int dr = static_cast<int>(threadIdx.x) < k ? P.drafts[b * k + threadIdx.x] : 0;
+    for (int t = wp; t < n; t += nw) row_top8_warp<Tag>(P, b * n + t, sm.surv[wp], sm.top[t]);
+    if (static_cast<int>(threadIdx.x) < k) sm.drafts[threadIdx.x] = dr;
+    __syncthreads();
+    for (int o = threadIdx.x; o < n * 8; o += nthreads) {
+        const int t = o >> 3, e = o & 7;
+        const int64_t r = b * n + t;
+        const uint64_t key = sm.top[t][e];
+        if (e == 0) sm.am[t] = key_index(key);
+        if (e < P.topk) {
+            int id = -1;
+            float val = __uint_as_float(0x7fc00000u);
+            if (key != 0ull) {
+                id = key_index(key);
+                val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + id);
+            }
+            P.topk_ids[r * P.topk + e] = id;
+            P.topk_vals[r * P.topk + e] = val;
+        }
+        if (e == 0 && r < kThetaRows) P.theta_row[r] = 0u;
+    }
+    __syncthreads();
+    greedy_accept(P, b, sm.drafts, sm.am);
 }
 
 }  // namespace specdec
