@@ -28,7 +28,7 @@ constexpr size_t kPartialBase = kThetaBase + static_cast<size_t>(kThetaRows) * s
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-    int64_t nv = 0, nv_full = 0, cpr = 0, NC = 0;
+    int64_t nv = 0, nv_full = 0, cpr = 0, NC = 0, cpr2 = 0;
     size_t partials1 = 0, state = 0, masses = 0, units = 0, total = 0;
 };
 
@@ -47,10 +47,11 @@ Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t
     if (rejection) {
         L.state = align_up(end, 256);
         end = L.state + static_cast<size_t>(B) * sizeof(RejState);
+        L.cpr2 = chunks_per_row(L.nv_full, vec, kU2);
         L.masses = align_up(end, 256);
-        end = L.masses + static_cast<size_t>(B) * static_cast<size_t>(L.cpr) * sizeof(double2);
+        end = L.masses + static_cast<size_t>(B) * static_cast<size_t>(L.cpr2) * sizeof(double2);
         L.units = align_up(end, 256);
-        end = L.units + static_cast<size_t>(B) * static_cast<size_t>(L.cpr) *
+        end = L.units + static_cast<size_t>(B) * static_cast<size_t>(L.cpr2) *
                             static_cast<size_t>(units_per_chunk(vec)) * sizeof(double2);
     }
     (void)rows_per_req;
@@ -334,7 +335,7 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
     Q.q_stride = q_row_stride;
     Q.V = V;
     Q.nv_full = static_cast<int>(L.nv_full);
-    Q.cpr = static_cast<int>(L.cpr);
+    Q.cpr = static_cast<int>(L.cpr2);
     Q.B = B;
     Q.k = k;
     Q.invT = static_cast<float>(invT_d);

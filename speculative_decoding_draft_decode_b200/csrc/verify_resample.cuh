@@ -34,8 +34,16 @@
 
 namespace specdec {
 
+// The resample pass's chunks: kU2 vectors per thread (half the streaming
+// pass's), so its grid of B x chunks holds enough CTAs to balance the SMs
+// even for a few requests.
+#ifndef SPECDEC_RESAMPLE_U
+#define SPECDEC_RESAMPLE_U 4
+#endif
+constexpr int kU2 = SPECDEC_RESAMPLE_U;
+
 // Units per chunk, plus one slot for the ragged row end (last chunk only).
-__host__ __device__ constexpr int units_per_chunk(int vec) { return chunk_upt(vec) * NWARPS + 1; }
+__host__ __device__ constexpr int units_per_chunk(int vec) { return chunk_upt(vec, kU2) * NWARPS + 1; }
 
 struct Pass2Params {
     const void* logits;
@@ -124,35 +132,28 @@ __device__ __forceinline__ Pass2Row pass2_row(const Pass2Params& P, int64_t b, c
     return R;
 }
 
-// Warp-collective transpose-reduce of 16 values per lane: lane L returns the
-// warp total of value (L >> 1) & 15 (each total lands in two lanes).  Four
-// halving exchanges and one full one: 16 shuffles instead of 16 x 5.
-__device__ __forceinline__ double warp_sum16(double (&v)[16]) {
+// Warp-collective transpose-reduce of N values per lane (N a power of two,
+// 2 <= N <= 16): lane L returns the warp total of value
+// (L >> (5 - log2 N)) & (N - 1), each total landing in 32 / N lanes.  The
+// halving exchanges over lane bits 4, 3, ... each pass half of the values
+// still held; the rest add the partner lanes: N - 1 + 5 - log2 N shuffles
+// instead of 5 N.
+template <int N>
+__device__ __forceinline__ double warp_sum_transpose(double (&v)[N]) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const bool hi = (lane & 16) != 0;
-        const double send = hi ? v[i] : v[i + 8];
-        v[i] = (hi ? v[i + 8] : v[i]) + __shfl_xor_sync(FULL_MASK, send, 16);
-    }
+    for (int h = N / 2, off = 16; h >= 1; h >>= 1, off >>= 1) {
+        const bool hi = (lane & off) != 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const bool hi = (lane & 8) != 0;
-        const double send = hi ? v[i] : v[i + 4];
-        v[i] = (hi ? v[i + 4] : v[i]) + __shfl_xor_sync(FULL_MASK, send, 8);
+        for (int i = 0; i < h; ++i) {
+            const double send = hi ? v[i] : v[i + h];
+            v[i] = (hi ? v[i + h] : v[i]) + __shfl_xor_sync(FULL_MASK, send, off);
+        }
     }
+    constexpr int kFirstFull = 32 / N;  // the lane bits below the value index
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const bool hi = (lane & 4) != 0;
-        const double send = hi ? v[i] : v[i + 2];
-        v[i] = (hi ? v[i + 2] : v[i]) + __shfl_xor_sync(FULL_MASK, send, 4);
-    }
-    {
-        const bool hi = (lane & 2) != 0;
-        const double send = hi ? v[0] : v[1];
-        v[0] = (hi ? v[1] : v[0]) + __shfl_xor_sync(FULL_MASK, send, 2);
-    }
-    return v[0] + __shfl_xor_sync(FULL_MASK, v[0], 1);
+    for (int off = kFirstFull / 2; off >= 1; off >>= 1) v[0] += __shfl_xor_sync(FULL_MASK, v[0], off);
+    return v[0];
 }
 
 // ---------------------------------------------------------------------------
@@ -164,10 +165,12 @@ template <class Tag, int VEC>
 __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P) {
     __shared__ double red[2][NWARPS];
     using Elem = typename Tag::storage;
-    constexpr int CH = chunk_vecs(VEC);
-    constexpr int UPT = chunk_upt(VEC);
+    constexpr int CH = chunk_vecs(VEC, kU2);
+    constexpr int UPT = chunk_upt(VEC, kU2);
     constexpr int UPC = units_per_chunk(VEC);
-    static_assert(kU == 8, "the unit transpose-reduce takes 8 vectors per thread per batch");
+    constexpr int NV = 2 * kU2;        // masses per batch: r and p of kU2 vectors
+    constexpr int kShift = 5 - (NV == 16 ? 4 : NV == 8 ? 3 : NV == 4 ? 2 : 1);
+    static_assert(NV == 2 || NV == 4 || NV == 8 || NV == 16, "kU2 must be 1, 2, 4 or 8");
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const int t = static_cast<int>(threadIdx.x);
 
@@ -180,20 +183,20 @@ __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P
     if (!st.valid) return;  // CTA-uniform
     const Pass2Row R = pass2_row<Tag>(P, b, st);
     const Elem* row = static_cast<const Elem*>(R.row);
-    const int cnt = chunk_count(P.nv_full, sub, VEC);
+    const int cnt = chunk_count(P.nv_full, sub, VEC, kU2);
     double2* um = P.unit_mass + (b * P.cpr + sub) * UPC;
 
     double sr = 0.0, sp = 0.0;
-    for (int u0 = 0; u0 < UPT; u0 += kU) {
-        ResidualVec<Tag, VEC> v[kU];
+    for (int u0 = 0; u0 < UPT; u0 += kU2) {
+        ResidualVec<Tag, VEC> v[kU2];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
+        for (int u = 0; u < kU2; ++u) {
             const int i = stream_pos(u0 + u, t);
             if (i < cnt) v[u].load(row, R.qrow, sub * CH + i, R.has_q);
         }
-        double m[16];
+        double m[NV];
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
+        for (int u = 0; u < kU2; ++u) {
             double ar = 0.0, ap = 0.0;
             if (stream_pos(u0 + u, t) < cnt) {
                 float p[VEC], r[VEC];
@@ -205,17 +208,17 @@ __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P
                 }
             }
             m[u] = ar;
-            m[kU + u] = ap;
+            m[kU2 + u] = ap;
             sr += ar;
             sp += ap;
         }
         // Unit (u, warp) is the 32 vectors u*NT + warp*32 + [0, 32); its index
         // in the chunk is u*NWARPS + warp, which is index order.
-        const double tot = warp_sum16(m);
-        const int which = (lane >> 1) & 15;
-        if ((lane & 1) == 0) {
-            double* dst = reinterpret_cast<double*>(&um[(u0 + (which & 7)) * NWARPS + wp]);
-            dst[which >> 3] = tot;
+        const double tot = warp_sum_transpose<NV>(m);
+        const int which = (lane >> kShift) & (NV - 1);
+        if ((lane & ((1 << kShift) - 1)) == 0) {
+            double* dst = reinterpret_cast<double*>(&um[(u0 + which % kU2) * NWARPS + wp]);
+            dst[which / kU2] = tot;
         }
     }
     // The ragged row end (fewer than VEC elements): lanes of warp 0, stored
@@ -343,7 +346,7 @@ __device__ __forceinline__ int warp_find_level(const double2* m, int n, bool use
 template <class Tag, int VEC>
 __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass2Params P) {
     using Elem = typename Tag::storage;
-    constexpr int CH = chunk_vecs(VEC);
+    constexpr int CH = chunk_vecs(VEC, kU2);
     constexpr int UPC = units_per_chunk(VEC);
     const int lane = threadIdx.x & 31;
 
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
             const int pos = stream_pos(u, w * 32 + lane);
             const int j = chunk * CH + pos;
             x0 = j * VEC;
-            if (pos < chunk_count(P.nv_full, chunk, VEC)) {
+            if (pos < chunk_count(P.nv_full, chunk, VEC, kU2)) {
                 nx = VEC;
                 ResidualVec<Tag, VEC> v;
                 v.load(row, R.qrow, j, R.has_q);
