@@ -403,6 +403,67 @@ CONFIGS = {
 }
 
 
+@dataclass
+class RaggedInputs:
+    """Inputs of one verify call in the packed layout of variable speculation
+    lengths: request b owns drafts [offsets[b], offsets[b+1]) (k_b of them)
+    and the k_b + 1 logit rows starting at row offsets[b] + b.
+
+    logits: [R, V] with R = B + offsets[-1]; drafts: [offsets[-1]] int32;
+    offsets: [B+1] int32; q (rejection only): [offsets[-1], V] float32.
+    """
+    name: str
+    dtype: str
+    logits: np.ndarray
+    drafts: np.ndarray
+    offsets: np.ndarray
+    B: int
+    max_k: int
+    V: int
+    topk: int = 0
+    q: Optional[np.ndarray] = None
+    temperature: float = 1.0
+    seed: int = 1234
+    offset: int = 0
+
+    @property
+    def rows(self) -> int:
+        return self.B + int(self.offsets[-1])
+
+
+def pack_ragged(name, dtype, logits, drafts, kb, max_k, q=None, **kw) -> RaggedInputs:
+    """Pack fixed-layout inputs ([B, K+1, V] logits, [B, K] drafts, optional
+    [B, K, V] q) into the ragged layout, keeping request b's first kb[b]
+    drafts and kb[b] + 1 rows."""
+    kb = np.asarray(kb, np.int64)
+    B = len(kb)
+    offsets = np.zeros(B + 1, np.int32)
+    offsets[1:] = np.cumsum(kb)
+    rows = np.concatenate([logits[b, :kb[b] + 1] for b in range(B)]) if B else logits.reshape(0, logits.shape[-1])
+    d = np.concatenate([drafts[b, :kb[b]] for b in range(B)]).astype(np.int32) if B else np.zeros(0, np.int32)
+    qq = None
+    if q is not None:
+        qq = np.concatenate([q[b, :kb[b]] for b in range(B)]) if B else q.reshape(0, q.shape[-1])
+    return RaggedInputs(name, dtype, np.ascontiguousarray(rows), d, offsets, B, int(max_k), logits.shape[-1],
+                        q=None if qq is None else np.ascontiguousarray(qq, dtype=np.float32), **kw)
+
+
+def greedy_ragged_tiers(seed: int = 6, B: int = 64, tiers=(1, 3, 7), V: int = LLAMA3_VOCAB, alpha: float = 0.8,
+                        dtype: str = BF16, topk: int = 0) -> RaggedInputs:
+    """Greedy verify with a speculation length per request drawn uniformly from
+    SGLang's default tiers [1, 3, 7] (handbook page, "Adaptive speculative
+    decoding"), packed; logits and draft agreement as in the Llama-3 greedy
+    workload (N(0, sigma^2) + 8 at one uniform token per row, drafts agree
+    w.p. alpha per position)."""
+    rng = np.random.default_rng(seed)
+    kb = rng.choice(np.asarray(tiers, np.int64), size=B)
+    K = int(max(tiers))
+    base = greedy_llama3(seed + 1000, B, K, V, alpha, dtype)
+    r = pack_ragged("greedy_ragged_tiers", dtype, base.logits, base.drafts, kb, K)
+    r.topk = topk
+    return r
+
+
 def algorithmic_bytes(inp) -> int:
     """Bytes one verify call must move: one read of every logit row the mode
     needs, the gathers, and the outputs (the rejection pass-2 row re-read is
@@ -420,4 +481,9 @@ def algorithmic_bytes(inp) -> int:
         R = inp.B * (inp.k + 1)
         out = inp.B * 4 + inp.B * (inp.k + 1) * 4
         return R * inp.V * es + inp.B * inp.k * 4 + 2 * inp.B * inp.k * 4 + out
+    if isinstance(inp, RaggedInputs):
+        R, T = inp.rows, int(inp.offsets[-1])
+        out = inp.B * 4 + R * 4 + R * inp.topk * 8
+        extra = 2 * T * 4 if inp.q is not None else 0
+        return R * inp.V * es + T * 4 + (inp.B + 1) * 4 + extra + out
     raise TypeError(type(inp))

@@ -138,6 +138,155 @@ void uniforms(uint64_t seed, uint64_t offset, uint32_t b, uint32_t i, double* u_
 
 }  // namespace
 
+namespace {
+
+// The topk largest elements of row r (value descending, index ascending on
+// ties; NaN lowest) into ids[0..topk) / vals[0..topk); -1 / NaN past V.
+void topk_row(const void* logits, int dtype, int64_t row_stride, int64_t r, int V, int topk, int32_t* ids,
+              float* vals) {
+    std::vector<int32_t> idx(V);
+    for (int x = 0; x < V; ++x) idx[x] = x;
+    auto before = [&](int32_t a, int32_t b) {
+        int c = logit_cmp(logit_at(logits, dtype, row_stride, r, a), logit_at(logits, dtype, row_stride, r, b));
+        return c > 0 || (c == 0 && a < b);
+    };
+    int m = std::min(topk, V);
+    std::partial_sort(idx.begin(), idx.begin() + m, idx.end(), before);
+    for (int j = 0; j < topk; ++j) {
+        if (j < m) {
+            ids[j] = idx[j];
+            vals[j] = logit_at(logits, dtype, row_stride, r, idx[j]);
+        } else {
+            ids[j] = -1;
+            vals[j] = std::numeric_limits<float>::quiet_NaN();
+        }
+    }
+}
+
+// One request of the greedy verifier: rows row0 .. row0 + k of `logits`,
+// drafts d[0..k).  h = the number of leading drafts equal to the target's
+// greedy choice at their position; out[0..k] = d_0..d_{h-1}, the target's
+// choice at position h (the correction or bonus token), then -1.
+// [HANDBOOK] "How does speculative decoding work", steps 2-4; [VLLM]
+// section 1; [ARCTIC] "Verifier optimisation" and "A Simple Example".
+void greedy_request(const void* logits, int dtype, int64_t row_stride, int64_t row0, const int32_t* d, int k,
+                    int V, int32_t* accept_len, int32_t* out) {
+    std::vector<int32_t> am(k + 1);
+    for (int j = 0; j <= k; ++j) am[j] = row_argmax(logits, dtype, row_stride, row0 + j, V);
+    int h = 0;
+    while (h < k) {
+        if (d[h] < 0 || d[h] >= V || d[h] != am[h]) break;  // first disagreement stops the scan
+        ++h;
+    }
+    *accept_len = h;
+    for (int i = 0; i <= k; ++i) {
+        if (i < h) out[i] = d[i];
+        else if (i == h) out[i] = am[h];
+        else out[i] = -1;
+    }
+}
+
+// The acceptance counters of one valid request with k drafts, h accepted.
+void count_request(int64_t* ctr, int k, int h) {
+    ctr[0] += 1;
+    ctr[1] += k;
+    ctr[2] += h;
+    for (int i = 0; i < h; ++i) ctr[3 + i] += 1;
+}
+
+// One request of the rejection verifier: target rows row0 .. row0 + k, q rows
+// q0 .. q0 + k - 1, drafts d[0..k), uniforms of request index b.  Writes
+// accept_len, out[0..k], p_draft[0..k), margin (see oracle_verify_rejection).
+void rejection_request(const void* target, int dtype, int64_t row_stride, int64_t row0, const float* q,
+                       int64_t q_row_stride, int64_t q0, const int32_t* d, int k, int V, double T, uint64_t seed,
+                       uint64_t offset, uint32_t b, int32_t* accept_len, int32_t* out, double* p_draft,
+                       double* margin) {
+    std::vector<double> m(k + 1), Z(k + 1), r(V);
+    // 1. softmax statistics of every target row of the request
+    bool valid = true;
+    for (int i = 0; i <= k; ++i) {
+        int64_t row = row0 + i;
+        bool any_above_neg_inf = false, bad = false;
+        double mi = -std::numeric_limits<double>::infinity();
+        for (int x = 0; x < V; ++x) {
+            float l = logit_at(target, dtype, row_stride, row, x);
+            if (std::isnan(l) || (std::isinf(l) && l > 0)) bad = true;
+            if (!(std::isinf(l) && l < 0)) any_above_neg_inf = true;
+            double sx = static_cast<double>(l) / T;
+            if (sx > mi) mi = sx;
+        }
+        if (bad || !any_above_neg_inf) { valid = false; break; }
+        double zi = 0.0;
+        for (int x = 0; x < V; ++x) {
+            double sx = static_cast<double>(logit_at(target, dtype, row_stride, row, x)) / T;
+            zi += std::exp(sx - mi);
+        }
+        m[i] = mi;
+        Z[i] = zi;
+    }
+    if (!valid) {
+        *accept_len = -1;
+        for (int i = 0; i <= k; ++i) out[i] = -1;
+        for (int i = 0; i < k; ++i) p_draft[i] = std::numeric_limits<double>::quiet_NaN();
+        *margin = std::numeric_limits<double>::infinity();
+        return;
+    }
+    auto p_of = [&](int i, int x) {
+        double sx = static_cast<double>(logit_at(target, dtype, row_stride, row0 + i, x)) / T;
+        return std::exp(sx - m[i]) / Z[i];
+    };
+    auto q_of = [&](int i, int x) { return static_cast<double>(q[(q0 + i) * q_row_stride + x]); };
+    for (int i = 0; i < k; ++i) p_draft[i] = (d[i] >= 0 && d[i] < V) ? p_of(i, d[i]) : 0.0;
+
+    // 2. accept test, position by position
+    double mg = std::numeric_limits<double>::infinity();
+    int h = 0;
+    for (; h < k; ++h) {
+        double ua, ur;
+        uniforms(seed, offset, b, (uint32_t)h, &ua, &ur);
+        if (d[h] < 0 || d[h] >= V) break;
+        double p = p_draft[h];
+        double qd = q_of(h, d[h]);
+        mg = std::min(mg, qd > 0.0 ? std::fabs(ua - p / qd) : p);
+        if (!(ua * qd < p)) break;
+    }
+    // 3. the correction (h < k) or bonus (h = k) token
+    double ua, ur;
+    uniforms(seed, offset, b, (uint32_t)h, &ua, &ur);
+    double S = 0.0;
+    if (h < k) {
+        for (int x = 0; x < V; ++x) { r[x] = std::max(0.0, p_of(h, x) - q_of(h, x)); S += r[x]; }
+        mg = std::min(mg, S);
+        if (!(S > 0.0)) {
+            S = 0.0;
+            for (int x = 0; x < V; ++x) { r[x] = p_of(h, x); S += r[x]; }
+        }
+    } else {
+        for (int x = 0; x < V; ++x) { r[x] = p_of(k, x); S += r[x]; }
+    }
+    double t = ur * S;
+    double c = 0.0, prev = 0.0;
+    int tokv = -1;
+    for (int x = 0; x < V; ++x) {
+        prev = c;
+        c += r[x];
+        if (c > t) { tokv = x; break; }
+    }
+    if (tokv < 0) {
+        for (int x = V - 1; x >= 0; --x)
+            if (r[x] > 0.0) { tokv = x; break; }
+        if (tokv < 0) tokv = V - 1;
+        mg = 0.0;
+    } else {
+        mg = std::min(mg, std::min(t - prev, c - t) / S);
+    }
+    *accept_len = h;
+    for (int i = 0; i <= k; ++i) out[i] = (i < h) ? d[i] : (i == h ? tokv : -1);
+    *margin = mg;
+}
+
+}  // namespace
+
 extern "C" {
 
 // Philox block function, exported for the pins.
@@ -159,25 +308,7 @@ void oracle_argmax_rows(const void* logits, int dtype, int64_t row_stride, int64
 // row under that order.  Values are the stored logits widened exactly.
 void oracle_topk_rows(const void* logits, int dtype, int64_t row_stride, int64_t R, int V, int topk,
                       int32_t* ids, float* vals) {
-    std::vector<int32_t> idx(V);
-    for (int64_t r = 0; r < R; ++r) {
-        for (int x = 0; x < V; ++x) idx[x] = x;
-        auto before = [&](int32_t a, int32_t b) {
-            int c = logit_cmp(logit_at(logits, dtype, row_stride, r, a), logit_at(logits, dtype, row_stride, r, b));
-            return c > 0 || (c == 0 && a < b);
-        };
-        int m = std::min(topk, V);
-        std::partial_sort(idx.begin(), idx.begin() + m, idx.end(), before);
-        for (int j = 0; j < topk; ++j) {
-            if (j < m) {
-                ids[r * topk + j] = idx[j];
-                vals[r * topk + j] = logit_at(logits, dtype, row_stride, r, idx[j]);
-            } else {
-                ids[r * topk + j] = -1;
-                vals[r * topk + j] = std::numeric_limits<float>::quiet_NaN();
-            }
-        }
-    }
+    for (int64_t r = 0; r < R; ++r) topk_row(logits, dtype, row_stride, r, V, topk, ids + r * topk, vals + r * topk);
 }
 
 // Greedy verification of B requests with k drafts each.
@@ -193,25 +324,51 @@ void oracle_topk_rows(const void* logits, int dtype, int64_t row_stride, int64_t
 void oracle_verify_greedy(const void* logits, int dtype, int64_t row_stride, const int32_t* drafts,
                           int B, int k, int V, int32_t* accept_len, int32_t* out_tokens,
                           int topk, int32_t* topk_ids, float* topk_vals) {
-    std::vector<int32_t> am(k + 1);
-    for (int b = 0; b < B; ++b) {
-        for (int j = 0; j <= k; ++j) am[j] = row_argmax(logits, dtype, row_stride, (int64_t)b * (k + 1) + j, V);
-        int h = 0;
-        while (h < k) {
-            int32_t d = drafts[(int64_t)b * k + h];
-            if (d < 0 || d >= V || d != am[h]) break;  // first disagreement stops the scan
-            ++h;
-        }
-        accept_len[b] = h;
-        int32_t* out = out_tokens + (int64_t)b * (k + 1);
-        for (int i = 0; i <= k; ++i) {
-            if (i < h) out[i] = drafts[(int64_t)b * k + i];
-            else if (i == h) out[i] = am[h];
-            else out[i] = -1;
-        }
-    }
+    for (int b = 0; b < B; ++b)
+        greedy_request(logits, dtype, row_stride, (int64_t)b * (k + 1), drafts + (int64_t)b * k, k, V,
+                       &accept_len[b], out_tokens + (int64_t)b * (k + 1));
     if (topk > 0)
         oracle_topk_rows(logits, dtype, row_stride, (int64_t)B * (k + 1), V, topk, topk_ids, topk_vals);
+}
+
+// Greedy verification with a draft count of its own per request, in the
+// packed layout serving engines use for variable speculation lengths
+// ([HANDBOOK] "Adaptive speculative decoding": the speculation length changes
+// per batch or request, e.g. SGLang's tiers), with the acceptance counters
+// of [VLLM] section 3, result 4 (accepted tokens in total and per draft
+// position, and draft tokens in total).
+//   draft_offsets [B+1]  request b owns drafts [off[b], off[b+1]); k_b =
+//                        off[b+1] - off[b]; its k_b + 1 logit rows and output
+//                        slots start at row off[b] + b.  A request whose
+//                        offsets are not 0 <= off[b] <= off[b+1] <= off[B]
+//                        with k_b <= max_k is invalid: accept_len -1 and
+//                        nothing else written for it.
+//   logits        [B + off[B], V]; drafts [off[B]]
+//   out_tokens    [B + off[B]]; topk_ids / topk_vals [B + off[B], topk]
+//   counters      [3 + max_k] int64 or NULL, accumulated over valid requests:
+//                 [0] requests, [1] draft tokens (sum of k_b), [2] accepted
+//                 tokens (sum of h), [3 + i] requests whose draft i was
+//                 accepted (h > i).
+void oracle_verify_greedy_ragged(const void* logits, int dtype, int64_t row_stride, const int32_t* drafts,
+                                 const int32_t* draft_offsets, int B, int max_k, int V,
+                                 int32_t* accept_len, int32_t* out_tokens, int topk, int32_t* topk_ids,
+                                 float* topk_vals, int64_t* counters) {
+    const int64_t total = B > 0 ? draft_offsets[B] : 0;
+    for (int b = 0; b < B; ++b) {
+        const int64_t o0 = draft_offsets[b], o1 = draft_offsets[b + 1];
+        if (!(o0 >= 0 && o0 <= o1 && o1 <= total && o1 - o0 <= max_k)) {
+            accept_len[b] = -1;
+            continue;
+        }
+        const int kb = static_cast<int>(o1 - o0);
+        const int64_t row0 = o0 + b;
+        greedy_request(logits, dtype, row_stride, row0, drafts + o0, kb, V, &accept_len[b], out_tokens + row0);
+        if (topk > 0)
+            for (int i = 0; i <= kb; ++i)
+                topk_row(logits, dtype, row_stride, row0 + i, V, topk, topk_ids + (row0 + i) * topk,
+                         topk_vals + (row0 + i) * topk);
+        if (counters) count_request(counters, kb, accept_len[b]);
+    }
 }
 
 // Greedy verification of a draft tree per request.
@@ -296,96 +453,37 @@ void oracle_verify_rejection(const void* target, int dtype, int64_t row_stride,
                              const float* q, int64_t q_row_stride, const int32_t* drafts,
                              int B, int k, int V, double temperature, uint64_t seed, uint64_t offset,
                              int32_t* accept_len, int32_t* out_tokens, double* p_draft, double* margin) {
-    const double T = temperature;
-    std::vector<double> m(k + 1), Z(k + 1), r(V);
+    for (int b = 0; b < B; ++b)
+        rejection_request(target, dtype, row_stride, (int64_t)b * (k + 1), q, q_row_stride, (int64_t)b * k,
+                          drafts + (int64_t)b * k, k, V, temperature, seed, offset, (uint32_t)b, &accept_len[b],
+                          out_tokens + (int64_t)b * (k + 1), p_draft + (int64_t)b * k, &margin[b]);
+}
+
+// Rejection-sampling verification in the packed layout of
+// oracle_verify_greedy_ragged: request b's k_b + 1 target rows and output
+// slots start at row off[b] + b, its q rows and p_draft entries at off[b];
+// the uniforms are those of (request b, position i) as in the fixed layout.
+// An invalid request (offsets out of order or k_b > max_k) gets accept_len
+// -1 and nothing else written; counters as in the greedy case, over the
+// requests whose distributions are defined.
+void oracle_verify_rejection_ragged(const void* target, int dtype, int64_t row_stride, const float* q,
+                                    int64_t q_row_stride, const int32_t* drafts, const int32_t* draft_offsets,
+                                    int B, int max_k, int V, double temperature, uint64_t seed, uint64_t offset,
+                                    int32_t* accept_len, int32_t* out_tokens, double* p_draft, double* margin,
+                                    int64_t* counters) {
+    const int64_t total = B > 0 ? draft_offsets[B] : 0;
     for (int b = 0; b < B; ++b) {
-        int32_t* out = out_tokens + (int64_t)b * (k + 1);
-        const int32_t* d = drafts + (int64_t)b * k;
-        // 1. softmax statistics of every target row of the request
-        bool valid = true;
-        for (int i = 0; i <= k; ++i) {
-            int64_t row = (int64_t)b * (k + 1) + i;
-            bool any_above_neg_inf = false, bad = false;
-            double mi = -std::numeric_limits<double>::infinity();
-            for (int x = 0; x < V; ++x) {
-                float l = logit_at(target, dtype, row_stride, row, x);
-                if (std::isnan(l) || (std::isinf(l) && l > 0)) bad = true;
-                if (!(std::isinf(l) && l < 0)) any_above_neg_inf = true;
-                double s = static_cast<double>(l) / T;
-                if (s > mi) mi = s;
-            }
-            if (bad || !any_above_neg_inf) { valid = false; break; }
-            double zi = 0.0;
-            for (int x = 0; x < V; ++x) {
-                double s = static_cast<double>(logit_at(target, dtype, row_stride, row, x)) / T;
-                zi += std::exp(s - mi);
-            }
-            m[i] = mi;
-            Z[i] = zi;
-        }
-        if (!valid) {
+        const int64_t o0 = draft_offsets[b], o1 = draft_offsets[b + 1];
+        if (!(o0 >= 0 && o0 <= o1 && o1 <= total && o1 - o0 <= max_k)) {
             accept_len[b] = -1;
-            for (int i = 0; i <= k; ++i) out[i] = -1;
-            for (int i = 0; i < k; ++i) p_draft[(int64_t)b * k + i] = std::numeric_limits<double>::quiet_NaN();
             margin[b] = std::numeric_limits<double>::infinity();
             continue;
         }
-        auto p_of = [&](int i, int x) {
-            int64_t row = (int64_t)b * (k + 1) + i;
-            double s = static_cast<double>(logit_at(target, dtype, row_stride, row, x)) / T;
-            return std::exp(s - m[i]) / Z[i];
-        };
-        auto q_of = [&](int i, int x) {
-            return static_cast<double>(q[((int64_t)b * k + i) * q_row_stride + x]);
-        };
-        for (int i = 0; i < k; ++i)
-            p_draft[(int64_t)b * k + i] = (d[i] >= 0 && d[i] < V) ? p_of(i, d[i]) : 0.0;
-
-        // 2. accept test, position by position
-        double mg = std::numeric_limits<double>::infinity();
-        int h = 0;
-        for (; h < k; ++h) {
-            double ua, ur;
-            uniforms(seed, offset, (uint32_t)b, (uint32_t)h, &ua, &ur);
-            if (d[h] < 0 || d[h] >= V) break;
-            double p = p_draft[(int64_t)b * k + h];
-            double qd = q_of(h, d[h]);
-            mg = std::min(mg, qd > 0.0 ? std::fabs(ua - p / qd) : p);
-            if (!(ua * qd < p)) break;
-        }
-        // 3. the correction (h < k) or bonus (h = k) token
-        double ua, ur;
-        uniforms(seed, offset, (uint32_t)b, (uint32_t)h, &ua, &ur);
-        double S = 0.0;
-        if (h < k) {
-            for (int x = 0; x < V; ++x) { r[x] = std::max(0.0, p_of(h, x) - q_of(h, x)); S += r[x]; }
-            mg = std::min(mg, S);
-            if (!(S > 0.0)) {
-                S = 0.0;
-                for (int x = 0; x < V; ++x) { r[x] = p_of(h, x); S += r[x]; }
-            }
-        } else {
-            for (int x = 0; x < V; ++x) { r[x] = p_of(k, x); S += r[x]; }
-        }
-        double t = ur * S;
-        double c = 0.0, prev = 0.0;
-        int tokv = -1;
-        for (int x = 0; x < V; ++x) {
-            prev = c;
-            c += r[x];
-            if (c > t) { tokv = x; break; }
-        }
-        if (tokv < 0) {
-            for (int x = V - 1; x >= 0; --x)
-                if (r[x] > 0.0) { tokv = x; break; }
-            if (tokv < 0) tokv = V - 1;
-            mg = 0.0;
-        } else {
-            mg = std::min(mg, std::min(t - prev, c - t) / S);
-        }
-        accept_len[b] = h;
-        for (int i = 0; i <= k; ++i) out[i] = (i < h) ? d[i] : (i == h ? tokv : -1);
-        margin[b] = mg;
+        const int kb = static_cast<int>(o1 - o0);
+        const int64_t row0 = o0 + b;
+        rejection_request(target, dtype, row_stride, row0, q, q_row_stride, o0, drafts + o0, kb, V, temperature,
+                          seed, offset, (uint32_t)b, &accept_len[b], out_tokens + row0, p_draft + o0, &margin[b]);
+        if (counters && accept_len[b] >= 0) count_request(counters, kb, accept_len[b]);
     }
 }
 

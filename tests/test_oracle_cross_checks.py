@@ -62,16 +62,16 @@ MUTANTS = [
      "                      logit_at(logits, dtype, row_stride, row, best)) >= 0)",
      [lambda: pins.test_argmax_and_topk_match_sorting(7)]),
     ("draft compared with the next row's choice",
-     "if (d < 0 || d >= V || d != am[h]) break;",
-     "if (d < 0 || d >= V || d != am[h + 1]) break;",
+     "if (d[h] < 0 || d[h] >= V || d[h] != am[h]) break;",
+     "if (d[h] < 0 || d[h] >= V || d[h] != am[h + 1]) break;",
      [pins.test_worked_example_greedy, pins.test_greedy_scan_brute_force]),
     ("bonus token taken from the previous row",
      "else if (i == h) out[i] = am[h];",
      "else if (i == h) out[i] = am[h > 0 ? h - 1 : 0];",
      [pins.test_worked_example_greedy, pins.test_all_accept_example]),
     ("scan does not stop at the first disagreement",
-     "if (d < 0 || d >= V || d != am[h]) break;  // first disagreement stops the scan\n            ++h;",
-     "if (d < 0 || d >= V || d != am[h]) { ++h; continue; }\n            ++h;",
+     "if (d[h] < 0 || d[h] >= V || d[h] != am[h]) break;  // first disagreement stops the scan\n        ++h;",
+     "if (d[h] < 0 || d[h] >= V || d[h] != am[h]) { ++h; continue; }\n        ++h;",
      [pins.test_greedy_scan_brute_force]),
     ("NaN ranked above numbers",
      "    if (na) return -1;\n    if (nb) return 1;",
@@ -86,8 +86,8 @@ MUTANTS = [
      "if (!(ua * p < qd)) break;",
      [pins.test_rejection_expected_accept_len]),
     ("temperature multiplies instead of divides",
-     "double s = static_cast<double>(logit_at(target, dtype, row_stride, row, x)) / T;\n            return",
-     "double s = static_cast<double>(logit_at(target, dtype, row_stride, row, x)) * T;\n            return",
+     "double sx = static_cast<double>(logit_at(target, dtype, row_stride, row0 + i, x)) / T;\n        return",
+     "double sx = static_cast<double>(logit_at(target, dtype, row_stride, row0 + i, x)) * T;\n        return",
      [pins.test_rejection_softmax_closed_forms]),
     ("bonus sampled from row k-1",
      "for (int x = 0; x < V; ++x) { r[x] = p_of(k, x); S += r[x]; }",
