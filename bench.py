@@ -85,12 +85,17 @@ def recorded_traffic(workload):
 def make_workload(name, seed_offset=0):
     base = {"greedy_llama3": (gen.greedy_llama3, 1), "greedy_tiny": (gen.greedy_tiny, 0),
             "greedy_large_batch": (gen.greedy_large_batch, 3), "tree_medusa": (gen.tree_medusa, 4),
-            "rejection_qwen": (gen.rejection_qwen, 2)}
+            "rejection_qwen": (gen.rejection_qwen, 2), "greedy_ragged_tiers": (gen.greedy_ragged_tiers, 6)}
     fn, seed = base[name]
     return fn(seed=seed + 1000 * seed_offset)
 
 
 def describe(inp):
+    if isinstance(inp, gen.RaggedInputs):
+        kb = np.diff(inp.offsets)
+        return {"B": inp.B, "max_k": inp.max_k, "V": inp.V, "rows": inp.rows, "drafts": int(inp.offsets[-1]),
+                "k_per_request": "tiers %s, mean %.2f" % (sorted(set(kb.tolist())), kb.mean()),
+                "layout": "packed (draft offsets)", "counters": True}
     if isinstance(inp, gen.TreeInputs):
         return {"B": inp.B, "N": inp.N, "V": inp.V, "rows": inp.B * (inp.N + 1), "max_depth": inp.max_depth}
     d = {"B": inp.B, "k": inp.k, "V": inp.V, "rows": inp.B * (inp.k + 1)}
@@ -101,8 +106,12 @@ def describe(inp):
     return d
 
 
-def rows_of(inp):
-    return inp.B * ((inp.N + 1) if isinstance(inp, gen.TreeInputs) else (inp.k + 1))
+def rows_of(inp, req=None):
+    """Logit rows of the first `req` requests (all by default)."""
+    req = inp.B if req is None else req
+    if isinstance(inp, gen.RaggedInputs):
+        return int(inp.offsets[req]) + req
+    return req * ((inp.N + 1) if isinstance(inp, gen.TreeInputs) else (inp.k + 1))
 
 
 # ---------------------------------------------------------------------------
@@ -126,6 +135,8 @@ def host_tensors(inp):
     if isinstance(inp, gen.RejectionInputs):
         return {"target": logits_t(inp.target, inp.dtype),
                 "q": torch.from_numpy(np.ascontiguousarray(inp.q, dtype=np.float32)), "drafts": i32(inp.drafts)}
+    if isinstance(inp, gen.RaggedInputs):
+        return {"logits": logits_t(inp.logits, inp.dtype), "drafts": i32(inp.drafts), "offsets": i32(inp.offsets)}
     return {"logits": logits_t(inp.logits, inp.dtype), "drafts": i32(inp.drafts)}
 
 
@@ -197,6 +208,18 @@ def setup_calls(inp, sets, ver, device):
             calls.append(lambda s=s: ver.rejection(s["target"], s["q"], s["drafts"], inp.temperature, inp.seed,
                                                    inp.offset, out=outs))
         kernels = 4  # softmax pass, request epilogue, chunk masses, token search
+    elif isinstance(inp, gen.RaggedInputs):
+        R, T = inp.rows, int(inp.offsets[-1])
+        al = torch.empty(B, dtype=torch.int32, device=device)
+        ot = torch.empty(R, dtype=torch.int32, device=device)
+        ids = torch.empty(R, max(inp.topk, 1), dtype=torch.int32, device=device)
+        vals = torch.empty(R, max(inp.topk, 1), dtype=torch.float32, device=device)
+        ctr = torch.zeros(3 + inp.max_k, dtype=torch.int64, device=device)
+        outs = (al, ot, ids, vals, ctr)
+        for s in sets:
+            calls.append(lambda s=s: ver.greedy_ragged(s["logits"], s["drafts"], s["offsets"], T, inp.max_k,
+                                                       topk=inp.topk, counters=ctr, out=outs[:4]))
+        kernels = 2  # streaming pass + request epilogue (acceptance counters fused)
     else:
         k1 = inp.k + 1
         al = torch.empty(B, dtype=torch.int32, device=device)
@@ -448,11 +471,14 @@ def oracle_call(inp, req):
     if isinstance(inp, gen.RejectionInputs):
         return oracle.verify_rejection(inp.target[:req], inp.dtype, inp.q[:req], inp.drafts[:req],
                                        inp.temperature, inp.seed, inp.offset)
+    if isinstance(inp, gen.RaggedInputs):
+        t = int(inp.offsets[req])
+        return oracle.verify_greedy_ragged(inp.logits[:t + req], inp.dtype, inp.drafts[:t], inp.offsets[:req + 1],
+                                           inp.max_k, topk=inp.topk)
     return oracle.verify_greedy(inp.logits[:req], inp.dtype, inp.drafts[:req], topk=inp.topk)
 
 
 def time_oracle(inp, seconds):
-    rpr = rows_of(inp) // inp.B
     t0 = time.perf_counter()
     oracle_call(inp, 1)
     one = max(time.perf_counter() - t0, 1e-6)
@@ -462,7 +488,7 @@ def time_oracle(inp, seconds):
         t0 = time.perf_counter()
         oracle_call(inp, req)
         el += time.perf_counter() - t0
-        rows += req * rpr
+        rows += rows_of(inp, req)
     return rows / el, req, rows
 
 
@@ -481,7 +507,7 @@ def run_reference(args):
     budget = 120.0
     # each step verifies a bounded sample of requests so the run fits the budget
     v1, req1, _ = time_oracle(inp, 2.0)
-    rpr = rows_of(inp) // inp.B
+    rpr = rows_of(inp) / inp.B
     step_budget = budget / max(1, args.steps + args.warmup)
     req = int(max(1, min(inp.B, step_budget * v1 / rpr)))
     for _ in range(args.warmup):
@@ -490,7 +516,7 @@ def run_reference(args):
     for _ in range(args.steps):
         oracle_call(inp, req)
     el = time.perf_counter() - t0
-    value = req * rpr * args.steps / el
+    value = rows_of(inp, req) * args.steps / el
     sample = "first %d of %d requests per step, single-threaded fp64 C++ oracle" % (req, inp.B)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
@@ -508,7 +534,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="greedy_llama3",
-                    choices=["greedy_llama3", "greedy_tiny", "rejection_qwen", "greedy_large_batch", "tree_medusa"])
+                    choices=["greedy_llama3", "greedy_tiny", "rejection_qwen", "greedy_large_batch", "tree_medusa",
+                             "greedy_ragged_tiers"])
     ap.add_argument("--sets", type=int, default=None, help="input sets in the rotation (default: > 4x L2)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)

@@ -175,6 +175,71 @@ specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int6
                                    int32_t* accept_len, int32_t* accept_nodes, int32_t* out_tokens,
                                    void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
+/* ---------------------------------------------------------------------------
+ * Variable speculation length per request (handbook page, "Adaptive
+ * speculative decoding": the speculation length is changed per batch or
+ * request, e.g. SGLang's tiers [1, 3, 7]) in the packed layout serving
+ * engines use for it, with the acceptance counters of the vLLM page
+ * (section 3, result 4: accepted tokens in total and per draft position,
+ * draft tokens in total).
+ *
+ * Layout: request b owns drafts [off[b], off[b+1]) of the packed draft
+ * arrays, k_b = off[b+1] - off[b] of them, and the k_b + 1 logit rows and
+ * output slots starting at row off[b] + b; rows = B + total_drafts.
+ *   draft_offsets [B+1] int32, device.  A request whose offsets are not
+ *                 0 <= off[b] <= off[b+1] <= min(off[B], total_drafts) with
+ *                 k_b <= max_k is invalid: accept_len[b] = -1 and nothing
+ *                 else is written for it (its rows are unknown).
+ *   total_drafts  the number of drafts the caller laid out (host value);
+ *                 0 <= total_drafts <= B * max_k
+ *   max_k         bound on every k_b, 0 <= max_k <= SPECDEC_MAX_K
+ *   counters      [SPECDEC_COUNTERS(max_k)] int64, device, or NULL; each call
+ *                 ADDS, over its valid requests: [0] requests, [1] draft
+ *                 tokens (sum of k_b), [2] accepted tokens (sum of h),
+ *                 [3 + i] requests whose draft i was accepted (h > i).  The
+ *                 caller zeroes them when it wants a fresh count; tokens per
+ *                 step = 1 + [2] / [0] = 1 + sum_i [3 + i] / [0].
+ * Verification of each request is that of the fixed-layout call with its own
+ * k_b drafts (the rejection uniforms stay keyed by (request b, position i)).
+ * Workspace: specdec_workspace_size_ragged.
+ * ------------------------------------------------------------------------- */
+#define SPECDEC_COUNTERS(max_k) (3 + (max_k))
+
+/* Workspace bytes of a packed-layout greedy or rejection call; 0 for
+ * arguments outside the limits. */
+size_t specdec_workspace_size_ragged(specdec_mode mode, int B, int total_drafts, int V, specdec_dtype dtype);
+
+/* Greedy verification, packed layout.
+ *   logits       [B + total_drafts, V] of `dtype`, row stride `row_stride`
+ *   draft_tokens [total_drafts] int32 (may be NULL when total_drafts == 0)
+ *   accept_len   [B] int32 out
+ *   out_tokens   [B + total_drafts] int32 out: request b's slots from row
+ *                off[b] + b hold d_0..d_{h-1}, the greedy choice of row h,
+ *                then -1
+ *   topk_ids, topk_vals [B + total_drafts, topk] out, as specdec_verify_greedy */
+specdec_status specdec_verify_greedy_ragged(const void* logits, specdec_dtype dtype, int64_t row_stride,
+                                            const int32_t* draft_tokens, const int32_t* draft_offsets, int B,
+                                            int total_drafts, int max_k, int V, int32_t* accept_len,
+                                            int32_t* out_tokens, int topk, int32_t* topk_ids, float* topk_vals,
+                                            int64_t* counters, void* ws, size_t ws_bytes,
+                                            struct CUstream_st* stream);
+
+/* Rejection-sampling verification, packed layout.
+ *   target_logits [B + total_drafts, V]
+ *   draft_probs   [total_drafts, V] float32, row stride q_row_stride: q row
+ *                 off[b] + i belongs to request b's draft i
+ *   p_draft_out   [total_drafts] float32 out or NULL
+ *   out_tokens    [B + total_drafts] int32 out, slots as the greedy call
+ * Everything else as specdec_verify_rejection; counters over the requests
+ * whose target distributions are defined. */
+specdec_status specdec_verify_rejection_ragged(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
+                                               const float* draft_probs, int64_t q_row_stride,
+                                               const int32_t* draft_tokens, const int32_t* draft_offsets, int B,
+                                               int total_drafts, int max_k, int V, float temperature, uint64_t seed,
+                                               uint64_t offset, int32_t* accept_len, int32_t* out_tokens,
+                                               float* p_draft_out, int64_t* counters, void* ws, size_t ws_bytes,
+                                               struct CUstream_st* stream);
+
 /* Greedy verification without a caller workspace.  The pages have no
  * counterpart: this entry point exists for callers that cannot allocate
  * device memory (plug-ins and engine hooks handed only input and output

@@ -30,8 +30,8 @@ def _bind(path):
     L.oracle_verify_tree.argtypes = [P, i32, i64, P, P, i32, i32, i32, i32, P, P, P]
     L.oracle_verify_rejection.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f64, u64, u64,
                                           P, P, P, P]
-    L.oracle_verify_greedy_ragged.argtypes = [P, i32, i64, P, P, i32, i32, i32, P, P, i32, P, P, P]
-    L.oracle_verify_rejection_ragged.argtypes = [P, i32, i64, P, i64, P, P, i32, i32, i32, f64, u64, u64,
+    L.oracle_verify_greedy_ragged.argtypes = [P, i32, i64, P, P, i32, i64, i32, i32, P, P, i32, P, P, P]
+    L.oracle_verify_rejection_ragged.argtypes = [P, i32, i64, P, i64, P, P, i32, i64, i32, i32, f64, u64, u64,
                                                  P, P, P, P, P]
     for f in ("oracle_philox4x32_10", "oracle_uniforms", "oracle_argmax_rows", "oracle_topk_rows",
               "oracle_verify_greedy", "oracle_verify_tree", "oracle_verify_rejection",
@@ -174,15 +174,18 @@ def counters_size(max_k):
 
 
 def verify_greedy_ragged(logits, dtype, drafts, offsets, max_k, topk=0, counters=None):
-    """logits [R, V] (R = B + offsets[-1]); drafts [offsets[-1]]; offsets [B+1]
-    -> (accept_len [B], out_tokens [R], topk_ids [R, topk], topk_vals [R, topk],
-    counters [3 + max_k], accumulated into `counters` when given)."""
+    """logits [R, V] (R = B + T); drafts [T]; offsets [B+1] -> (accept_len
+    [B], out_tokens [R], topk_ids [R, topk], topk_vals [R, topk], counters
+    [3 + max_k], accumulated into `counters` when given).  T, the drafts the
+    arrays hold, bounds every request's offsets besides offsets[-1]."""
     x = _logit_array(logits, dtype)
     V = x.shape[-1]
     x = x.reshape(-1, V)
     off = _c(offsets, np.int32)
     B = off.size - 1
     d = _c(drafts, np.int32)
+    T = d.size
+    assert x.shape[0] == B + T, "logits must hold B + len(drafts) rows"
     if d.size == 0:
         d = np.zeros(1, np.int32)
     R = x.shape[0]
@@ -192,7 +195,7 @@ def verify_greedy_ragged(logits, dtype, drafts, offsets, max_k, topk=0, counters
     vals = np.full((R, max(topk, 1)), np.nan, np.float32)
     ctr = np.zeros(counters_size(max_k), np.int64) if counters is None else counters
     assert ctr.dtype == np.int64 and ctr.size == counters_size(max_k) and ctr.flags.c_contiguous
-    lib().oracle_verify_greedy_ragged(_ptr(x), DTYPE_CODE[dtype], V, _ptr(d), _ptr(off), B, max_k, V,
+    lib().oracle_verify_greedy_ragged(_ptr(x), DTYPE_CODE[dtype], V, _ptr(d), _ptr(off), B, T, max_k, V,
                                       _ptr(al), _ptr(out), topk, _ptr(ids), _ptr(vals), _ptr(ctr))
     return al, out, ids[:, :topk], vals[:, :topk], ctr
 
@@ -206,8 +209,10 @@ def verify_rejection_ragged(target, dtype, q, drafts, offsets, max_k, temperatur
     x = x.reshape(-1, V)
     off = _c(offsets, np.int32)
     B = off.size - 1
-    T = int(off[-1]) if B > 0 else 0
+    T = int(np.asarray(drafts).size)
+    assert x.shape[0] == B + T, "target must hold B + len(drafts) rows"
     qq = _c(q, np.float32).reshape(-1, V) if T > 0 else np.zeros((1, V), np.float32)
+    assert qq.shape[0] >= T
     d = _c(drafts, np.int32) if T > 0 else np.zeros(1, np.int32)
     R = x.shape[0]
     al = np.zeros(B, np.int32)
@@ -216,7 +221,7 @@ def verify_rejection_ragged(target, dtype, q, drafts, offsets, max_k, temperatur
     mg = np.zeros(B, np.float64)
     ctr = np.zeros(counters_size(max_k), np.int64) if counters is None else counters
     assert ctr.dtype == np.int64 and ctr.size == counters_size(max_k) and ctr.flags.c_contiguous
-    lib().oracle_verify_rejection_ragged(_ptr(x), DTYPE_CODE[dtype], V, _ptr(qq), V, _ptr(d), _ptr(off), B, max_k,
-                                         V, float(temperature), int(seed), int(offset), _ptr(al), _ptr(out),
+    lib().oracle_verify_rejection_ragged(_ptr(x), DTYPE_CODE[dtype], V, _ptr(qq), V, _ptr(d), _ptr(off), B, T,
+                                         max_k, V, float(temperature), int(seed), int(offset), _ptr(al), _ptr(out),
                                          _ptr(pd), _ptr(mg), _ptr(ctr))
     return al, out, pd[:T], mg, ctr

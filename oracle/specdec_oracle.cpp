@@ -340,9 +340,10 @@ void oracle_verify_greedy(const void* logits, int dtype, int64_t row_stride, con
 //   draft_offsets [B+1]  request b owns drafts [off[b], off[b+1]); k_b =
 //                        off[b+1] - off[b]; its k_b + 1 logit rows and output
 //                        slots start at row off[b] + b.  A request whose
-//                        offsets are not 0 <= off[b] <= off[b+1] <= off[B]
-//                        with k_b <= max_k is invalid: accept_len -1 and
-//                        nothing else written for it.
+//                        offsets are not 0 <= off[b] <= off[b+1] <= min(off[B],
+//                        total_drafts) with k_b <= max_k is invalid:
+//                        accept_len -1 and nothing else written for it.
+//   total_drafts         the drafts the arrays were laid out for
 //   logits        [B + off[B], V]; drafts [off[B]]
 //   out_tokens    [B + off[B]]; topk_ids / topk_vals [B + off[B], topk]
 //   counters      [3 + max_k] int64 or NULL, accumulated over valid requests:
@@ -350,10 +351,10 @@ void oracle_verify_greedy(const void* logits, int dtype, int64_t row_stride, con
 //                 tokens (sum of h), [3 + i] requests whose draft i was
 //                 accepted (h > i).
 void oracle_verify_greedy_ragged(const void* logits, int dtype, int64_t row_stride, const int32_t* drafts,
-                                 const int32_t* draft_offsets, int B, int max_k, int V,
+                                 const int32_t* draft_offsets, int B, int64_t total_drafts, int max_k, int V,
                                  int32_t* accept_len, int32_t* out_tokens, int topk, int32_t* topk_ids,
                                  float* topk_vals, int64_t* counters) {
-    const int64_t total = B > 0 ? draft_offsets[B] : 0;
+    const int64_t total = B > 0 ? std::min<int64_t>(draft_offsets[B], total_drafts) : 0;
     for (int b = 0; b < B; ++b) {
         const int64_t o0 = draft_offsets[b], o1 = draft_offsets[b + 1];
         if (!(o0 >= 0 && o0 <= o1 && o1 <= total && o1 - o0 <= max_k)) {
@@ -468,10 +469,10 @@ void oracle_verify_rejection(const void* target, int dtype, int64_t row_stride,
 // requests whose distributions are defined.
 void oracle_verify_rejection_ragged(const void* target, int dtype, int64_t row_stride, const float* q,
                                     int64_t q_row_stride, const int32_t* drafts, const int32_t* draft_offsets,
-                                    int B, int max_k, int V, double temperature, uint64_t seed, uint64_t offset,
-                                    int32_t* accept_len, int32_t* out_tokens, double* p_draft, double* margin,
-                                    int64_t* counters) {
-    const int64_t total = B > 0 ? draft_offsets[B] : 0;
+                                    int B, int64_t total_drafts, int max_k, int V, double temperature,
+                                    uint64_t seed, uint64_t offset, int32_t* accept_len, int32_t* out_tokens,
+                                    double* p_draft, double* margin, int64_t* counters) {
+    const int64_t total = B > 0 ? std::min<int64_t>(draft_offsets[B], total_drafts) : 0;
     for (int b = 0; b < B; ++b) {
         const int64_t o0 = draft_offsets[b], o1 = draft_offsets[b + 1];
         if (!(o0 >= 0 && o0 <= o1 && o1 <= total && o1 - o0 <= max_k)) {

@@ -92,6 +92,14 @@ def lib():
         L.specdec_verify_rejection.restype = i32
         L.specdec_verify_tree.argtypes = [P, i32, i64, P, P, i32, i32, i32, i32, P, P, P, P, sz, P]
         L.specdec_verify_tree.restype = i32
+        L.specdec_workspace_size_ragged.argtypes = [i32, i32, i32, i32, i32]
+        L.specdec_workspace_size_ragged.restype = sz
+        L.specdec_verify_greedy_ragged.argtypes = [P, i32, i64, P, P, i32, i32, i32, i32, P, P, i32, P, P, P,
+                                                   P, sz, P]
+        L.specdec_verify_greedy_ragged.restype = i32
+        L.specdec_verify_rejection_ragged.argtypes = [P, i32, i64, P, i64, P, P, i32, i32, i32, i32, f32, u64,
+                                                      u64, P, P, P, P, P, sz, P]
+        L.specdec_verify_rejection_ragged.restype = i32
         _lib = L
     return _lib
 
@@ -157,6 +165,35 @@ def specdec_verify_tree(logits, dtype, row_stride, parents, node_tokens, B, N, V
     return lib().specdec_verify_tree(_ptr(logits), dtype, row_stride, _ptr(parents), _ptr(node_tokens),
                                      B, N, V, max_depth, _ptr(accept_len), _ptr(accept_nodes),
                                      _ptr(out_tokens), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def specdec_counters(max_k: int) -> int:
+    return 3 + max_k
+
+
+def specdec_workspace_size_ragged(mode: int, B: int, total_drafts: int, V: int, dtype: int) -> int:
+    return lib().specdec_workspace_size_ragged(mode, B, total_drafts, V, dtype)
+
+
+def specdec_verify_greedy_ragged(logits, dtype, row_stride, draft_tokens, draft_offsets, B, total_drafts, max_k, V,
+                                 accept_len, out_tokens, topk, topk_ids, topk_vals, counters, ws, ws_bytes,
+                                 stream=None) -> int:
+    return lib().specdec_verify_greedy_ragged(_ptr(logits), dtype, row_stride, _ptr(draft_tokens),
+                                              _ptr(draft_offsets), B, total_drafts, max_k, V, _ptr(accept_len),
+                                              _ptr(out_tokens), topk, _ptr(topk_ids), _ptr(topk_vals),
+                                              _ptr(counters), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def specdec_verify_rejection_ragged(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens,
+                                    draft_offsets, B, total_drafts, max_k, V, temperature, seed, offset,
+                                    accept_len, out_tokens, p_draft_out, counters, ws, ws_bytes,
+                                    stream=None) -> int:
+    return lib().specdec_verify_rejection_ragged(_ptr(target_logits), dtype, row_stride, _ptr(draft_probs),
+                                                 q_row_stride, _ptr(draft_tokens), _ptr(draft_offsets), B,
+                                                 total_drafts, max_k, V, float(temperature),
+                                                 int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
+                                                 _ptr(accept_len), _ptr(out_tokens), _ptr(p_draft_out),
+                                                 _ptr(counters), _ptr(ws), ws_bytes, _stream(stream))
 
 
 def _check(status, what):
@@ -297,6 +334,80 @@ class Verifier:
                                         draft_tokens if k > 0 else None, B, k, V, temperature, seed, offset,
                                         al, ot, pd, ws, wsb, stream), "verify_rejection")
         return al, ot, (pd[:, :k] if pd is not None else None)
+
+
+    # -- packed layout: a speculation length per request ----------------------
+    @staticmethod
+    def _ragged_args(logits, draft_offsets, draft_tokens, total_drafts, max_k):
+        import torch
+        if logits.dim() != 2 or logits.stride(1) != 1:
+            raise ValueError("logits must be a 2-D [B + total_drafts, V] tensor with a contiguous last dimension")
+        if draft_offsets.dtype != torch.int32 or not draft_offsets.is_contiguous() or draft_offsets.dim() != 1:
+            raise ValueError("draft_offsets must be a contiguous int32 [B + 1] tensor")
+        B = draft_offsets.numel() - 1
+        if B < 0 or logits.shape[0] != B + total_drafts:
+            raise ValueError("logits must have B + total_drafts rows")
+        if total_drafts > 0 and (draft_tokens.dtype != torch.int32 or not draft_tokens.is_contiguous()
+                                 or draft_tokens.numel() != total_drafts):
+            raise ValueError("draft_tokens must be a contiguous int32 [total_drafts] tensor")
+        rs = int(logits.stride(0)) if logits.shape[0] > 1 else int(logits.shape[1])
+        return B, rs
+
+    def greedy_ragged(self, logits, draft_tokens, draft_offsets, total_drafts: int, max_k: int, topk: int = 0,
+                      counters=None, stream=None, out=None):
+        """logits [B + T, V], draft_tokens [T] int32, draft_offsets [B+1]
+        int32 (request b owns drafts [off[b], off[b+1]) and rows from
+        off[b] + b) -> (accept_len [B], out_tokens [B + T][, topk_ids,
+        topk_vals]); `counters` (int64 [3 + max_k]) accumulates."""
+        import torch
+        B, rs = self._ragged_args(logits, draft_offsets, draft_tokens, total_drafts, max_k)
+        R, V = logits.shape
+        dt = _dtype_code(logits)
+        dev = logits.device
+        if out is None:
+            al = torch.empty(B, dtype=torch.int32, device=dev)
+            ot = torch.empty(R, dtype=torch.int32, device=dev)
+            ids = torch.empty(R, max(topk, 1), dtype=torch.int32, device=dev) if topk else None
+            vals = torch.empty(R, max(topk, 1), dtype=torch.float32, device=dev) if topk else None
+        else:
+            al, ot, ids, vals = (tuple(out) + (None, None))[:4]
+        need = specdec_workspace_size_ragged(SPECDEC_MODE_GREEDY, B, total_drafts, V, dt)
+        ws, wsb = self.workspace(need, stream)
+        _check(specdec_verify_greedy_ragged(logits, dt, rs, draft_tokens if total_drafts > 0 else None,
+                                            draft_offsets, B, total_drafts, max_k, V, al, ot, topk, ids, vals,
+                                            counters, ws, wsb, stream), "verify_greedy_ragged")
+        return (al, ot, ids, vals) if topk else (al, ot)
+
+    def rejection_ragged(self, target_logits, draft_probs, draft_tokens, draft_offsets, total_drafts: int,
+                         max_k: int, temperature: float, seed: int, offset: int = 0, counters=None, stream=None,
+                         out=None, want_p_draft: bool = True):
+        """target_logits [B + T, V], draft_probs [T, V] f32, draft_tokens [T]
+        int32, draft_offsets [B+1] int32 -> (accept_len [B], out_tokens
+        [B + T], p_draft [T])."""
+        import torch
+        B, rs = self._ragged_args(target_logits, draft_offsets, draft_tokens, total_drafts, max_k)
+        R, V = target_logits.shape
+        dt = _dtype_code(target_logits)
+        qs = V
+        if total_drafts > 0:
+            if draft_probs.dtype != torch.float32 or draft_probs.dim() != 2 or draft_probs.stride(1) != 1 \
+                    or tuple(draft_probs.shape) != (total_drafts, V):
+                raise ValueError("draft_probs must be a float32 [total_drafts, V] tensor")
+            qs = int(draft_probs.stride(0)) if total_drafts > 1 else V
+        dev = target_logits.device
+        if out is None:
+            al = torch.empty(B, dtype=torch.int32, device=dev)
+            ot = torch.empty(R, dtype=torch.int32, device=dev)
+            pd = torch.empty(max(total_drafts, 1), dtype=torch.float32, device=dev) if want_p_draft else None
+        else:
+            al, ot, pd = out
+        need = specdec_workspace_size_ragged(SPECDEC_MODE_REJECTION, B, total_drafts, V, dt)
+        ws, wsb = self.workspace(need, stream)
+        _check(specdec_verify_rejection_ragged(target_logits, dt, rs, draft_probs if total_drafts > 0 else None, qs,
+                                               draft_tokens if total_drafts > 0 else None, draft_offsets, B,
+                                               total_drafts, max_k, V, temperature, seed, offset, al, ot, pd,
+                                               counters, ws, wsb, stream), "verify_rejection_ragged")
+        return al, ot, (pd[:total_drafts] if pd is not None else None)
 
 
 def specdec_verify_greedy_static_scratch(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len, out_tokens,

@@ -177,6 +177,111 @@ void fill_common(Pass1Params& P, const void* logits, int64_t row_stride, int V, 
 }  // namespace
 }  // namespace specdec
 
+namespace specdec {
+namespace {
+
+// Greedy verification over `rows` logit rows: the fixed layout (offsets null,
+// k drafts per request, rows = B (k + 1)) or the packed one (offsets [B+1],
+// k = the bound on every request's count, rows = B + total drafts).
+specdec_status greedy_impl(const void* logits, specdec_dtype dtype, int64_t row_stride, const int32_t* draft_tokens,
+                           const int32_t* offsets, int64_t total, int B, int k, int V, int32_t* accept_len,
+                           int32_t* out_tokens, int topk, int32_t* topk_ids, float* topk_vals, int64_t* counters,
+                           void* ws, size_t ws_bytes, cudaStream_t s) {
+    const int64_t rows = offsets ? B + total : static_cast<int64_t>(B) * (k + 1);
+    if (!rows_fit(rows, row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
+    if (logits == nullptr || accept_len == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (total > 0 && draft_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (topk > 0 && (topk_ids == nullptr || topk_vals == nullptr)) return SPECDEC_ERR_INVALID_ARG;
+    const bool vec = vector_path_ok(logits, row_stride, elem_size(dtype));
+    const int ve = vec ? vec_elems(dtype) : 1;
+    const Layout L = make_layout(rows, k + 1, B, V, ve, topk > 0 ? kTop8ChunkBytes : kArgmaxChunkBytes, false);
+    specdec_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != SPECDEC_OK) return st;
+    Pass1Params P;
+    fill_common(P, logits, row_stride, V, L, rows, k + 1, B, ws);
+    P.drafts = draft_tokens;
+    P.k = k;
+    P.draft_offsets = offsets;
+    P.total_drafts = total;
+    P.counters = counters;
+    P.accept_len = accept_len;
+    P.out_tokens = out_tokens;
+    P.topk = topk;
+    P.topk_ids = topk_ids;
+    P.topk_vals = topk_vals;
+    if (topk > 0) return dispatch_pass1<MODE_TOP8>(dtype, vec, P, s);
+    return dispatch_pass1<MODE_ARGMAX>(dtype, vec, P, s);
+}
+
+// Rejection-sampling verification, fixed or packed layout as greedy_impl.
+specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
+                              const float* draft_probs, int64_t q_row_stride, const int32_t* draft_tokens,
+                              const int32_t* offsets, int64_t total, int B, int k, int V, float temperature,
+                              uint64_t seed, uint64_t offset, int32_t* accept_len, int32_t* out_tokens,
+                              float* p_draft_out, int64_t* counters, void* ws, size_t ws_bytes, cudaStream_t s) {
+    if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
+    const int64_t rows = offsets ? B + total : static_cast<int64_t>(B) * (k + 1);
+    if (!rows_fit(rows, row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
+    if (target_logits == nullptr || accept_len == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (total > 0 && (draft_tokens == nullptr || draft_probs == nullptr)) return SPECDEC_ERR_INVALID_ARG;
+    if (total > 0 && !rows_fit(total, q_row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
+    const bool vec = vector_path_ok(target_logits, row_stride, elem_size(dtype)) &&
+                     (total == 0 || vector_path_ok(draft_probs, q_row_stride, 4));
+    const int ve = vec ? vec_elems(dtype) : 1;
+    const Layout L = make_layout(rows, k + 1, B, V, ve, kSoftmaxChunkBytes, true);
+    specdec_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != SPECDEC_OK) return st;
+    const double invT_d = 1.0 / static_cast<double>(temperature);
+    RejState* state = reinterpret_cast<RejState*>(static_cast<char*>(ws) + L.state);
+    Pass1Params P;
+    fill_common(P, target_logits, row_stride, V, L, rows, k + 1, B, ws);
+    P.drafts = draft_tokens;
+    P.k = k;
+    P.draft_offsets = offsets;
+    P.total_drafts = total;
+    P.counters = counters;
+    P.accept_len = accept_len;
+    P.out_tokens = out_tokens;
+    P.q = draft_probs;
+    P.q_stride = q_row_stride;
+    P.invT = static_cast<float>(invT_d);
+    P.invT_d = invT_d;
+    P.seed = seed;
+    P.offset = offset;
+    P.p_draft_out = p_draft_out;
+    P.state = state;
+    st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
+    if (st != SPECDEC_OK) return st;
+    Pass2Params Q;
+    memset(&Q, 0, sizeof(Q));
+    Q.logits = target_logits;
+    Q.row_stride = row_stride;
+    Q.q = draft_probs;
+    Q.q_stride = q_row_stride;
+    Q.V = V;
+    Q.nv_full = static_cast<int>(L.nv_full);
+    Q.cpr = static_cast<int>(L.cpr2);
+    Q.B = B;
+    Q.k = k;
+    Q.invT = static_cast<float>(invT_d);
+    Q.seed = seed;
+    Q.offset = offset;
+    Q.state = state;
+    Q.chunk_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.masses);
+    Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
+    Q.out_tokens = out_tokens;
+    return dispatch_pass2(dtype, vec, Q, s);
+}
+
+// Host checks of a packed-layout call.
+bool ragged_args_ok(const int32_t* offsets, int B, int total, int max_k) {
+    if (offsets == nullptr || total < 0 || max_k < 0 || max_k > SPECDEC_MAX_K) return false;
+    return static_cast<int64_t>(total) <= static_cast<int64_t>(B) * max_k;
+}
+
+}  // namespace
+}  // namespace specdec
+
 using namespace specdec;
 
 extern "C" {
@@ -215,6 +320,17 @@ size_t specdec_workspace_size(specdec_mode mode, int B, int k_or_N, int V, specd
     return a.total > b.total ? a.total : b.total;
 }
 
+size_t specdec_workspace_size_ragged(specdec_mode mode, int B, int total_drafts, int V, specdec_dtype dtype) {
+    if (!dtype_ok(dtype) || B < 0 || B > SPECDEC_MAX_B || V < 1 || V > SPECDEC_MAX_V) return 0;
+    if (mode != SPECDEC_MODE_GREEDY && mode != SPECDEC_MODE_REJECTION) return 0;
+    if (total_drafts < 0 || static_cast<int64_t>(total_drafts) > static_cast<int64_t>(B) * SPECDEC_MAX_K) return 0;
+    const int64_t rows = static_cast<int64_t>(B) + total_drafts;
+    const bool rej = mode == SPECDEC_MODE_REJECTION;
+    const Layout a = make_layout(rows, 1, B, V, vec_elems(dtype), slot_bytes(mode), rej);
+    const Layout b = make_layout(rows, 1, B, V, 1, slot_bytes(mode), rej);
+    return a.total > b.total ? a.total : b.total;
+}
+
 specdec_status specdec_workspace_init(void* ws, size_t bytes, struct CUstream_st* stream) {
     if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % 16 != 0) return SPECDEC_ERR_WORKSPACE;
     if (bytes == 0) return SPECDEC_OK;
@@ -231,28 +347,25 @@ specdec_status specdec_verify_greedy(const void* logits, specdec_dtype dtype, in
         return SPECDEC_ERR_INVALID_ARG;
     if (topk < 0 || topk > SPECDEC_MAX_TOPK) return SPECDEC_ERR_INVALID_ARG;
     if (B == 0) return SPECDEC_OK;
-    const int64_t rows = static_cast<int64_t>(B) * (k + 1);
-    if (!rows_fit(rows, row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
-    if (logits == nullptr || accept_len == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
-    if (k > 0 && draft_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
-    if (topk > 0 && (topk_ids == nullptr || topk_vals == nullptr)) return SPECDEC_ERR_INVALID_ARG;
-    const bool vec = vector_path_ok(logits, row_stride, elem_size(dtype));
-    const int ve = vec ? vec_elems(dtype) : 1;
-    const Layout L = make_layout(rows, k + 1, B, V, ve, topk > 0 ? kTop8ChunkBytes : kArgmaxChunkBytes, false);
-    specdec_status st = check_ws(ws, ws_bytes, L.total);
-    if (st != SPECDEC_OK) return st;
-    Pass1Params P;
-    fill_common(P, logits, row_stride, V, L, rows, k + 1, B, ws);
-    P.drafts = draft_tokens;
-    P.k = k;
-    P.accept_len = accept_len;
-    P.out_tokens = out_tokens;
-    P.topk = topk;
-    P.topk_ids = topk_ids;
-    P.topk_vals = topk_vals;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (topk > 0) return dispatch_pass1<MODE_TOP8>(dtype, vec, P, s);
-    return dispatch_pass1<MODE_ARGMAX>(dtype, vec, P, s);
+    return greedy_impl(logits, dtype, row_stride, draft_tokens, nullptr, static_cast<int64_t>(B) * k, B, k, V,
+                       accept_len, out_tokens, topk, topk_ids, topk_vals, nullptr, ws, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+specdec_status specdec_verify_greedy_ragged(const void* logits, specdec_dtype dtype, int64_t row_stride,
+                                            const int32_t* draft_tokens, const int32_t* draft_offsets, int B,
+                                            int total_drafts, int max_k, int V, int32_t* accept_len,
+                                            int32_t* out_tokens, int topk, int32_t* topk_ids, float* topk_vals,
+                                            int64_t* counters, void* ws, size_t ws_bytes,
+                                            struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || V < 1 || V > SPECDEC_MAX_V) return SPECDEC_ERR_INVALID_ARG;
+    if (topk < 0 || topk > SPECDEC_MAX_TOPK) return SPECDEC_ERR_INVALID_ARG;
+    if (!ragged_args_ok(draft_offsets, B, total_drafts, max_k)) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    return greedy_impl(logits, dtype, row_stride, draft_tokens, draft_offsets, total_drafts, B, max_k, V, accept_len,
+                       out_tokens, topk, topk_ids, topk_vals, counters, ws, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int64_t row_stride,
@@ -297,55 +410,26 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
         return SPECDEC_ERR_INVALID_ARG;
     if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
     if (B == 0) return SPECDEC_OK;
-    const int64_t rows = static_cast<int64_t>(B) * (k + 1);
-    if (!rows_fit(rows, row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
-    if (target_logits == nullptr || accept_len == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
-    if (k > 0 && (draft_tokens == nullptr || draft_probs == nullptr)) return SPECDEC_ERR_INVALID_ARG;
-    if (k > 0 && !rows_fit(static_cast<int64_t>(B) * k, q_row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
-    const bool vec = vector_path_ok(target_logits, row_stride, elem_size(dtype)) &&
-                     (k == 0 || vector_path_ok(draft_probs, q_row_stride, 4));
-    const int ve = vec ? vec_elems(dtype) : 1;
-    const Layout L = make_layout(rows, k + 1, B, V, ve, kSoftmaxChunkBytes, true);
-    specdec_status st = check_ws(ws, ws_bytes, L.total);
-    if (st != SPECDEC_OK) return st;
-    const double invT_d = 1.0 / static_cast<double>(temperature);
-    RejState* state = reinterpret_cast<RejState*>(static_cast<char*>(ws) + L.state);
-    Pass1Params P;
-    fill_common(P, target_logits, row_stride, V, L, rows, k + 1, B, ws);
-    P.drafts = draft_tokens;
-    P.k = k;
-    P.accept_len = accept_len;
-    P.out_tokens = out_tokens;
-    P.q = draft_probs;
-    P.q_stride = q_row_stride;
-    P.invT = static_cast<float>(invT_d);
-    P.invT_d = invT_d;
-    P.seed = seed;
-    P.offset = offset;
-    P.p_draft_out = p_draft_out;
-    P.state = state;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
-    if (st != SPECDEC_OK) return st;
-    Pass2Params Q;
-    memset(&Q, 0, sizeof(Q));
-    Q.logits = target_logits;
-    Q.row_stride = row_stride;
-    Q.q = draft_probs;
-    Q.q_stride = q_row_stride;
-    Q.V = V;
-    Q.nv_full = static_cast<int>(L.nv_full);
-    Q.cpr = static_cast<int>(L.cpr2);
-    Q.B = B;
-    Q.k = k;
-    Q.invT = static_cast<float>(invT_d);
-    Q.seed = seed;
-    Q.offset = offset;
-    Q.state = state;
-    Q.chunk_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.masses);
-    Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
-    Q.out_tokens = out_tokens;
-    return dispatch_pass2(dtype, vec, Q, s);
+    return rejection_impl(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens, nullptr,
+                          static_cast<int64_t>(B) * k, B, k, V, temperature, seed, offset, accept_len, out_tokens,
+                          p_draft_out, nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+specdec_status specdec_verify_rejection_ragged(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
+                                               const float* draft_probs, int64_t q_row_stride,
+                                               const int32_t* draft_tokens, const int32_t* draft_offsets, int B,
+                                               int total_drafts, int max_k, int V, float temperature, uint64_t seed,
+                                               uint64_t offset, int32_t* accept_len, int32_t* out_tokens,
+                                               float* p_draft_out, int64_t* counters, void* ws, size_t ws_bytes,
+                                               struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || V < 1 || V > SPECDEC_MAX_V) return SPECDEC_ERR_INVALID_ARG;
+    if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
+    if (!ragged_args_ok(draft_offsets, B, total_drafts, max_k)) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    return rejection_impl(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens, draft_offsets,
+                          total_drafts, B, max_k, V, temperature, seed, offset, accept_len, out_tokens, p_draft_out,
+                          counters, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

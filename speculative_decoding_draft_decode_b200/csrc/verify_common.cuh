@@ -17,7 +17,9 @@ struct RejState {
     float M;         // max logit of row h
     float pad;
     double Z;        // sum exp((l - M)/T) of row h
-    double pad2;
+    int64_t row;     // logit row h, which is also the output slot of the drawn token
+    int64_t qrow;    // q row h when a draft was rejected (residual), else -1 (bonus from p)
+    int64_t pad2;
 };
 
 // Programmatic dependent launch: a kernel launched with programmatic stream

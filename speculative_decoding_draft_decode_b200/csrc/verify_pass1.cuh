@@ -85,7 +85,10 @@ struct Pass1Params {
     void* partials;             // [R * cpr * NWARPS] slots
     // greedy / rejection
     const int32_t* drafts;
-    int k;
+    int k;                      // drafts per request (packed layout: the bound max_k)
+    const int32_t* draft_offsets;  // [B+1] packed layout, or null: k drafts per request
+    int64_t total_drafts;       // packed layout: drafts (and q rows) the caller laid out
+    int64_t* counters;          // [3 + k] acceptance counters, or null
     int32_t* accept_len;
     int32_t* out_tokens;
     int topk;
@@ -629,10 +632,59 @@ __device__ void row_top8_warp(const Pass1Params& P, int64_t r, uint64_t* surv, u
 // ---------------------------------------------------------------------------
 // Request epilogues (every thread of the last-ticket CTA).
 // ---------------------------------------------------------------------------
+// Where request b's rows, drafts and outputs are.  Fixed layout: k drafts
+// per request, rows b*(k+1) ...  Packed layout (variable speculation length,
+// handbook page "Adaptive speculative decoding"): request b owns drafts
+// [off[b], off[b+1]), k_b = off[b+1] - off[b], and the k_b + 1 rows and
+// output slots from row off[b] + b.  A request whose offsets are out of
+// order, end past the caller's total or exceed the bound k is invalid (ok =
+// false) and nothing but accept_len = -1 is written for it, so no index can
+// leave the caller's arrays.
+struct ReqGeom {
+    int64_t row0;  // first logit row / output slot
+    int64_t d0;    // first draft (and q row, p_draft entry)
+    int kb;        // drafts of the request
+    bool ok;
+};
+
+__device__ __forceinline__ ReqGeom req_geom(const Pass1Params& P, int64_t b) {
+    ReqGeom g;
+    if (P.draft_offsets == nullptr) {
+        g.row0 = b * (P.k + 1);
+        g.d0 = b * P.k;
+        g.kb = P.k;
+        g.ok = true;
+        return g;
+    }
+    const int64_t o0 = __ldg(&P.draft_offsets[b]), o1 = __ldg(&P.draft_offsets[b + 1]);
+    const int64_t tot = __ldg(&P.draft_offsets[P.B]);
+    g.ok = o0 >= 0 && o0 <= o1 && o1 <= tot && o1 <= P.total_drafts && o1 - o0 <= P.k;
+    g.kb = g.ok ? static_cast<int>(o1 - o0) : 0;
+    g.d0 = o0;
+    g.row0 = o0 + b;
+    return g;
+}
+
+// Acceptance counters (vLLM page, section 3 result 4): [0] requests, [1]
+// draft tokens, [2] accepted tokens, [3 + i] requests whose draft i was
+// accepted.  Warp-collective (one warp), h <= 32.
+__device__ __forceinline__ void count_request(int64_t* ctr, int kb, int h) {
+    if (ctr == nullptr) return;
+    const int lane = threadIdx.x & 31;
+    unsigned long long* c = reinterpret_cast<unsigned long long*>(ctr);
+    if (lane == 0) {
+        atomicAdd(&c[0], 1ull);
+        atomicAdd(&c[1], static_cast<unsigned long long>(kb));
+        atomicAdd(&c[2], static_cast<unsigned long long>(h));
+    }
+    if (lane < h) atomicAdd(&c[3 + lane], 1ull);
+}
+
 // Greedy accept scan of request b (warp 0): h = the number of leading drafts
 // equal to their row's argmax; out = d_0..d_{h-1}, argmax_h, then -1.
-__device__ __forceinline__ void greedy_accept(const Pass1Params& P, int64_t b, const int* drafts, const int* am) {
-    const int k = P.k;
+__device__ __forceinline__ void greedy_accept(const Pass1Params& P, int64_t b, const ReqGeom& g, const int* drafts,
+                                              const int* am) {
+    const int k = g.kb;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x < 32) {
         bool match = false;
@@ -646,23 +698,29 @@ __device__ __forceinline__ void greedy_accept(const Pass1Params& P, int64_t b, c
             int tokv = -1;
             if (i < h) tokv = drafts[i];
             else if (i == h) tokv = am[h];
-            P.out_tokens[b * (k + 1) + i] = tokv;
+            P.out_tokens[g.row0 + i] = tokv;
         }
         if (lane == 0) P.accept_len[b] = h;
+        count_request(P.counters, k, h);
     }
 }
 
 template <class Tag, class Smem>
 __device__ void epilogue_greedy(const Pass1Params& P, int64_t b, Smem& sm) {
-    const int k = P.k;
+    const ReqGeom g = req_geom(P, b);
+    if (!g.ok) {
+        if (threadIdx.x == 0) P.accept_len[b] = -1;
+        return;
+    }
+    const int k = g.kb;
     // The drafts are loaded into registers first and stored after the merge
     // has issued its loads, so the two round trips overlap.
-    const int dr = threadIdx.x < k ? P.drafts[b * k + threadIdx.x] : 0;
-    merge_argmax_rows<Tag>(P, b * (k + 1), k + 1, sm.rowkey);
-    if (threadIdx.x <= k) sm.am[threadIdx.x] = key_index(sm.rowkey[threadIdx.x]);
-    if (threadIdx.x < k) sm.drafts[threadIdx.x] = dr;
+    const int dr = static_cast<int>(threadIdx.x) < k ? P.drafts[g.d0 + threadIdx.x] : 0;
+    merge_argmax_rows<Tag>(P, g.row0, k + 1, sm.rowkey);
+    if (static_cast<int>(threadIdx.x) <= k) sm.am[threadIdx.x] = key_index(sm.rowkey[threadIdx.x]);
+    if (static_cast<int>(threadIdx.x) < k) sm.drafts[threadIdx.x] = dr;
     __syncthreads();
-    greedy_accept(P, b, sm.drafts, sm.am);
+    greedy_accept(P, b, g, sm.drafts, sm.am);
 }
 
 template <class Tag>
@@ -776,7 +834,17 @@ __device__ void epilogue_tree(const Pass1Params& P, int64_t b, Pass1SmemTree& sm
 
 template <class Tag>
 __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& sm) {
-    const int k = P.k;
+    const ReqGeom g = req_geom(P, b);
+    if (!g.ok) {
+        if (threadIdx.x == 0) {
+            P.accept_len[b] = -1;
+            RejState st = {};
+            st.valid = 0;
+            P.state[b] = st;
+        }
+        return;
+    }
+    const int k = g.kb;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     constexpr int kGatherWarp = NWARPS - 1;
     // The last warp fetches the drafts and their logits and q values first;
@@ -784,15 +852,15 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
     int d = -1;
     float ld = 0.0f, qf = 0.0f;
     if (wp == kGatherWarp && lane < k) {
-        d = P.drafts[b * k + lane];
+        d = P.drafts[g.d0 + lane];
         if (d >= 0 && d < P.V) {
-            const int64_t r = b * (k + 1) + lane;
+            const int64_t r = g.row0 + lane;
             ld = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + d);
-            qf = __ldg(P.q + (b * k + lane) * P.q_stride + d);
+            qf = __ldg(P.q + (g.d0 + lane) * P.q_stride + d);
         }
     }
     for (int t = wp; t <= k; t += NWARPS) {
-        const int64_t r = b * (k + 1) + t;
+        const int64_t r = g.row0 + t;
         const int np = P.cpr * NWARPS;
         const SoftmaxPartial* p = static_cast<const SoftmaxPartial*>(P.partials) + r * np;
         MaxSum acc;
@@ -824,9 +892,9 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
     }
     bad = __syncthreads_or(bad);
     if (bad) {
-        for (int i = threadIdx.x; i <= k; i += NT) P.out_tokens[b * (k + 1) + i] = -1;
+        for (int i = threadIdx.x; i <= k; i += NT) P.out_tokens[g.row0 + i] = -1;
         if (P.p_draft_out)
-            for (int i = threadIdx.x; i < k; i += NT) P.p_draft_out[b * k + i] = __uint_as_float(0x7fc00000u);
+            for (int i = threadIdx.x; i < k; i += NT) P.p_draft_out[g.d0 + i] = __uint_as_float(0x7fc00000u);
         if (threadIdx.x == 0) {
             P.accept_len[b] = -1;
             RejState st = {};
@@ -844,16 +912,16 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
                 p = exp((static_cast<double>(ld) - static_cast<double>(sm.rowM[lane])) * P.invT_d) / sm.rowZ[lane];
                 qd = static_cast<double>(qf);
             }
-            if (P.p_draft_out) P.p_draft_out[b * k + lane] = static_cast<float>(p);
+            if (P.p_draft_out) P.p_draft_out[g.d0 + lane] = static_cast<float>(p);
             const double2 u = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(lane));
             accept = in && (u.x * qd < p);
         }
         const unsigned rej = __ballot_sync(FULL_MASK, lane < k && !accept);
         const int h = rej ? __ffs(rej) - 1 : k;
         // out_tokens[i] = d_i for i < h, -1 after h; slot h is the resample's.
-        if (lane < h) P.out_tokens[b * (k + 1) + lane] = d;
-        else if (lane > h && lane <= k) P.out_tokens[b * (k + 1) + lane] = -1;
-        if (k == 32 && lane == 0 && h < 32) P.out_tokens[b * (k + 1) + 32] = -1;
+        if (lane < h) P.out_tokens[g.row0 + lane] = d;
+        else if (lane > h && lane <= k) P.out_tokens[g.row0 + lane] = -1;
+        if (k == 32 && lane == 0 && h < 32) P.out_tokens[g.row0 + 32] = -1;
         if (lane == 0) {
             P.accept_len[b] = h;
             RejState st = {};
@@ -861,8 +929,11 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
             st.valid = 1;
             st.M = sm.rowM[h];
             st.Z = sm.rowZ[h];
+            st.row = g.row0 + h;
+            st.qrow = h < k ? g.d0 + h : -1;
             P.state[b] = st;
         }
+        count_request(P.counters, k, h);
     }
 }
 
@@ -1001,39 +1072,50 @@ __global__ void __launch_bounds__(NT) verify_epilogue_kernel(const Pass1Params P
 // Greedy top-8 request epilogue, one CTA per request of 32 * min(k + 1, 16)
 // threads: one warp per row (rows beyond 16 take a second turn), then the
 // top-k outputs (values re-read at the winning indices, so they are the
-// stored bits), the row thresholds back to zero, and the accept scan.
+// stored bits) and the accept scan.  Every row's threshold word goes back to
+// zero: CTA b clears rows [b R / B, (b+1) R / B), which are its own rows in
+// the fixed layout and cover every row in the packed one whatever the
+// offsets hold (a word cleared before its owner read it only weakens that
+// owner's filter).
 template <class Tag>
 __global__ void __launch_bounds__(32 * kTop8EpiWarps) verify_top8_epilogue_kernel(const Pass1Params P) {
     __shared__ Top8EpiSmem sm;
-    const int k = P.k, n = k + 1;
     const int nthreads = static_cast<int>(blockDim.x), nw = nthreads >> 5;
     const int wp = threadIdx.x >> 5;
     grid_dependency_wait();
     grid_launch_dependents();
     const int64_t b = blockIdx.x;
-    const int dr = static_cast<int>(threadIdx.x) < k ? P.drafts[b * k + threadIdx.x] : 0;
-    for (int t = wp; t < n; t += nw) row_top8_warp<Tag>(P, b * n + t, sm.surv[wp], sm.top[t]);
-    if (static_cast<int>(threadIdx.x) < k) sm.drafts[threadIdx.x] = dr;
-    __syncthreads();
-    for (int o = threadIdx.x; o < n * 8; o += nthreads) {
-        const int t = o >> 3, e = o & 7;
-        const int64_t r = b * n + t;
-        const uint64_t key = sm.top[t][e];
-        if (e == 0) sm.am[t] = key_index(key);
-        if (e < P.topk) {
-            int id = -1;
-            float val = __uint_as_float(0x7fc00000u);
-            if (key != 0ull) {
-                id = key_index(key);
-                val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + id);
+    const ReqGeom g = req_geom(P, b);
+    if (g.ok) {
+        const int k = g.kb, n = k + 1;
+        const int dr = static_cast<int>(threadIdx.x) < k ? P.drafts[g.d0 + threadIdx.x] : 0;
+        for (int t = wp; t < n; t += nw) row_top8_warp<Tag>(P, g.row0 + t, sm.surv[wp], sm.top[t]);
+        if (static_cast<int>(threadIdx.x) < k) sm.drafts[threadIdx.x] = dr;
+        __syncthreads();
+        for (int o = threadIdx.x; o < n * 8; o += nthreads) {
+            const int t = o >> 3, e = o & 7;
+            const int64_t r = g.row0 + t;
+            const uint64_t key = sm.top[t][e];
+            if (e == 0) sm.am[t] = key_index(key);
+            if (e < P.topk) {
+                int id = -1;
+                float val = __uint_as_float(0x7fc00000u);
+                if (key != 0ull) {
+                    id = key_index(key);
+                    val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride +
+                                           id);
+                }
+                P.topk_ids[r * P.topk + e] = id;
+                P.topk_vals[r * P.topk + e] = val;
             }
-            P.topk_ids[r * P.topk + e] = id;
-            P.topk_vals[r * P.topk + e] = val;
         }
-        if (e == 0 && r < kThetaRows) P.theta_row[r] = 0u;
+        __syncthreads();
+        greedy_accept(P, b, g, sm.drafts, sm.am);
+    } else if (threadIdx.x == 0) {
+        P.accept_len[b] = -1;
     }
-    __syncthreads();
-    greedy_accept(P, b, sm.drafts, sm.am);
+    const int64_t c0 = b * P.R / P.B, c1 = (b + 1) * P.R / P.B;
+    for (int64_t r = c0 + threadIdx.x; r < c1 && r < kThetaRows; r += nthreads) P.theta_row[r] = 0u;
 }
 
 }  // namespace specdec

@@ -123,11 +123,11 @@ struct Pass2Row {
 };
 
 template <class Tag>
-__device__ __forceinline__ Pass2Row pass2_row(const Pass2Params& P, int64_t b, const RejState& st) {
+__device__ __forceinline__ Pass2Row pass2_row(const Pass2Params& P, const RejState& st) {
     Pass2Row R;
-    R.row = static_cast<const typename Tag::storage*>(P.logits) + (b * (P.k + 1) + st.h) * P.row_stride;
-    R.has_q = st.h < P.k;
-    R.qrow = R.has_q ? P.q + (b * P.k + st.h) * P.q_stride : nullptr;
+    R.row = static_cast<const typename Tag::storage*>(P.logits) + st.row * P.row_stride;
+    R.has_q = st.qrow >= 0;
+    R.qrow = R.has_q ? P.q + st.qrow * P.q_stride : nullptr;
     R.invZ = static_cast<float>(1.0 / st.Z);
     return R;
 }
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P
     const int sub = static_cast<int>(blockIdx.y);
     const RejState st = P.state[b];
     if (!st.valid) return;  // CTA-uniform
-    const Pass2Row R = pass2_row<Tag>(P, b, st);
+    const Pass2Row R = pass2_row<Tag>(P, st);
     const Elem* row = static_cast<const Elem*>(R.row);
     const int cnt = chunk_count(P.nv_full, sub, VEC, kU2);
     double2* um = P.unit_mass + (b * P.cpr + sub) * UPC;
@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
     if (b >= P.B) return;  // warp-uniform
     const RejState st = P.state[b];
     if (!st.valid) return;  // the statistics pass already wrote -1 everywhere
-    const int64_t out_at = b * (P.k + 1) + st.h;
+    const int64_t out_at = st.row;  // the drawn token's slot is row h's
 
     // Totals of r and p over the chunk masses, then u_res * S.
     const double2* cm = P.chunk_mass + b * P.cpr;
@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
     const int unit = warp_find_level(um, has_tail ? UPC : UPC - 1, use_p, before, target, found, before);
     int token = P.V - 1;
     if (unit >= 0) {
-        const Pass2Row R = pass2_row<Tag>(P, b, st);
+        const Pass2Row R = pass2_row<Tag>(P, st);
         const Elem* row = static_cast<const Elem*>(R.row);
         float m[VEC];
         int x0 = 0, nx = 0;  // first element of the lane and how many it holds

@@ -1,0 +1,186 @@
+"""CUDA verifier in the packed layout of variable speculation lengths
+(handbook page, "Adaptive speculative decoding") with its acceptance counters
+(vLLM page, section 3 result 4), against the oracle: bit-exact for greedy,
+the rejection tolerance of test_gpu_parity for sampling, exact counters."""
+import numpy as np
+import pytest
+
+import gen
+import oracle
+from gpu_util import dev_f32, dev_i32, dev_logits, host, require_cuda
+from test_gpu_parity import MARGIN, EXEMPT_FRACTION, P_DRAFT_RTOL
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def V_():
+    torch = require_cuda()
+    import speculative_decoding_draft_decode_b200 as sd
+    return sd.Verifier(torch.device("cuda", 0))
+
+
+def _kb(rng, B, max_k):
+    kb = rng.integers(0, max_k + 1, size=B)
+    kb[0], kb[-1] = 0, max_k
+    return kb
+
+
+def _valid_rows(offsets, al):
+    """Output slots of the valid requests."""
+    rows = []
+    for b in range(len(offsets) - 1):
+        if al[b] >= 0:
+            r0 = offsets[b] + b
+            rows.extend(range(r0, r0 + offsets[b + 1] - offsets[b] + 1))
+    return np.array(rows, np.int64)
+
+
+def run_greedy_ragged(ver, r, offsets=None, topk=0, counters=None):
+    import torch
+    off = r.offsets if offsets is None else offsets
+    x = dev_logits(r.logits, r.dtype)
+    d = dev_i32(r.drafts if r.drafts.size else np.zeros(1, np.int32))
+    o = dev_i32(off)
+    ctr = counters if counters is not None else torch.zeros(3 + r.max_k, dtype=torch.int64, device="cuda")
+    res = ver.greedy_ragged(x, d, o, int(r.offsets[-1]), r.max_k, topk=topk, counters=ctr)
+    return [host(t) for t in res] + [host(ctr)]
+
+
+def check_greedy_ragged(ver, r, offsets=None, topk=0):
+    off = r.offsets if offsets is None else offsets
+    got = run_greedy_ragged(ver, r, offsets, topk)
+    al, out, ids, vals, ctr = oracle.verify_greedy_ragged(r.logits, r.dtype, r.drafts, off, r.max_k, topk=topk)
+    assert np.array_equal(got[0], al)
+    rows = _valid_rows(off, al)
+    assert np.array_equal(got[1][rows], out[rows])
+    if topk:
+        assert np.array_equal(got[2][rows], ids[rows])
+        assert np.array_equal(got[3][rows].view(np.uint32), vals[rows].view(np.uint32))
+    assert np.array_equal(got[-1], ctr), (got[-1], ctr)
+    return got
+
+
+@pytest.mark.parametrize("dtype,V,topk", [("f32", 1000, 0), ("bf16", 4099, 8), ("f32", 50001, 8), ("bf16", 7, 3)])
+def test_greedy_ragged_random_lengths(V_, dtype, V, topk):
+    rng = np.random.default_rng(V)
+    base = gen.greedy_synthetic(seed=V, B=37, k=8, V=V, alpha=0.8, dtype=dtype)
+    r = gen.pack_ragged("t", dtype, base.logits, base.drafts, _kb(rng, 37, 8), 8)
+    check_greedy_ragged(V_, r, topk=topk)
+
+
+def test_greedy_ragged_all_k_equals_fixed(V_):
+    import torch
+    base = gen.greedy_synthetic(seed=21, B=16, k=5, V=3000, alpha=0.7, dtype="bf16")
+    r = gen.pack_ragged("t", "bf16", base.logits, base.drafts, np.full(16, 5), 5)
+    got = run_greedy_ragged(V_, r, topk=8)
+    fixed = V_.greedy(dev_logits(base.logits, "bf16"), dev_i32(base.drafts), topk=8)
+    f = [host(t) for t in fixed]
+    assert np.array_equal(got[0], f[0])
+    assert np.array_equal(got[1].reshape(16, 6), f[1])
+    assert np.array_equal(got[2].reshape(16, 6, 8), f[2])
+
+
+def test_greedy_ragged_tier_workload(V_):
+    r = gen.greedy_ragged_tiers()
+    check_greedy_ragged(V_, r)
+    r.topk = 8
+    check_greedy_ragged(V_, r, topk=8)
+
+
+def test_greedy_ragged_invalid_offsets(V_):
+    rng = np.random.default_rng(2)
+    base = gen.greedy_synthetic(seed=22, B=12, k=4, V=800, alpha=0.9)
+    r = gen.pack_ragged("t", "f32", base.logits, base.drafts, _kb(rng, 12, 4), 4)
+    off = r.offsets.copy()
+    off[3] = off[2] - 1          # request 2 runs backwards (request 3 starts one draft early)
+    off[9] = off[8] + 6          # request 8 has 6 > max_k drafts
+    check_greedy_ragged(V_, r, offsets=off, topk=8)
+    off2 = r.offsets.copy()
+    off2[5:] += 9                # request 4 too long; the later ones shifted, some past the caller's total
+    got = check_greedy_ragged(V_, r, offsets=off2)
+    assert got[0][4] == -1 and got[0][-1] == -1
+
+
+def test_counters_accumulate_and_replay(V_):
+    import torch
+    rng = np.random.default_rng(3)
+    base = gen.greedy_synthetic(seed=23, B=24, k=7, V=2000, alpha=0.8, dtype="bf16")
+    r = gen.pack_ragged("t", "bf16", base.logits, base.drafts, _kb(rng, 24, 7), 7)
+    _, _, _, _, ctr1 = oracle.verify_greedy_ragged(r.logits, "bf16", r.drafts, r.offsets, 7)
+    x, d, o = dev_logits(r.logits, "bf16"), dev_i32(r.drafts), dev_i32(r.offsets)
+    T = int(r.offsets[-1])
+    ctr = torch.zeros(10, dtype=torch.int64, device="cuda")
+    al = torch.empty(24, dtype=torch.int32, device="cuda")
+    ot = torch.empty(24 + T, dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        V_.greedy_ragged(x, d, o, T, 7, counters=ctr, out=(al, ot))  # workspace sized before capture
+    s.synchronize()
+    assert np.array_equal(host(ctr), ctr1)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        V_.greedy_ragged(x, d, o, T, 7, counters=ctr, out=(al, ot))
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(host(ctr), 4 * ctr1)
+
+
+def test_top8_thresholds_clean_between_layouts(V_):
+    """Packed top-8 calls leave no row threshold behind: a fixed-layout call
+    on other data through the same workspace stays exact."""
+    rng = np.random.default_rng(4)
+    base = gen.greedy_synthetic(seed=24, B=20, k=6, V=70000, alpha=0.8, dtype="bf16")
+    r = gen.pack_ragged("t", "bf16", base.logits, base.drafts, _kb(rng, 20, 6), 6)
+    off = r.offsets.copy()
+    off[4] = off[5] + 1          # one request invalid: its rows are streamed but not owned
+    check_greedy_ragged(V_, r, offsets=off, topk=8)
+    other = gen.greedy_synthetic(seed=25, B=26, k=6, V=70000, alpha=0.8, dtype="bf16")
+    got = [host(t) for t in V_.greedy(dev_logits(other.logits, "bf16"), dev_i32(other.drafts), topk=8)]
+    ids, vals = oracle.topk_rows(other.logits.reshape(-1, 70000), "bf16", 8)
+    assert np.array_equal(got[2].reshape(-1, 8), ids)
+
+
+def run_rejection_ragged(ver, r, counters=None):
+    import torch
+    T = int(r.offsets[-1])
+    x = dev_logits(r.logits, r.dtype)
+    q = dev_f32(r.q if T else np.zeros((1, r.V), np.float32))
+    d = dev_i32(r.drafts if T else np.zeros(1, np.int32))
+    o = dev_i32(r.offsets)
+    ctr = torch.zeros(3 + r.max_k, dtype=torch.int64, device="cuda")
+    al, out, pd = ver.rejection_ragged(x, q, d, o, T, r.max_k, r.temperature, r.seed, r.offset, counters=ctr)
+    return host(al), host(out), host(pd), host(ctr)
+
+
+@pytest.mark.parametrize("V,dtype,T", [(1000, "f32", 1.0), (4099, "bf16", 0.7), (151936, "f32", 1.0)])
+def test_rejection_ragged_vs_oracle(V_, V, dtype, T):
+    rng = np.random.default_rng(V)
+    B, K = (40, 6) if V < 100000 else (6, 4)
+    tgt = (rng.standard_normal((B, K + 1, V)) * 1.5).astype(np.float32)
+    noisy = tgt[:, :K].astype(np.float64) + rng.standard_normal((B, K, V))
+    q = np.exp(noisy - noisy.max(-1, keepdims=True))
+    q = (q / q.sum(-1, keepdims=True)).astype(np.float32)
+    drafts = np.empty((B, K), np.int32)
+    for b in range(B):
+        for i in range(K):
+            c = np.cumsum(q[b, i].astype(np.float64))
+            drafts[b, i] = min(int(np.searchsorted(c, rng.random() * c[-1], side="right")), V - 1)
+    target = gen.f32_to_bf16_bits(tgt) if dtype == "bf16" else tgt
+    r = gen.pack_ragged("t", dtype, target, drafts, _kb(rng, B, K), K, q=q, temperature=T, seed=5, offset=9)
+    al, out, pd, ctr = run_rejection_ragged(V_, r)
+    e_al, e_out, e_pd, e_mg, e_ctr = oracle.verify_rejection_ragged(r.logits, dtype, r.q, r.drafts, r.offsets, K,
+                                                                   T, 5, 9)
+    pos = e_pd > 0
+    assert np.all(np.abs(pd[pos] - e_pd[pos]) <= P_DRAFT_RTOL * e_pd[pos])
+    mism = 0
+    for b in range(B):
+        r0, kb = r.offsets[b] + b, r.offsets[b + 1] - r.offsets[b]
+        same = al[b] == e_al[b] and np.array_equal(out[r0:r0 + kb + 1], e_out[r0:r0 + kb + 1])
+        if not same:
+            assert e_mg[b] < MARGIN, b
+            mism += 1
+    assert mism <= max(1, EXEMPT_FRACTION * B)
+    if mism == 0:
+        assert np.array_equal(ctr, e_ctr)

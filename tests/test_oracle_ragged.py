@@ -114,6 +114,10 @@ def test_invalid_offsets():
     al2, *_ = oracle.verify_greedy_ragged(r.logits, "f32", r.drafts, off2, 3)
     assert al2[-1] == -1 and al2[-2] == -1   # both now end past the total
     assert al2[0] == 3
+    off3 = r.offsets.copy()
+    off3[3:] += 2                  # offsets past the drafts the arrays hold
+    al3, *_ = oracle.verify_greedy_ragged(r.logits, "f32", r.drafts, off3, 3)
+    assert al3[-1] == -1 and al3[0] == 3
 
 
 def test_counters_reproduce_page_per_position_acceptance():
