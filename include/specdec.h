@@ -240,6 +240,32 @@ specdec_status specdec_verify_rejection_ragged(const void* target_logits, specde
                                                float* p_draft_out, int64_t* counters, void* ws, size_t ws_bytes,
                                                struct CUstream_st* stream);
 
+/* Speculation-length tiers (handbook page, "Adaptive speculative decoding":
+ * SGLang keeps an exponential moving average of the accepted length after
+ * every verify round and switches among predefined speculation lengths,
+ * default [1, 3, 7], each with its own captured CUDA graph).  Host-only
+ * helpers; they launch nothing.
+ *   specdec_tier_update  ema <- decay * ema + (1 - decay) * accepted, where
+ *                        `accepted` is the mean accepted drafts per request of
+ *                        the last round (from the counters: the change of [2]
+ *                        over the change of [0]); the first update sets ema =
+ *                        accepted.  decay in [0, 1).  Returns the new ema, or
+ *                        NaN for invalid arguments (state unchanged).
+ *   specdec_tier_select  the smallest tier t with t >= ema + 1/2, else the
+ *                        largest tier; tiers must be strictly increasing and
+ *                        in [0, SPECDEC_MAX_K].  The accepted length cannot
+ *                        exceed the tier it was measured at, so a saturated
+ *                        tier (nearly every draft accepted) moves up, and a
+ *                        tier whose drafts mostly fail moves down.  Returns -1
+ *                        for invalid arguments.  The page does not state the
+ *                        switching rule; this is the library's reading of it. */
+typedef struct {
+    double ema;
+    int initialized;
+} specdec_tier_state;
+double specdec_tier_update(specdec_tier_state* state, double accepted, double decay);
+int specdec_tier_select(const int* tiers, int n_tiers, double ema);
+
 /* Greedy verification without a caller workspace.  The pages have no
  * counterpart: this entry point exists for callers that cannot allocate
  * device memory (plug-ins and engine hooks handed only input and output

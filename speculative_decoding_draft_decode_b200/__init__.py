@@ -100,6 +100,10 @@ def lib():
         L.specdec_verify_rejection_ragged.argtypes = [P, i32, i64, P, i64, P, P, i32, i32, i32, i32, f32, u64,
                                                       u64, P, P, P, P, P, sz, P]
         L.specdec_verify_rejection_ragged.restype = i32
+        L.specdec_tier_update.argtypes = [P, ctypes.c_double, ctypes.c_double]
+        L.specdec_tier_update.restype = ctypes.c_double
+        L.specdec_tier_select.argtypes = [P, i32, ctypes.c_double]
+        L.specdec_tier_select.restype = i32
         _lib = L
     return _lib
 
@@ -194,6 +198,19 @@ def specdec_verify_rejection_ragged(target_logits, dtype, row_stride, draft_prob
                                                  int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
                                                  _ptr(accept_len), _ptr(out_tokens), _ptr(p_draft_out),
                                                  _ptr(counters), _ptr(ws), ws_bytes, _stream(stream))
+
+
+class specdec_tier_state(ctypes.Structure):
+    _fields_ = [("ema", ctypes.c_double), ("initialized", ctypes.c_int)]
+
+
+def specdec_tier_update(state: "specdec_tier_state", accepted: float, decay: float) -> float:
+    return lib().specdec_tier_update(ctypes.byref(state), float(accepted), float(decay))
+
+
+def specdec_tier_select(tiers, ema: float) -> int:
+    arr = (ctypes.c_int * len(tiers))(*[int(t) for t in tiers])
+    return lib().specdec_tier_select(ctypes.cast(arr, ctypes.c_void_p), len(tiers), float(ema))
 
 
 def _check(status, what):

@@ -432,6 +432,29 @@ specdec_status specdec_verify_rejection_ragged(const void* target_logits, specde
                           counters, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+double specdec_tier_update(specdec_tier_state* state, double accepted, double decay) {
+    if (state == nullptr || !(decay >= 0.0 && decay < 1.0) || !(accepted >= 0.0 && accepted <= SPECDEC_MAX_K))
+        return NAN;
+    if (!state->initialized) {
+        state->ema = accepted;
+        state->initialized = 1;
+    } else {
+        state->ema = decay * state->ema + (1.0 - decay) * accepted;
+    }
+    return state->ema;
+}
+
+int specdec_tier_select(const int* tiers, int n_tiers, double ema) {
+    if (tiers == nullptr || n_tiers < 1 || !(ema >= 0.0)) return -1;
+    for (int i = 0; i < n_tiers; ++i) {
+        if (tiers[i] < 0 || tiers[i] > SPECDEC_MAX_K) return -1;
+        if (i > 0 && tiers[i] <= tiers[i - 1]) return -1;
+    }
+    for (int i = 0; i < n_tiers; ++i)
+        if (static_cast<double>(tiers[i]) >= ema + 0.5) return tiers[i];
+    return tiers[n_tiers - 1];
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
