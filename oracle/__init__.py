@@ -33,9 +33,14 @@ def _bind(path):
     L.oracle_verify_greedy_ragged.argtypes = [P, i32, i64, P, P, i32, i64, i32, i32, P, P, i32, P, P, P]
     L.oracle_verify_rejection_ragged.argtypes = [P, i32, i64, P, i64, P, P, i32, i64, i32, i32, f64, u64, u64,
                                                  P, P, P, P, P]
+    L.oracle_verify_greedy_parallel.argtypes = [P, i32, i64, P, i32, i32, i32, P, P, i32, P, P, i32]
+    L.oracle_verify_tree_parallel.argtypes = [P, i32, i64, P, P, i32, i32, i32, i32, P, P, P, i32]
+    L.oracle_verify_rejection_parallel.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f64, u64, u64,
+                                                   P, P, P, P, i32]
     for f in ("oracle_philox4x32_10", "oracle_uniforms", "oracle_argmax_rows", "oracle_topk_rows",
               "oracle_verify_greedy", "oracle_verify_tree", "oracle_verify_rejection",
-              "oracle_verify_greedy_ragged", "oracle_verify_rejection_ragged"):
+              "oracle_verify_greedy_ragged", "oracle_verify_rejection_ragged", "oracle_verify_greedy_parallel",
+              "oracle_verify_tree_parallel", "oracle_verify_rejection_parallel"):
         getattr(L, f).restype = None
     return L
 
@@ -116,7 +121,7 @@ def topk_rows(logits, dtype, topk):
     return ids.reshape(x.shape[:-1] + (topk,)), vals.reshape(x.shape[:-1] + (topk,))
 
 
-def verify_greedy(logits, dtype, drafts, topk=0):
+def verify_greedy(logits, dtype, drafts, topk=0, threads=1):
     """logits [B, k+1, V]; drafts [B, k] -> (accept_len, out_tokens[, topk_ids, topk_vals])."""
     x = _logit_array(logits, dtype)
     B, k1, V = x.shape
@@ -126,14 +131,18 @@ def verify_greedy(logits, dtype, drafts, topk=0):
     out = np.zeros((B, k1), np.int32)
     ids = np.zeros((B, k1, max(topk, 1)), np.int32)
     vals = np.zeros((B, k1, max(topk, 1)), np.float32)
-    lib().oracle_verify_greedy(_ptr(x), DTYPE_CODE[dtype], V, _ptr(d), B, k, V, _ptr(al), _ptr(out),
-                               topk, _ptr(ids), _ptr(vals))
+    if threads > 1:
+        lib().oracle_verify_greedy_parallel(_ptr(x), DTYPE_CODE[dtype], V, _ptr(d), B, k, V, _ptr(al), _ptr(out),
+                                            topk, _ptr(ids), _ptr(vals), threads)
+    else:
+        lib().oracle_verify_greedy(_ptr(x), DTYPE_CODE[dtype], V, _ptr(d), B, k, V, _ptr(al), _ptr(out),
+                                   topk, _ptr(ids), _ptr(vals))
     if topk > 0:
         return al, out, ids, vals
     return al, out
 
 
-def verify_tree(logits, dtype, parents, node_tokens, max_depth):
+def verify_tree(logits, dtype, parents, node_tokens, max_depth, threads=1):
     """logits [B, N+1, V] -> (accept_len, accept_nodes, out_tokens)."""
     x = _logit_array(logits, dtype)
     B, n1, V = x.shape
@@ -142,12 +151,14 @@ def verify_tree(logits, dtype, parents, node_tokens, max_depth):
     al = np.zeros(B, np.int32)
     nodes = np.zeros((B, max_depth), np.int32)
     out = np.zeros((B, max_depth + 1), np.int32)
-    lib().oracle_verify_tree(_ptr(x), DTYPE_CODE[dtype], V, _ptr(par), _ptr(tok), B, n1 - 1, V, max_depth,
-                             _ptr(al), _ptr(nodes), _ptr(out))
+    fn = lib().oracle_verify_tree_parallel if threads > 1 else lib().oracle_verify_tree
+    extra = (threads,) if threads > 1 else ()
+    fn(_ptr(x), DTYPE_CODE[dtype], V, _ptr(par), _ptr(tok), B, n1 - 1, V, max_depth, _ptr(al), _ptr(nodes),
+       _ptr(out), *extra)
     return al, nodes, out
 
 
-def verify_rejection(target, dtype, q, drafts, temperature, seed, offset):
+def verify_rejection(target, dtype, q, drafts, temperature, seed, offset, threads=1):
     """target [B, k+1, V]; q [B, k, V] float32 -> (accept_len, out_tokens, p_draft, margin)."""
     x = _logit_array(target, dtype)
     B, k1, V = x.shape
@@ -158,9 +169,10 @@ def verify_rejection(target, dtype, q, drafts, temperature, seed, offset):
     out = np.zeros((B, k1), np.int32)
     pd = np.zeros((B, max(k, 1)), np.float64)
     mg = np.zeros(B, np.float64)
-    lib().oracle_verify_rejection(_ptr(x), DTYPE_CODE[dtype], V, _ptr(qq), V, _ptr(d), B, k, V,
-                                  float(temperature), int(seed), int(offset),
-                                  _ptr(al), _ptr(out), _ptr(pd), _ptr(mg))
+    fn = lib().oracle_verify_rejection_parallel if threads > 1 else lib().oracle_verify_rejection
+    extra = (threads,) if threads > 1 else ()
+    fn(_ptr(x), DTYPE_CODE[dtype], V, _ptr(qq), V, _ptr(d), B, k, V, float(temperature), int(seed), int(offset),
+       _ptr(al), _ptr(out), _ptr(pd), _ptr(mg), *extra)
     return al, out, pd[:, :k], mg
 
 

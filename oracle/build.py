@@ -1,7 +1,9 @@
 """Build the CPU oracle (test infrastructure) into oracle/_build/liboracle.so.
 
-Plain single-threaded C++17, compiled with g++ -O2 (no -ffast-math: the
-oracle's fp64 arithmetic must follow IEEE order as written).
+Plain C++17, compiled with g++ -O2 (no -ffast-math: the oracle's fp64
+arithmetic must follow IEEE order as written).  Every function is
+single-threaded except the request-parallel timing drivers, which run the
+same per-request code on std::threads.
 """
 from __future__ import annotations
 
@@ -19,7 +21,7 @@ def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
     tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = ["g++", "-std=c++17", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared",
+    cmd = ["g++", "-std=c++17", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
            SRC, "-o", tmp]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)

@@ -50,6 +50,7 @@
 #include <cstdint>
 #include <cstring>
 #include <limits>
+#include <thread>
 #include <vector>
 
 namespace {
@@ -285,6 +286,21 @@ void rejection_request(const void* target, int dtype, int64_t row_stride, int64_
     *margin = mg;
 }
 
+// Runs fn(b0, b1) on `threads` std::threads over contiguous blocks of [0, B).
+template <class F>
+void for_request_blocks(int B, int threads, F fn) {
+    if (threads < 1) threads = 1;
+    if (threads > B) threads = B > 0 ? B : 1;
+    std::vector<std::thread> pool;
+    for (int t = 0; t < threads; ++t) {
+        const int b0 = (int)((int64_t)B * t / threads), b1 = (int)((int64_t)B * (t + 1) / threads);
+        pool.emplace_back([=] { fn(b0, b1); });
+    }
+    for (auto& th : pool) th.join();
+}
+
+int elem_bytes(int dtype) { return dtype == 1 ? 2 : 4; }
+
 }  // namespace
 
 extern "C" {
@@ -486,6 +502,49 @@ void oracle_verify_rejection_ragged(const void* target, int dtype, int64_t row_s
                           seed, offset, (uint32_t)b, &accept_len[b], out_tokens + row0, p_draft + o0, &margin[b]);
         if (counters && accept_len[b] >= 0) count_request(counters, kb, accept_len[b]);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Request-parallel drivers, for timing the oracle on all host cores.  The
+// requests of a call are independent, so `threads` std::threads each run the
+// unchanged code above on a contiguous block of requests (the uniforms stay
+// keyed by the global request index); results equal the sequential calls.
+// ---------------------------------------------------------------------------
+void oracle_verify_greedy_parallel(const void* logits, int dtype, int64_t row_stride, const int32_t* drafts,
+                                   int B, int k, int V, int32_t* accept_len, int32_t* out_tokens, int topk,
+                                   int32_t* topk_ids, float* topk_vals, int threads) {
+    for_request_blocks(B, threads, [&](int b0, int b1) {
+        const int64_t r0 = (int64_t)b0 * (k + 1);
+        const char* base = static_cast<const char*>(logits) + r0 * row_stride * elem_bytes(dtype);
+        oracle_verify_greedy(base, dtype, row_stride, drafts + (int64_t)b0 * k, b1 - b0, k, V, accept_len + b0,
+                             out_tokens + r0, topk, topk > 0 ? topk_ids + r0 * topk : nullptr,
+                             topk > 0 ? topk_vals + r0 * topk : nullptr);
+    });
+}
+
+void oracle_verify_tree_parallel(const void* logits, int dtype, int64_t row_stride, const int32_t* parents,
+                                 const int32_t* node_tokens, int B, int N, int V, int max_depth,
+                                 int32_t* accept_len, int32_t* accept_nodes, int32_t* out_tokens, int threads) {
+    for_request_blocks(B, threads, [&](int b0, int b1) {
+        const int64_t n1 = N + 1;
+        const char* base = static_cast<const char*>(logits) + (int64_t)b0 * n1 * row_stride * elem_bytes(dtype);
+        oracle_verify_tree(base, dtype, row_stride, parents + b0 * n1, node_tokens + b0 * n1, b1 - b0, N, V,
+                           max_depth, accept_len + b0, accept_nodes + (int64_t)b0 * max_depth,
+                           out_tokens + (int64_t)b0 * (max_depth + 1));
+    });
+}
+
+void oracle_verify_rejection_parallel(const void* target, int dtype, int64_t row_stride, const float* q,
+                                      int64_t q_row_stride, const int32_t* drafts, int B, int k, int V,
+                                      double temperature, uint64_t seed, uint64_t offset, int32_t* accept_len,
+                                      int32_t* out_tokens, double* p_draft, double* margin, int threads) {
+    for_request_blocks(B, threads, [&](int b0, int b1) {
+        for (int b = b0; b < b1; ++b)
+            rejection_request(target, dtype, row_stride, (int64_t)b * (k + 1), q, q_row_stride, (int64_t)b * k,
+                              drafts + (int64_t)b * k, k, V, temperature, seed, offset, (uint32_t)b,
+                              &accept_len[b], out_tokens + (int64_t)b * (k + 1), p_draft + (int64_t)b * k,
+                              &margin[b]);
+    });
 }
 
 }  // extern "C"

@@ -154,3 +154,21 @@ def test_tier_workload_acceptance_closed_form():
         assert abs(ctr[3 + i] / B - p) < 4 * math.sqrt(p * (1 - p) / B) + 1e-12, i
     mean_tau = np.mean([(1 - alpha ** (t + 1)) / (1 - alpha) for t in kb])  # handbook "Key metrics" closed form
     assert abs((ctr[0] + ctr[2]) / B - mean_tau) < 4 * np.sqrt(np.var(al + 1) / B)
+
+
+def test_parallel_drivers_equal_sequential():
+    """The request-parallel timing drivers run the same per-request code:
+    results equal the sequential oracle exactly."""
+    g = gen.greedy_synthetic(seed=31, B=23, k=4, V=900, alpha=0.7, dtype="bf16")
+    a = oracle.verify_greedy(g.logits, "bf16", g.drafts, topk=8)
+    b = oracle.verify_greedy(g.logits, "bf16", g.drafts, topk=8, threads=5)
+    assert all(np.array_equal(x.view(np.uint32) if x.dtype == np.float32 else x,
+                              y.view(np.uint32) if y.dtype == np.float32 else y) for x, y in zip(a, b))
+    t = gen.tree_synthetic(seed=32, B=11, parents=gen.complete_tree_parents([3, 2]), V=300, dtype="f32")
+    a = oracle.verify_tree(t.logits, "f32", t.parents, t.node_tokens, t.max_depth)
+    b = oracle.verify_tree(t.logits, "f32", t.parents, t.node_tokens, t.max_depth, threads=4)
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+    r = gen.rejection_qwen(B=6, V=500)
+    a = oracle.verify_rejection(r.target, r.dtype, r.q, r.drafts, 1.0, 7, 1)
+    b = oracle.verify_rejection(r.target, r.dtype, r.q, r.drafts, 1.0, 7, 1, threads=3)
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
