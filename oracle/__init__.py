@@ -37,7 +37,8 @@ def _bind(path):
     L.oracle_verify_tree_parallel.argtypes = [P, i32, i64, P, P, i32, i32, i32, i32, P, P, P, i32]
     L.oracle_verify_rejection_parallel.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f64, u64, u64,
                                                    P, P, P, P, i32]
-    for f in ("oracle_philox4x32_10", "oracle_uniforms", "oracle_argmax_rows", "oracle_topk_rows",
+    L.oracle_draft_stats.argtypes = [P, i32, i64, P, i64, i32, i32, i32, f64, P, P]
+    for f in ("oracle_draft_stats", "oracle_philox4x32_10", "oracle_uniforms", "oracle_argmax_rows", "oracle_topk_rows",
               "oracle_verify_greedy", "oracle_verify_tree", "oracle_verify_rejection",
               "oracle_verify_greedy_ragged", "oracle_verify_rejection_ragged", "oracle_verify_greedy_parallel",
               "oracle_verify_tree_parallel", "oracle_verify_rejection_parallel"):
@@ -237,3 +238,16 @@ def verify_rejection_ragged(target, dtype, q, drafts, offsets, max_k, temperatur
                                          max_k, V, float(temperature), int(seed), int(offset), _ptr(al), _ptr(out),
                                          _ptr(pd), _ptr(mg), _ptr(ctr))
     return al, out, pd[:T], mg, ctr
+
+
+def draft_stats(target, dtype, q, temperature):
+    """target [B, k+1, V]; q [B, k, V] float32 -> (entropy [B, k], js_distance
+    [B, k]) in nats (AdaSD's statistics)."""
+    x = _logit_array(target, dtype)
+    B, k1, V = x.shape
+    k = k1 - 1
+    qq = _c(q, np.float32).reshape(B, k, V) if k > 0 else np.zeros((B, 0, V), np.float32)
+    e = np.zeros((B, max(k, 1)), np.float64)
+    j = np.zeros((B, max(k, 1)), np.float64)
+    lib().oracle_draft_stats(_ptr(x), DTYPE_CODE[dtype], V, _ptr(qq), V, B, k, V, float(temperature), _ptr(e), _ptr(j))
+    return e[:, :k], j[:, :k]

@@ -504,6 +504,63 @@ void oracle_verify_rejection_ragged(const void* target, int dtype, int64_t row_s
     }
 }
 
+// Statistics of AdaSD's adaptive rules ([HANDBOOK] "Adaptive speculative
+// decoding", AdaSD: the draft token's entropy decides when drafting stops,
+// the Jensen-Shannon distance between the draft and target distributions
+// decides whether a draft token is close enough to accept).  Per request b
+// and draft position i < k, with p_i = softmax(l_i / T) and q_i as given:
+//   entropy[b, i] = H(q_i) = -sum_x q log q                     (nats)
+//   js[b, i]      = sqrt(D_JS(p_i, q_i)), D_JS = (KL(p || m) + KL(q || m)) / 2,
+//                   m = (p + q) / 2                              (nats)
+// with 0 log 0 = 0.  A request whose target rows 0..k hold NaN or +inf or a
+// row of only -inf (the rejection verifier's invalid case) gets NaN.
+void oracle_draft_stats(const void* target, int dtype, int64_t row_stride, const float* q, int64_t q_row_stride,
+                        int B, int k, int V, double temperature, double* entropy, double* js) {
+    const double T = temperature;
+    std::vector<double> p(V);
+    for (int b = 0; b < B; ++b) {
+        bool valid = true;
+        for (int i = 0; i <= k && valid; ++i) {
+            const int64_t row = (int64_t)b * (k + 1) + i;
+            bool any = false;
+            for (int x = 0; x < V; ++x) {
+                const float l = logit_at(target, dtype, row_stride, row, x);
+                if (std::isnan(l) || (std::isinf(l) && l > 0)) valid = false;
+                if (!(std::isinf(l) && l < 0)) any = true;
+            }
+            if (!any) valid = false;
+        }
+        for (int i = 0; i < k; ++i) {
+            double* e = entropy + (int64_t)b * k + i;
+            double* j = js + (int64_t)b * k + i;
+            if (!valid) {
+                *e = *j = std::numeric_limits<double>::quiet_NaN();
+                continue;
+            }
+            const int64_t row = (int64_t)b * (k + 1) + i;
+            double mx = -std::numeric_limits<double>::infinity();
+            for (int x = 0; x < V; ++x)
+                mx = std::max(mx, static_cast<double>(logit_at(target, dtype, row_stride, row, x)) / T);
+            double Z = 0.0;
+            for (int x = 0; x < V; ++x) {
+                p[x] = std::exp(static_cast<double>(logit_at(target, dtype, row_stride, row, x)) / T - mx);
+                Z += p[x];
+            }
+            double H = 0.0, D = 0.0;
+            const float* qr = q + ((int64_t)b * k + i) * q_row_stride;
+            for (int x = 0; x < V; ++x) {
+                const double px = p[x] / Z, qx = static_cast<double>(qr[x]);
+                const double m = 0.5 * (px + qx);
+                if (qx > 0.0) H -= qx * std::log(qx);
+                if (px > 0.0) D += 0.5 * px * std::log(px / m);
+                if (qx > 0.0) D += 0.5 * qx * std::log(qx / m);
+            }
+            *e = H;
+            *j = std::sqrt(std::max(0.0, D));
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Request-parallel drivers, for timing the oracle on all host cores.  The
 // requests of a call are independent, so `threads` std::threads each run the

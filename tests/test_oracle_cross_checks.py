@@ -18,6 +18,7 @@ import oracle
 from oracle import build as oracle_build
 
 import test_oracle_pins as pins
+import test_oracle_adasd as adasd
 
 TORCH_PHILOX_MAIN = r"""
 #include <ATen/core/PhiloxRNGEngine.h>
@@ -105,6 +106,18 @@ MUTANTS = [
      "ok[c] = ok[par[c]] && t >= 0 && t < V && t == am[par[c]];",
      "ok[c] = ok[par[c]] && t >= 0 && t < V && t == am[c];",
      [pins.test_tree_brute_force_small, pins.test_tree_chain_reduces_to_greedy]),
+    ("AdaSD: Jensen-Shannon mixture not halved",
+     "const double m = 0.5 * (px + qx);",
+     "const double m = (px + qx);",
+     [lambda: adasd.test_matches_scipy(1.0), adasd.test_closed_forms]),
+    ("AdaSD: divergence terms not halved",
+     "if (px > 0.0) D += 0.5 * px * std::log(px / m);",
+     "if (px > 0.0) D += px * std::log(px / m);",
+     [lambda: adasd.test_matches_scipy(1.0), adasd.test_closed_forms]),
+    ("AdaSD: entropy of the target instead of the draft",
+     "if (qx > 0.0) H -= qx * std::log(qx);",
+     "if (px > 0.0) H -= px * std::log(px);",
+     [lambda: adasd.test_matches_scipy(1.0), adasd.test_closed_forms]),
 ]
 
 
