@@ -85,9 +85,13 @@ def recorded_traffic(workload):
 def make_workload(name, seed_offset=0):
     base = {"greedy_llama3": (gen.greedy_llama3, 1), "greedy_tiny": (gen.greedy_tiny, 0),
             "greedy_large_batch": (gen.greedy_large_batch, 3), "tree_medusa": (gen.tree_medusa, 4),
-            "rejection_qwen": (gen.rejection_qwen, 2), "greedy_ragged_tiers": (gen.greedy_ragged_tiers, 6)}
+            "rejection_qwen": (gen.rejection_qwen, 2), "greedy_ragged_tiers": (gen.greedy_ragged_tiers, 6),
+            "rejection_qwen_adasd": (gen.rejection_qwen, 2)}
     fn, seed = base[name]
-    return fn(seed=seed + 1000 * seed_offset)
+    inp = fn(seed=seed + 1000 * seed_offset)
+    if name == "rejection_qwen_adasd":
+        inp.stats = True
+    return inp
 
 
 def describe(inp):
@@ -103,6 +107,8 @@ def describe(inp):
         d["topk"] = inp.topk
     if isinstance(inp, gen.RejectionInputs):
         d["temperature"] = inp.temperature
+        if inp.stats:
+            d["adasd_stats"] = "draft entropy and Jensen-Shannon distance per draft position"
     return d
 
 
@@ -181,7 +187,10 @@ def resample_bytes(inp, outs):
     es = 2 if inp.dtype == gen.BF16 else 4
     al = outs[0].cpu().numpy()
     ok = al >= 0
-    return int(inp.V * (es * ok.sum() + 4 * (ok & (al < inp.k)).sum()))
+    extra = 0
+    if inp.stats:  # AdaSD statistics: target rows 0..k-1 and their q rows once more, 16 B out per position
+        extra = int(ok.sum()) * inp.k * (inp.V * (es + 4) + 16)
+    return int(inp.V * (es * ok.sum() + 4 * (ok & (al < inp.k)).sum())) + extra
 
 
 def setup_calls(inp, sets, ver, device):
@@ -204,10 +213,15 @@ def setup_calls(inp, sets, ver, device):
         ot = torch.empty(B, inp.k + 1, dtype=torch.int32, device=device)
         pd = torch.empty(B, max(inp.k, 1), dtype=torch.float32, device=device)
         outs = (al, ot, pd)
+        if inp.stats:
+            outs = outs + (torch.empty(B, max(inp.k, 1), dtype=torch.float64, device=device),
+                           torch.empty(B, max(inp.k, 1), dtype=torch.float64, device=device))
         for s in sets:
             calls.append(lambda s=s: ver.rejection(s["target"], s["q"], s["drafts"], inp.temperature, inp.seed,
-                                                   inp.offset, out=outs))
+                                                   inp.offset, out=outs, stats=inp.stats))
         kernels = 4  # softmax pass, request epilogue, chunk masses, token search
+        if inp.stats:
+            kernels += 2  # statistics chunks, statistics per position
     elif isinstance(inp, gen.RaggedInputs):
         R, T = inp.rows, int(inp.offsets[-1])
         al = torch.empty(B, dtype=torch.int32, device=device)
@@ -477,8 +491,11 @@ def oracle_call(inp, req, threads=1):
         return oracle.verify_tree(inp.logits[:req], inp.dtype, inp.parents[:req], inp.node_tokens[:req],
                                   inp.max_depth, threads=threads)
     if isinstance(inp, gen.RejectionInputs):
-        return oracle.verify_rejection(inp.target[:req], inp.dtype, inp.q[:req], inp.drafts[:req],
-                                       inp.temperature, inp.seed, inp.offset, threads=threads)
+        res = oracle.verify_rejection(inp.target[:req], inp.dtype, inp.q[:req], inp.drafts[:req],
+                                      inp.temperature, inp.seed, inp.offset, threads=threads)
+        if inp.stats:
+            res = res + oracle.draft_stats(inp.target[:req], inp.dtype, inp.q[:req], inp.temperature)
+        return res
     if isinstance(inp, gen.RaggedInputs):
         t = int(inp.offsets[req])
         return oracle.verify_greedy_ragged(inp.logits[:t + req], inp.dtype, inp.drafts[:t], inp.offsets[:req + 1],
@@ -556,7 +573,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="greedy_llama3",
                     choices=["greedy_llama3", "greedy_tiny", "rejection_qwen", "greedy_large_batch", "tree_medusa",
-                             "greedy_ragged_tiers"])
+                             "greedy_ragged_tiers", "rejection_qwen_adasd"])
     ap.add_argument("--sets", type=int, default=None, help="input sets in the rotation (default: > 4x L2)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)

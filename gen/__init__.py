@@ -122,6 +122,7 @@ class RejectionInputs:
     temperature: float = 1.0
     seed: int = 1234
     offset: int = 0
+    stats: bool = False  # also compute AdaSD's draft statistics
 
 
 @dataclass

@@ -175,6 +175,27 @@ specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int6
                                    int32_t* accept_len, int32_t* accept_nodes, int32_t* out_tokens,
                                    void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
+/* Rejection-sampling verification plus AdaSD's statistics (handbook page,
+ * "Adaptive speculative decoding", AdaSD: the draft token's entropy decides
+ * when drafting stops, the Jensen-Shannon distance between the draft and
+ * target distributions decides whether a draft token is close enough to
+ * accept).  Arguments and results as specdec_verify_rejection, plus
+ *   draft_entropy [B, k] float64 out: H(q_i) = -sum_x q log q (nats)
+ *   js_distance   [B, k] float64 out: sqrt(D_JS(p_i, q_i)) with
+ *                 D_JS = (KL(p || m) + KL(q || m)) / 2, m = (p + q) / 2, in
+ *                 nats; p_i = softmax(l_i / T)
+ * (0 log 0 = 0; NaN for a request whose target distributions are undefined).
+ * The verification itself is unchanged: the page gives no rule for turning
+ * the statistics into thresholds.  Two more kernels are enqueued, which read
+ * target rows 0..k-1 and the q rows once more. */
+specdec_status specdec_verify_rejection_stats(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
+                                              const float* draft_probs, int64_t q_row_stride,
+                                              const int32_t* draft_tokens, int B, int k, int V, float temperature,
+                                              uint64_t seed, uint64_t offset, int32_t* accept_len,
+                                              int32_t* out_tokens, float* p_draft_out, double* draft_entropy,
+                                              double* js_distance, void* ws, size_t ws_bytes,
+                                              struct CUstream_st* stream);
+
 /* ---------------------------------------------------------------------------
  * Variable speculation length per request (handbook page, "Adaptive
  * speculative decoding": the speculation length is changed per batch or

@@ -100,6 +100,9 @@ def lib():
         L.specdec_verify_rejection_ragged.argtypes = [P, i32, i64, P, i64, P, P, i32, i32, i32, i32, f32, u64,
                                                       u64, P, P, P, P, P, sz, P]
         L.specdec_verify_rejection_ragged.restype = i32
+        L.specdec_verify_rejection_stats.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f32, u64, u64,
+                                                     P, P, P, P, P, P, sz, P]
+        L.specdec_verify_rejection_stats.restype = i32
         L.specdec_tier_update.argtypes = [P, ctypes.c_double, ctypes.c_double]
         L.specdec_tier_update.restype = ctypes.c_double
         L.specdec_tier_select.argtypes = [P, i32, ctypes.c_double]
@@ -162,6 +165,17 @@ def specdec_verify_rejection(target_logits, dtype, row_stride, draft_probs, q_ro
                                           int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
                                           _ptr(accept_len), _ptr(out_tokens), _ptr(p_draft_out),
                                           _ptr(ws), ws_bytes, _stream(stream))
+
+
+def specdec_verify_rejection_stats(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens,
+                                   B, k, V, temperature, seed, offset, accept_len, out_tokens, p_draft_out,
+                                   draft_entropy, js_distance, ws, ws_bytes, stream=None) -> int:
+    return lib().specdec_verify_rejection_stats(_ptr(target_logits), dtype, row_stride, _ptr(draft_probs),
+                                                q_row_stride, _ptr(draft_tokens), B, k, V, float(temperature),
+                                                int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
+                                                _ptr(accept_len), _ptr(out_tokens), _ptr(p_draft_out),
+                                                _ptr(draft_entropy), _ptr(js_distance), _ptr(ws), ws_bytes,
+                                                _stream(stream))
 
 
 def specdec_verify_tree(logits, dtype, row_stride, parents, node_tokens, B, N, V, max_depth,
@@ -323,9 +337,11 @@ class Verifier:
         return al, nodes, ot
 
     def rejection(self, target_logits, draft_probs, draft_tokens, temperature: float, seed: int, offset: int = 0,
-                  stream=None, out=None, want_p_draft: bool = True):
+                  stream=None, out=None, want_p_draft: bool = True, stats: bool = False):
         """target_logits [B, k+1, V], draft_probs [B, k, V] f32, draft_tokens
-        [B, k] int32 -> (accept_len [B], out_tokens [B, k+1], p_draft [B, k])."""
+        [B, k] int32 -> (accept_len [B], out_tokens [B, k+1], p_draft [B, k]);
+        with stats=True also (draft_entropy [B, k], js_distance [B, k]) float64
+        (AdaSD's statistics; `out` then holds five tensors)."""
         import torch
         B, k1, V = target_logits.shape
         k = k1 - 1
@@ -343,13 +359,21 @@ class Verifier:
             al = torch.empty(B, dtype=torch.int32, device=dev)
             ot = torch.empty(B, k1, dtype=torch.int32, device=dev)
             pd = torch.empty(B, max(k, 1), dtype=torch.float32, device=dev) if want_p_draft else None
+            ent = torch.empty(B, max(k, 1), dtype=torch.float64, device=dev) if stats else None
+            js = torch.empty(B, max(k, 1), dtype=torch.float64, device=dev) if stats else None
         else:
-            al, ot, pd = out
+            al, ot, pd, ent, js = (tuple(out) + (None, None))[:5]
         need = specdec_workspace_size(SPECDEC_MODE_REJECTION, B, k, V, dt)
         ws, wsb = self.workspace(need, stream)
-        _check(specdec_verify_rejection(target_logits, dt, stride, draft_probs if k > 0 else None, q_stride,
-                                        draft_tokens if k > 0 else None, B, k, V, temperature, seed, offset,
-                                        al, ot, pd, ws, wsb, stream), "verify_rejection")
+        q = draft_probs if k > 0 else None
+        d = draft_tokens if k > 0 else None
+        if stats:
+            _check(specdec_verify_rejection_stats(target_logits, dt, stride, q, q_stride, d, B, k, V, temperature,
+                                                  seed, offset, al, ot, pd, ent, js, ws, wsb, stream),
+                   "verify_rejection_stats")
+            return al, ot, (pd[:, :k] if pd is not None else None), ent[:, :k], js[:, :k]
+        _check(specdec_verify_rejection(target_logits, dt, stride, q, q_stride, d, B, k, V, temperature, seed,
+                                        offset, al, ot, pd, ws, wsb, stream), "verify_rejection")
         return al, ot, (pd[:, :k] if pd is not None else None)
 
 

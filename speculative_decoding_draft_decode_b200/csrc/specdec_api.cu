@@ -18,6 +18,7 @@
 #include "../../include/specdec.h"
 #include "verify_pass1.cuh"
 #include "verify_resample.cuh"
+#include "verify_stats.cuh"
 
 namespace specdec {
 namespace {
@@ -29,7 +30,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
     int64_t nv = 0, nv_full = 0, cpr = 0, NC = 0, cpr2 = 0;
-    size_t partials1 = 0, state = 0, masses = 0, units = 0, total = 0;
+    size_t partials1 = 0, state = 0, masses = 0, units = 0, row_stat = 0, chunk_stats = 0, total = 0;
 };
 
 // Layout of one call.  `vec` = elements per vector (1 on the scalar path),
@@ -53,6 +54,11 @@ Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t
         L.units = align_up(end, 256);
         end = L.units + static_cast<size_t>(B) * static_cast<size_t>(L.cpr2) *
                             static_cast<size_t>(units_per_chunk(vec)) * sizeof(double2);
+        // draft statistics (fixed layout: rows - B = B k draft rows)
+        L.row_stat = align_up(end, 256);
+        end = L.row_stat + static_cast<size_t>(rows) * sizeof(RowStat);
+        L.chunk_stats = align_up(end, 256);
+        end = L.chunk_stats + static_cast<size_t>(rows - B) * static_cast<size_t>(L.cpr2) * sizeof(double2);
     }
     (void)rows_per_req;
     L.total = align_up(end, 256);
@@ -138,6 +144,25 @@ specdec_status dispatch_pass2(specdec_dtype dt, bool vec, Pass2Params P, cudaStr
     return vec ? launch_pass2<F32Tag, 4>(P, s) : launch_pass2<F32Tag, 1>(P, s);
 }
 
+// AdaSD statistics: the chunk sums of every draft row, then a warp per
+// (request, position).
+template <class Tag, int VEC>
+specdec_status launch_stats(StatsParams S, cudaStream_t stream) {
+    const int64_t rows = static_cast<int64_t>(S.B) * S.k;
+    if (S.cpr > 65535 || rows > 0x7fffffff) return SPECDEC_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>(rows), static_cast<unsigned>(S.cpr));
+    if (launch_pdl(verify_stats_kernel<Tag, VEC>, grid, 0, stream, S) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    if (launch_pdl(verify_stats_epilogue_kernel, dim3(static_cast<unsigned>((rows + NWARPS - 1) / NWARPS)), 0,
+                   stream, S) != cudaSuccess)
+        return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+specdec_status dispatch_stats(specdec_dtype dt, bool vec, StatsParams S, cudaStream_t s) {
+    if (dt == SPECDEC_BF16) return vec ? launch_stats<BF16Tag, 8>(S, s) : launch_stats<BF16Tag, 1>(S, s);
+    return vec ? launch_stats<F32Tag, 4>(S, s) : launch_stats<F32Tag, 1>(S, s);
+}
+
 bool dtype_ok(specdec_dtype dt) { return dt == SPECDEC_F32 || dt == SPECDEC_BF16; }
 
 // Pass-1 partial bytes per chunk: one argmax key per warp, 8 keys per warp
@@ -218,7 +243,8 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
                               const float* draft_probs, int64_t q_row_stride, const int32_t* draft_tokens,
                               const int32_t* offsets, int64_t total, int B, int k, int V, float temperature,
                               uint64_t seed, uint64_t offset, int32_t* accept_len, int32_t* out_tokens,
-                              float* p_draft_out, int64_t* counters, void* ws, size_t ws_bytes, cudaStream_t s) {
+                              float* p_draft_out, int64_t* counters, double* entropy, double* js, void* ws,
+                              size_t ws_bytes, cudaStream_t s) {
     if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
     const int64_t rows = offsets ? B + total : static_cast<int64_t>(B) * (k + 1);
     if (!rows_fit(rows, row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
@@ -250,6 +276,8 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     P.offset = offset;
     P.p_draft_out = p_draft_out;
     P.state = state;
+    const bool stats = entropy != nullptr && offsets == nullptr && k > 0;
+    P.row_stat = stats ? reinterpret_cast<RowStat*>(static_cast<char*>(ws) + L.row_stat) : nullptr;
     st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
     if (st != SPECDEC_OK) return st;
     Pass2Params Q;
@@ -270,7 +298,26 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     Q.chunk_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.masses);
     Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
     Q.out_tokens = out_tokens;
-    return dispatch_pass2(dtype, vec, Q, s);
+    st = dispatch_pass2(dtype, vec, Q, s);
+    if (st != SPECDEC_OK || !stats) return st;
+    StatsParams S;
+    memset(&S, 0, sizeof(S));
+    S.logits = target_logits;
+    S.row_stride = row_stride;
+    S.q = draft_probs;
+    S.q_stride = q_row_stride;
+    S.V = V;
+    S.nv_full = static_cast<int>(L.nv_full);
+    S.cpr = static_cast<int>(L.cpr2);
+    S.B = B;
+    S.k = k;
+    S.invT = static_cast<float>(invT_d);
+    S.state = state;
+    S.row_stat = P.row_stat;
+    S.chunk_stats = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.chunk_stats);
+    S.entropy = entropy;
+    S.js = js;
+    return dispatch_stats(dtype, vec, S, s);
 }
 
 // Host checks of a packed-layout call.
@@ -412,7 +459,27 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
     if (B == 0) return SPECDEC_OK;
     return rejection_impl(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens, nullptr,
                           static_cast<int64_t>(B) * k, B, k, V, temperature, seed, offset, accept_len, out_tokens,
-                          p_draft_out, nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+                          p_draft_out, nullptr, nullptr, nullptr, ws, ws_bytes,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+specdec_status specdec_verify_rejection_stats(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
+                                              const float* draft_probs, int64_t q_row_stride,
+                                              const int32_t* draft_tokens, int B, int k, int V, float temperature,
+                                              uint64_t seed, uint64_t offset, int32_t* accept_len,
+                                              int32_t* out_tokens, float* p_draft_out, double* draft_entropy,
+                                              double* js_distance, void* ws, size_t ws_bytes,
+                                              struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V < 1 || V > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
+    if (k > 0 && (draft_entropy == nullptr || js_distance == nullptr)) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    return rejection_impl(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens, nullptr,
+                          static_cast<int64_t>(B) * k, B, k, V, temperature, seed, offset, accept_len, out_tokens,
+                          p_draft_out, nullptr, draft_entropy, js_distance, ws, ws_bytes,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 specdec_status specdec_verify_rejection_ragged(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
@@ -429,7 +496,7 @@ specdec_status specdec_verify_rejection_ragged(const void* target_logits, specde
     if (B == 0) return SPECDEC_OK;
     return rejection_impl(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens, draft_offsets,
                           total_drafts, B, max_k, V, temperature, seed, offset, accept_len, out_tokens, p_draft_out,
-                          counters, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+                          counters, nullptr, nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 double specdec_tier_update(specdec_tier_state* state, double accepted, double decay) {

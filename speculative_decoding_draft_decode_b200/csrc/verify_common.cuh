@@ -22,6 +22,14 @@ struct RejState {
     int64_t pad2;
 };
 
+// Row statistics of the softmax pass, kept for every row when the draft
+// statistics are requested: M = max logit, Z = sum exp((l - M) / T).
+struct RowStat {
+    float M;
+    float pad;
+    double Z;
+};
+
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialisation may start while the previous kernel of the stream finishes;
 // griddepcontrol.wait blocks until that kernel has completed and its memory

@@ -108,6 +108,7 @@ struct Pass1Params {
     uint64_t offset;
     float* p_draft_out;
     RejState* state;
+    RowStat* row_stat;          // [rows] every row's (M, Z), or null
 };
 
 // Static shared memory of the pass-1 kernel.
@@ -885,6 +886,14 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
         }
     }
     __syncthreads();
+    if (P.row_stat != nullptr)
+        for (int t = threadIdx.x; t <= k; t += NT) {
+            RowStat rs;
+            rs.M = sm.rowM[t];
+            rs.pad = 0.0f;
+            rs.Z = sm.rowZ[t];
+            P.row_stat[g.row0 + t] = rs;
+        }
     int bad = 0;
     for (int t = threadIdx.x; t <= k; t += NT) {
         const double z = sm.rowZ[t];

@@ -1,0 +1,172 @@
+// verify_stats.cuh — AdaSD's statistics beside rejection verification.
+//
+// Handbook page, "Adaptive speculative decoding" (AdaSD): the draft token's
+// entropy decides when drafting stops, and the Jensen-Shannon distance
+// between the draft and target distributions decides whether a draft token
+// is close enough to accept.  For every request b and draft position i < k,
+// with p_i = softmax(l_i / T) from the row statistics of the softmax pass and
+// q_i as given:
+//   entropy[b, i] = -sum_x q log q                                    (nats)
+//   js[b, i]      = sqrt(D_JS(p_i, q_i)),  D_JS = (KL(p||m) + KL(q||m)) / 2,
+//                   m = (p + q) / 2                                  (nats)
+// with 0 log 0 = 0; NaN for a request whose target distributions are
+// undefined.  Only the statistics: how AdaSD turns them into thresholds is
+// not given on the page.
+//
+// Two kernels after the request epilogue of the softmax pass:
+//   verify_stats_kernel           one CTA per (row (b, i < k), chunk): the
+//                                 chunk's sums of the entropy and JS terms
+//                                 (one exp and two logs per element in fp32,
+//                                 fp32 sums within a 16-byte vector, fp64
+//                                 across vectors);
+//   verify_stats_epilogue_kernel  one warp per (b, i): the chunk sums in
+//                                 index order, then the outputs.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "device_utils.cuh"
+#include "geometry.h"
+#include "verify_common.cuh"
+#include "verify_resample.cuh"
+
+namespace specdec {
+
+struct StatsParams {
+    const void* logits;
+    int64_t row_stride;
+    const float* q;
+    int64_t q_stride;
+    int V;
+    int nv_full;
+    int cpr;  // chunks per row (resample geometry)
+    int B;
+    int k;
+    float invT;
+    const RejState* state;    // [B] validity
+    const RowStat* row_stat;  // [B * (k + 1)]
+    double2* chunk_stats;     // [B * k, cpr] (entropy sum, D_JS sum before the 1/2)
+    double* entropy;          // [B, k]
+    double* js;               // [B, k]
+};
+
+// The entropy and Jensen-Shannon terms of one element, from log p (known
+// from the row statistics: (l - M) / T - ln Z, so p needs one exp and no
+// log) and q: h -= q log q, d += p (log p - log m) + q (log q - log m).
+__device__ __forceinline__ void stat_terms(float lp, float q, float& h, float& d) {
+    const float p = expf(lp);
+    const float lm = logf(0.5f * (p + q));
+    if (q > 0.0f) {
+        const float lq = logf(q);
+        h -= q * lq;
+        d += q * (lq - lm);
+    }
+    if (p > 0.0f) d += p * (lp - lm);
+}
+
+template <class Tag, int VEC>
+__global__ void __launch_bounds__(NT) verify_stats_kernel(const StatsParams P) {
+    __shared__ double red[2][NWARPS];
+    using Elem = typename Tag::storage;
+    constexpr int CH = chunk_vecs(VEC, kU2);
+    constexpr int UPT = chunk_upt(VEC, kU2);
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    const int t = static_cast<int>(threadIdx.x);
+
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    const int64_t x = blockIdx.x;  // b * k + i
+    const int64_t b = x / P.k;
+    const int i = static_cast<int>(x % P.k);
+    const int sub = static_cast<int>(blockIdx.y);
+    if (!P.state[b].valid) return;  // CTA-uniform
+    const RowStat rs = P.row_stat[b * (P.k + 1) + i];
+    const float lnZ = static_cast<float>(log(rs.Z));
+    const Elem* row = static_cast<const Elem*>(P.logits) + (b * (P.k + 1) + i) * P.row_stride;
+    const float* qrow = P.q + x * P.q_stride;
+    const int cnt = chunk_count(P.nv_full, sub, VEC, kU2);
+
+    double h = 0.0, d = 0.0;
+    for (int u0 = 0; u0 < UPT; u0 += kU2) {
+        ResidualVec<Tag, VEC> v[kU2];
+#pragma unroll
+        for (int u = 0; u < kU2; ++u) {
+            const int pos = stream_pos(u0 + u, t);
+            if (pos < cnt) v[u].load(row, qrow, sub * CH + pos, true);
+        }
+#pragma unroll
+        for (int u = 0; u < kU2; ++u) {
+            if (stream_pos(u0 + u, t) < cnt) {
+                float lv[VEC];
+                RowLoader<Tag, VEC>::unpack(v[u].l, lv);
+                float hv = 0.0f, dv = 0.0f;  // one vector in fp32, then fp64
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) stat_terms((lv[e] - rs.M) * P.invT - lnZ, v[u].qv(e), hv, dv);
+                h += static_cast<double>(hv);
+                d += static_cast<double>(dv);
+            }
+        }
+    }
+    if (sub == P.cpr - 1 && wp == 0) {  // the ragged row end
+        const int xe = P.nv_full * VEC + lane;
+        if (xe < P.V) {
+            float hv = 0.0f, dv = 0.0f;
+            stat_terms((load_scalar<Tag>(row + xe) - rs.M) * P.invT - lnZ, __ldg(qrow + xe), hv, dv);
+            h += static_cast<double>(hv);
+            d += static_cast<double>(dv);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        h += __shfl_xor_sync(FULL_MASK, h, o);
+        d += __shfl_xor_sync(FULL_MASK, d, o);
+    }
+    if (lane == 0) {
+        red[0][wp] = h;
+        red[1][wp] = d;
+    }
+    __syncthreads();
+    if (t == 0) {
+        double a = 0.0, c = 0.0;
+#pragma unroll
+        for (int w = 0; w < NWARPS; ++w) {
+            a += red[0][w];
+            c += red[1][w];
+        }
+        P.chunk_stats[x * P.cpr + sub] = make_double2(a, c);
+    }
+}
+
+// One warp per (b, i): the chunk sums (lane-strided, then a fixed butterfly).
+__global__ void __launch_bounds__(NT) verify_stats_epilogue_kernel(const StatsParams P) {
+    const int lane = threadIdx.x & 31;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int64_t x = static_cast<int64_t>(blockIdx.x) * NWARPS + (threadIdx.x >> 5);
+    if (x >= static_cast<int64_t>(P.B) * P.k) return;  // warp-uniform
+    const int64_t b = x / P.k;
+    if (!P.state[b].valid) {
+        if (lane == 0) P.entropy[x] = P.js[x] = __longlong_as_double(0x7ff8000000000000ll);
+        return;
+    }
+    double h = 0.0, d = 0.0;
+    for (int c = lane; c < P.cpr; c += 32) {
+        const double2 s = __ldcg(&P.chunk_stats[x * P.cpr + c]);
+        h += s.x;
+        d += s.y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        h += __shfl_xor_sync(FULL_MASK, h, o);
+        d += __shfl_xor_sync(FULL_MASK, d, o);
+    }
+    if (lane == 0) {
+        P.entropy[x] = h;
+        P.js[x] = sqrt(fmax(0.0, 0.5 * d));
+    }
+}
+
+}  // namespace specdec

@@ -1,0 +1,62 @@
+"""AdaSD's statistics on the GPU (handbook page, "Adaptive speculative
+decoding": draft entropy and the Jensen-Shannon distance between draft and
+target distributions) against the oracle; the verification results of the
+call with statistics equal those of the plain call."""
+import numpy as np
+import pytest
+
+import gen
+import oracle
+from gpu_util import dev_f32, dev_i32, dev_logits, host, require_cuda
+
+pytestmark = pytest.mark.gpu
+
+# fp32 exp and log per element with fp64 sums: relative error ~1e-6 at most
+RTOL, ATOL = 2e-5, 1e-6
+
+
+@pytest.fixture(scope="module")
+def V_():
+    torch = require_cuda()
+    import speculative_decoding_draft_decode_b200 as sd
+    return sd.Verifier(torch.device("cuda", 0))
+
+
+def _run(ver, r, stats):
+    x = dev_logits(r.target, r.dtype)
+    q = dev_f32(r.q)
+    d = dev_i32(r.drafts)
+    res = ver.rejection(x, q, d, r.temperature, r.seed, r.offset, stats=stats)
+    return [host(t) for t in res]
+
+
+def _check(ver, r):
+    got = _run(ver, r, True)
+    plain = _run(ver, r, False)
+    assert np.array_equal(got[0], plain[0]) and np.array_equal(got[1], plain[1])
+    e, j = oracle.draft_stats(r.target, r.dtype, r.q, r.temperature)
+    bad = np.isnan(e)
+    assert np.array_equal(np.isnan(got[3]), bad) and np.array_equal(np.isnan(got[4]), bad)
+    assert np.allclose(got[3][~bad], e[~bad], rtol=RTOL, atol=ATOL), np.max(np.abs(got[3] - e))
+    assert np.allclose(got[4][~bad], j[~bad], rtol=RTOL, atol=ATOL), np.max(np.abs(got[4] - j))
+
+
+def test_adasd_stats_qwen(V_):
+    _check(V_, gen.rejection_qwen())
+
+
+@pytest.mark.parametrize("V,dtype,T", [(1000, "f32", 1.0), (4099, "bf16", 0.7), (33, "f32", 1.4)])
+def test_adasd_stats_small(V_, V, dtype, T):
+    rng = np.random.default_rng(V)
+    B, k = 24, 5
+    tgt = (rng.standard_normal((B, k + 1, V)) * 1.5).astype(np.float32)
+    noisy = tgt[:, :k].astype(np.float64) + rng.standard_normal((B, k, V)) * rng.uniform(0.1, 3, (B, k, 1))
+    q = np.exp(noisy - noisy.max(-1, keepdims=True))
+    q = (q / q.sum(-1, keepdims=True)).astype(np.float32)
+    q[1, 2, : V // 2] = 0.0                  # zeros in q
+    q[1, 2] /= q[1, 2].sum()
+    tgt[2, 3, 7] = np.nan                    # an invalid request
+    tgt[3, 1, : V // 3] = -np.inf            # probability-0 entries in p
+    drafts = np.argmax(q, axis=-1).astype(np.int32)
+    target = gen.f32_to_bf16_bits(tgt) if dtype == "bf16" else tgt
+    _check(V_, gen.RejectionInputs("adasd", dtype, target, q, drafts, B, k, V, temperature=T, seed=5, offset=2))
