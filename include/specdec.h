@@ -287,6 +287,42 @@ typedef struct {
 double specdec_tier_update(specdec_tier_state* state, double accepted, double decay);
 int specdec_tier_select(const int* tiers, int n_tiers, double ema);
 
+/* ---------------------------------------------------------------------------
+ * Vocabulary-sharded greedy verification (Arctic page, "Speculator
+ * optimisation": with the scorer's tensor parallelism each GPU holds a slice
+ * of the vocabulary of every logit row; each takes its own TopK, the results
+ * are all-gathered, and the global TopK is taken from them).  One exchange:
+ *   1. every rank: specdec_shard_greedy_rows over its columns;
+ *   2. all-gather of the row keys (and values) over the ranks, rank order;
+ *   3. every rank (or one): specdec_shard_greedy_combine.
+ * Results equal specdec_verify_greedy on the whole rows.
+ *
+ * Ordered keys: a row result is the uint64 key (ord(value) << 32) | ~index,
+ * index the GLOBAL vocabulary index, where ord maps a float to an unsigned
+ * integer in value order with NaN lowest and -0 equal to +0; a larger key is
+ * the larger value or, among equal values, the lower index; 0 = no element.
+ * ------------------------------------------------------------------------- */
+size_t specdec_workspace_size_shard(int rows, int V_shard, int topk, specdec_dtype dtype);
+
+/* This rank's part: every row's argmax key (topk == 0: row_keys [rows]) or
+ * its 8 best keys and their stored values (topk > 0: row_keys [rows, 8],
+ * row_vals [rows, 8] float32, NaN past the row's end), over this shard's
+ * columns [vocab_offset, vocab_offset + V_shard) of the global vocabulary.
+ *   logits  [rows, V_shard] of `dtype` (this shard's columns), row stride
+ *           `row_stride`; rows = B (k + 1) of the batch being verified */
+specdec_status specdec_shard_greedy_rows(const void* logits, specdec_dtype dtype, int64_t row_stride, int rows,
+                                         int V_shard, int vocab_offset, int topk, uint64_t* row_keys,
+                                         float* row_vals, void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
+/* The combine after the all-gather: gathered_keys [world, B (k+1), kk] (kk =
+ * 8 when topk > 0, else 1) and gathered_vals [world, B (k+1), 8] (topk > 0)
+ * in rank order, 1 <= world <= 32; outputs as specdec_verify_greedy over the
+ * global vocabulary V.  No workspace. */
+specdec_status specdec_shard_greedy_combine(const uint64_t* gathered_keys, const float* gathered_vals, int world,
+                                            const int32_t* draft_tokens, int B, int k, int V, int32_t* accept_len,
+                                            int32_t* out_tokens, int topk, int32_t* topk_ids, float* topk_vals,
+                                            struct CUstream_st* stream);
+
 /* Greedy verification without a caller workspace.  The pages have no
  * counterpart: this entry point exists for callers that cannot allocate
  * device memory (plug-ins and engine hooks handed only input and output

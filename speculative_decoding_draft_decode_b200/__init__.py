@@ -103,6 +103,12 @@ def lib():
         L.specdec_verify_rejection_stats.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f32, u64, u64,
                                                      P, P, P, P, P, P, sz, P]
         L.specdec_verify_rejection_stats.restype = i32
+        L.specdec_workspace_size_shard.argtypes = [i32, i32, i32, i32]
+        L.specdec_workspace_size_shard.restype = sz
+        L.specdec_shard_greedy_rows.argtypes = [P, i32, i64, i32, i32, i32, i32, P, P, P, sz, P]
+        L.specdec_shard_greedy_rows.restype = i32
+        L.specdec_shard_greedy_combine.argtypes = [P, P, i32, P, i32, i32, i32, P, P, i32, P, P, P]
+        L.specdec_shard_greedy_combine.restype = i32
         L.specdec_tier_update.argtypes = [P, ctypes.c_double, ctypes.c_double]
         L.specdec_tier_update.restype = ctypes.c_double
         L.specdec_tier_select.argtypes = [P, i32, ctypes.c_double]
@@ -212,6 +218,23 @@ def specdec_verify_rejection_ragged(target_logits, dtype, row_stride, draft_prob
                                                  int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
                                                  _ptr(accept_len), _ptr(out_tokens), _ptr(p_draft_out),
                                                  _ptr(counters), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def specdec_workspace_size_shard(rows: int, V_shard: int, topk: int, dtype: int) -> int:
+    return lib().specdec_workspace_size_shard(rows, V_shard, topk, dtype)
+
+
+def specdec_shard_greedy_rows(logits, dtype, row_stride, rows, V_shard, vocab_offset, topk, row_keys, row_vals,
+                              ws, ws_bytes, stream=None) -> int:
+    return lib().specdec_shard_greedy_rows(_ptr(logits), dtype, row_stride, rows, V_shard, vocab_offset, topk,
+                                           _ptr(row_keys), _ptr(row_vals), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def specdec_shard_greedy_combine(gathered_keys, gathered_vals, world, draft_tokens, B, k, V, accept_len,
+                                 out_tokens, topk, topk_ids, topk_vals, stream=None) -> int:
+    return lib().specdec_shard_greedy_combine(_ptr(gathered_keys), _ptr(gathered_vals), world, _ptr(draft_tokens),
+                                              B, k, V, _ptr(accept_len), _ptr(out_tokens), topk, _ptr(topk_ids),
+                                              _ptr(topk_vals), _stream(stream))
 
 
 class specdec_tier_state(ctypes.Structure):
@@ -449,6 +472,51 @@ class Verifier:
                                                total_drafts, max_k, V, temperature, seed, offset, al, ot, pd,
                                                counters, ws, wsb, stream), "verify_rejection_ragged")
         return al, ot, (pd[:total_drafts] if pd is not None else None)
+
+
+    # -- vocabulary-sharded greedy -------------------------------------------
+    def shard_greedy_rows(self, logits_shard, vocab_offset: int, topk: int = 0, stream=None, out=None):
+        """logits_shard [B, k+1, V_shard] (this rank's vocabulary columns; a
+        column slice of the full rows is fine) -> row_keys int64 [B (k+1)]
+        (topk == 0) or [B (k+1), 8] with row_vals float32 [B (k+1), 8]:
+        ordered keys with global indices (bit patterns of uint64)."""
+        import torch
+        B, k1, Vs = logits_shard.shape
+        rows = B * k1
+        dt = _dtype_code(logits_shard)
+        stride = _row_stride(logits_shard, "logits_shard")
+        dev = logits_shard.device
+        kk = 8 if topk else 1
+        if out is None:
+            keys = torch.empty(rows, kk, dtype=torch.int64, device=dev)
+            vals = torch.empty(rows, 8, dtype=torch.float32, device=dev) if topk else None
+        else:
+            keys, vals = out
+        need = specdec_workspace_size_shard(rows, Vs, topk, dt)
+        ws, wsb = self.workspace(need, stream)
+        _check(specdec_shard_greedy_rows(logits_shard, dt, stride, rows, Vs, vocab_offset, topk, keys, vals, ws, wsb,
+                                         stream), "shard_greedy_rows")
+        return (keys, vals) if topk else keys
+
+    def shard_greedy_combine(self, gathered_keys, gathered_vals, draft_tokens, V: int, topk: int = 0, stream=None,
+                             out=None):
+        """gathered_keys int64 [world, B (k+1), kk], gathered_vals float32
+        [world, B (k+1), 8] (topk > 0), draft_tokens [B, k] -> as greedy()."""
+        import torch
+        world = gathered_keys.shape[0]
+        B, k = draft_tokens.shape
+        dev = gathered_keys.device
+        if out is None:
+            al = torch.empty(B, dtype=torch.int32, device=dev)
+            ot = torch.empty(B, k + 1, dtype=torch.int32, device=dev)
+            ids = torch.empty(B, k + 1, max(topk, 1), dtype=torch.int32, device=dev) if topk else None
+            vals = torch.empty(B, k + 1, max(topk, 1), dtype=torch.float32, device=dev) if topk else None
+        else:
+            al, ot, ids, vals = (tuple(out) + (None, None))[:4]
+        _check(specdec_shard_greedy_combine(gathered_keys.contiguous(), gathered_vals, world,
+                                            draft_tokens if k > 0 else None, B, k, V, al, ot, topk, ids, vals,
+                                            stream), "shard_greedy_combine")
+        return (al, ot, ids, vals) if topk else (al, ot)
 
 
 def specdec_verify_greedy_static_scratch(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len, out_tokens,

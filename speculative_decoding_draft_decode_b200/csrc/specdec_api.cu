@@ -320,6 +320,25 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     return dispatch_stats(dtype, vec, S, s);
 }
 
+// Vocabulary-sharded greedy: this shard's streaming pass, then its row keys.
+template <class Tag, int VEC, int MODE>
+specdec_status launch_shard_rows(Pass1Params P, cudaStream_t stream) {
+    if (P.R > 0x7fffffff || P.cpr > 65535) return SPECDEC_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>(P.R), static_cast<unsigned>(P.cpr));
+    if (launch_pdl(verify_pass1_kernel<Tag, VEC, MODE>, grid, 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    const int64_t per = MODE == MODE_TOP8 ? NWARPS : kShardRowsArgmax;
+    const dim3 grid2(static_cast<unsigned>((P.R + per - 1) / per));
+    if (launch_pdl(verify_shard_rows_kernel<Tag, MODE>, grid2, 0, stream, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+template <int MODE>
+specdec_status dispatch_shard_rows(specdec_dtype dt, bool vec, Pass1Params P, cudaStream_t s) {
+    if (dt == SPECDEC_BF16)
+        return vec ? launch_shard_rows<BF16Tag, 8, MODE>(P, s) : launch_shard_rows<BF16Tag, 1, MODE>(P, s);
+    return vec ? launch_shard_rows<F32Tag, 4, MODE>(P, s) : launch_shard_rows<F32Tag, 1, MODE>(P, s);
+}
+
 // Host checks of a packed-layout call.
 bool ragged_args_ok(const int32_t* offsets, int B, int total, int max_k) {
     if (offsets == nullptr || total < 0 || max_k < 0 || max_k > SPECDEC_MAX_K) return false;
@@ -365,6 +384,75 @@ size_t specdec_workspace_size(specdec_mode mode, int B, int k_or_N, int V, specd
     const Layout a = make_layout(rows, rpr, B, V, vec_elems(dtype), slot_bytes(mode), rej);
     const Layout b = make_layout(rows, rpr, B, V, 1, slot_bytes(mode), rej);
     return a.total > b.total ? a.total : b.total;
+}
+
+size_t specdec_workspace_size_shard(int rows, int V_shard, int topk, specdec_dtype dtype) {
+    if (!dtype_ok(dtype) || rows < 0 || V_shard < 1 || V_shard > SPECDEC_MAX_V || topk < 0 || topk > SPECDEC_MAX_TOPK)
+        return 0;
+    const size_t slot = topk > 0 ? kTop8ChunkBytes : kArgmaxChunkBytes;
+    const Layout a = make_layout(rows, 1, 1, V_shard, vec_elems(dtype), slot, false);
+    const Layout b = make_layout(rows, 1, 1, V_shard, 1, slot, false);
+    return a.total > b.total ? a.total : b.total;
+}
+
+specdec_status specdec_shard_greedy_rows(const void* logits, specdec_dtype dtype, int64_t row_stride, int rows,
+                                         int V_shard, int vocab_offset, int topk, uint64_t* row_keys,
+                                         float* row_vals, void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (rows < 0 || V_shard < 1 || V_shard > SPECDEC_MAX_V || topk < 0 || topk > SPECDEC_MAX_TOPK)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (vocab_offset < 0 || static_cast<int64_t>(vocab_offset) + V_shard > SPECDEC_MAX_V) return SPECDEC_ERR_INVALID_ARG;
+    if (rows == 0) return SPECDEC_OK;
+    if (!rows_fit(rows, row_stride, V_shard)) return SPECDEC_ERR_INVALID_ARG;
+    if (logits == nullptr || row_keys == nullptr || (topk > 0 && row_vals == nullptr)) return SPECDEC_ERR_INVALID_ARG;
+    const bool vec = vector_path_ok(logits, row_stride, elem_size(dtype));
+    const int ve = vec ? vec_elems(dtype) : 1;
+    const Layout L = make_layout(rows, 1, 1, V_shard, ve, topk > 0 ? kTop8ChunkBytes : kArgmaxChunkBytes, false);
+    specdec_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != SPECDEC_OK) return st;
+    Pass1Params P;
+    fill_common(P, logits, row_stride, V_shard, L, rows, 1, 1, ws);
+    P.vocab_offset = vocab_offset;
+    P.shard_keys = row_keys;
+    P.shard_vals = row_vals;
+    P.topk = topk;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (topk > 0) return dispatch_shard_rows<MODE_TOP8>(dtype, vec, P, s);
+    return dispatch_shard_rows<MODE_ARGMAX>(dtype, vec, P, s);
+}
+
+specdec_status specdec_shard_greedy_combine(const uint64_t* gathered_keys, const float* gathered_vals, int world,
+                                            const int32_t* draft_tokens, int B, int k, int V, int32_t* accept_len,
+                                            int32_t* out_tokens, int topk, int32_t* topk_ids, float* topk_vals,
+                                            struct CUstream_st* stream) {
+    if (world < 1 || world > 32 || B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V < 1 ||
+        V > SPECDEC_MAX_V || topk < 0 || topk > SPECDEC_MAX_TOPK)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    if (gathered_keys == nullptr || accept_len == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (k > 0 && draft_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (topk > 0 && (gathered_vals == nullptr || topk_ids == nullptr || topk_vals == nullptr))
+        return SPECDEC_ERR_INVALID_ARG;
+    Pass1Params P;
+    memset(&P, 0, sizeof(P));
+    P.V = V;
+    P.R = static_cast<int64_t>(B) * (k + 1);
+    P.B = B;
+    P.k = k;
+    P.drafts = draft_tokens;
+    P.accept_len = accept_len;
+    P.out_tokens = out_tokens;
+    P.topk = topk;
+    P.topk_ids = topk_ids;
+    P.topk_vals = topk_vals;
+    P.gathered_keys = gathered_keys;
+    P.gathered_vals = gathered_vals;
+    P.world = world;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = topk > 0 ? launch_pdl(verify_shard_combine_kernel<MODE_TOP8>, dim3(static_cast<unsigned>(B)), 0, s, P)
+                             : launch_pdl(verify_shard_combine_kernel<MODE_ARGMAX>, dim3(static_cast<unsigned>(B)), 0, s, P);
+    if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 
 size_t specdec_workspace_size_ragged(specdec_mode mode, int B, int total_drafts, int V, specdec_dtype dtype) {

@@ -109,6 +109,13 @@ struct Pass1Params {
     float* p_draft_out;
     RejState* state;
     RowStat* row_stat;          // [rows] every row's (M, Z), or null
+    // vocabulary-sharded greedy
+    int vocab_offset;               // global index of this shard's column 0
+    uint64_t* shard_keys;           // [R, kk] out: this shard's row keys, global indices
+    float* shard_vals;              // [R, 8] out (top-8): the stored values of those keys
+    const uint64_t* gathered_keys;  // [world, R, kk] every shard's row keys
+    const float* gathered_vals;     // [world, R, 8] (top-8)
+    int world;
 };
 
 // Static shared memory of the pass-1 kernel.
@@ -1125,6 +1132,128 @@ __global__ void __launch_bounds__(32 * kTop8EpiWarps) verify_top8_epilogue_kerne
     }
     const int64_t c0 = b * P.R / P.B, c1 = (b + 1) * P.R / P.B;
     for (int64_t r = c0 + threadIdx.x; r < c1 && r < kThetaRows; r += nthreads) P.theta_row[r] = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// Vocabulary-sharded greedy verification (Arctic page, "Speculator
+// optimisation": the logits are sharded over the vocabulary as the scorer's
+// tensor parallelism leaves them; each shard takes its own TopK, the shards'
+// results are all-gathered, and the global TopK is taken from them).
+//
+// verify_shard_rows_kernel: after the streaming pass over this shard's
+// columns, every row's argmax key (argmax) or 8 best keys and their stored
+// values (top-8), with global indices.  An ordered key's low word is ~index,
+// so the key of index + offset is key - offset (indices stay below 2^24).
+// ---------------------------------------------------------------------------
+constexpr int kShardRowsArgmax = 32;  // rows per CTA (argmax); top-8: one row per warp
+
+__device__ __forceinline__ uint64_t globalize(uint64_t key, int offset) {
+    return key != 0ull ? key - static_cast<uint64_t>(offset) : 0ull;
+}
+
+template <class Tag, int MODE>
+__global__ void __launch_bounds__(NT) verify_shard_rows_kernel(const Pass1Params P) {
+    grid_dependency_wait();
+    grid_launch_dependents();
+    if constexpr (MODE == MODE_TOP8) {
+        __shared__ Top8EpiSmem sm;
+        const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+        const int64_t r = static_cast<int64_t>(blockIdx.x) * NWARPS + wp;
+        if (r >= P.R) return;  // warp-uniform; no CTA barrier below
+        row_top8_warp<Tag>(P, r, sm.surv[wp], sm.top[wp]);
+        if (lane < 8) {
+            const uint64_t key = sm.top[wp][lane];
+            float val = __uint_as_float(0x7fc00000u);
+            if (key != 0ull)
+                val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride +
+                                       key_index(key));
+            P.shard_keys[r * 8 + lane] = globalize(key, P.vocab_offset);
+            P.shard_vals[r * 8 + lane] = val;
+        }
+        if (lane == 0 && r < kThetaRows) P.theta_row[r] = 0u;
+    } else {
+        __shared__ Pass1Smem sm;
+        const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kShardRowsArgmax;
+        const int n = static_cast<int>(P.R - r0 < kShardRowsArgmax ? P.R - r0 : kShardRowsArgmax);
+        merge_argmax_rows<Tag>(P, r0, n, sm.rowkey);
+        if (static_cast<int>(threadIdx.x) < n) P.shard_keys[r0 + threadIdx.x] = globalize(sm.rowkey[threadIdx.x], P.vocab_offset);
+    }
+}
+
+// verify_shard_combine_kernel: one CTA per request over the gathered shard
+// results: each row's argmax (the largest shard key) or 8 best (warp top-8
+// of the world's 8 x world keys, the values carried from the owning shard),
+// then the accept scan.
+template <int MODE>
+__global__ void __launch_bounds__(NT) verify_shard_combine_kernel(const Pass1Params P) {
+    __shared__ Pass1Smem sm;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int64_t b = blockIdx.x;
+    const ReqGeom g = req_geom(P, b);
+    const int k = g.kb;
+    const int dr = static_cast<int>(threadIdx.x) < k ? P.drafts[g.d0 + threadIdx.x] : 0;
+    for (int t = wp; t <= k; t += NWARPS) {
+        const int64_t r = g.row0 + t;
+        if constexpr (MODE == MODE_TOP8) {
+            constexpr int kSlots = 8;  // candidates per lane: world <= 32 shards x 8 keys
+            uint64_t c[kSlots];
+            float cv[kSlots];
+#pragma unroll
+            for (int j = 0; j < kSlots; ++j) {
+                const int i = lane + 32 * j;  // candidate i = (shard i / 8, slot i % 8)
+                c[j] = 0ull;
+                cv[j] = 0.0f;
+                if (i < P.world * 8) {
+                    const int64_t at = (static_cast<int64_t>(i >> 3) * P.R + r) * 8 + (i & 7);
+                    c[j] = __ldcg(&P.gathered_keys[at]);
+                    cv[j] = __ldcg(&P.gathered_vals[at]);
+                }
+            }
+            uint64_t l[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) l[e] = 0ull;
+#pragma unroll
+            for (int j = 0; j < kSlots; ++j)
+                if (c[j] > l[7]) top8_insert(l, c[j]);
+            const uint64_t mine = warp_top8(l);
+            // the value of each winner, from the lane that holds it
+            float myval = __uint_as_float(0x7fc00000u);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint64_t w = __shfl_sync(FULL_MASK, mine, e);
+                float v = 0.0f;
+                bool has = false;
+#pragma unroll
+                for (int j = 0; j < kSlots; ++j)
+                    if (w != 0ull && c[j] == w) {
+                        v = cv[j];
+                        has = true;
+                    }
+                const unsigned who = __ballot_sync(FULL_MASK, has);
+                const float got = __shfl_sync(FULL_MASK, v, who ? __ffs(who) - 1 : 0);
+                if (lane == e && who) myval = got;
+            }
+            const uint64_t top0 = __shfl_sync(FULL_MASK, mine, 0);
+            if (lane == 0) sm.am[t] = key_index(top0);
+            if (lane < P.topk) {
+                P.topk_ids[r * P.topk + lane] = mine != 0ull ? key_index(mine) : -1;
+                P.topk_vals[r * P.topk + lane] = mine != 0ull ? myval : __uint_as_float(0x7fc00000u);
+            }
+        } else {
+            uint64_t best = 0ull;
+            for (int w = lane; w < P.world; w += 32) {
+                const uint64_t kx = __ldcg(&P.gathered_keys[static_cast<int64_t>(w) * P.R + r]);
+                best = kx > best ? kx : best;
+            }
+            best = warp_max_u64(best);
+            if (lane == 0) sm.am[t] = key_index(best);
+        }
+    }
+    if (static_cast<int>(threadIdx.x) < k) sm.drafts[threadIdx.x] = dr;
+    __syncthreads();
+    greedy_accept(P, b, g, sm.drafts, sm.am);
 }
 
 }  // namespace specdec

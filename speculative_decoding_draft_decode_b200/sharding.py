@@ -1,12 +1,18 @@
-"""Splitting one batch of verify requests over ranks (one process per GPU).
+"""Splitting verification over ranks (one process per GPU).
 
-Requests are independent, so a batch shards by request with no exchange on
-the data path: rank i verifies requests [start_i, stop_i) of the global batch
-and the per-request outputs are concatenated in rank order.  Greedy and tree
-results are identical to the unsharded call.  In rejection mode the Philox
-counter uses the request index *within the call*, so a sharded call draws
-other (equally valid) uniforms than an unsharded one unless every rank passes
-a distinct `offset`.
+By request: requests are independent, so a batch shards by request with no
+exchange on the data path: rank i verifies requests [start_i, stop_i) of the
+global batch and the per-request outputs are concatenated in rank order.
+Greedy and tree results are identical to the unsharded call.  In rejection
+mode the Philox counter uses the request index *within the call*, so a
+sharded call draws other (equally valid) uniforms than an unsharded one
+unless every rank passes a distinct `offset`.
+
+By vocabulary (Arctic page, "Speculator optimisation": with the scorer's
+tensor parallelism each GPU holds a slice of the vocabulary of every logit
+row; each takes its TopK, the results are all-gathered, and the global TopK
+is taken from them): greedy verification in three steps, one exchange of
+B (k+1) x 8 bytes per rank (x 8 keys and values with top-k).
 """
 from __future__ import annotations
 
@@ -44,3 +50,41 @@ def gather_requests(local, B: int, group=None):
         dist.all_gather(bufs, pad, group=group)
         out.append(torch.cat([b[: e - s] for b, (s, e) in zip(bufs, counts)], dim=0))
     return out
+
+
+def vocab_range(V: int, world: int, rank: int):
+    """[v0, v1) of the vocabulary columns rank `rank` of `world` holds (the
+    first V % world ranks take one extra column)."""
+    return request_range(V, world, rank)
+
+
+def gather_shard_rows(keys, vals=None, group=None):
+    """The exchange step of vocabulary-sharded greedy verification: every
+    rank's row keys (int64 [rows] or [rows, 8]) and top-k values (float32
+    [rows, 8]) all-gathered in rank order -> ([world, rows, kk], [world,
+    rows, 8] or None)."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    k2 = keys.reshape(keys.shape[0], -1).contiguous()
+    kb = [torch.empty_like(k2) for _ in range(world)]
+    dist.all_gather(kb, k2, group=group)
+    gk = torch.stack(kb)
+    gv = None
+    if vals is not None:
+        v2 = vals.contiguous()
+        vb = [torch.empty_like(v2) for _ in range(world)]
+        dist.all_gather(vb, v2, group=group)
+        gv = torch.stack(vb)
+    return gk, gv
+
+
+def sharded_verify_greedy(verifier, logits_shard, vocab_offset: int, V: int, draft_tokens, topk: int = 0,
+                          group=None):
+    """Greedy verification with the vocabulary sharded over the ranks of
+    `group`: this rank's row results (its CUDA kernels), the all-gather, and
+    the combine (its CUDA kernel).  Every rank returns the full results."""
+    res = verifier.shard_greedy_rows(logits_shard, vocab_offset, topk)
+    keys, vals = (res if topk else (res, None))
+    gk, gv = gather_shard_rows(keys, vals, group)
+    return verifier.shard_greedy_combine(gk, gv, draft_tokens, V, topk)

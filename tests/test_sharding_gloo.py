@@ -73,3 +73,59 @@ def test_sharded_verify_matches_unsharded_gloo():
     assert all(p.exitcode == 0 for p in procs)
     res = sorted(q.get(timeout=10) for _ in range(world))
     assert all(ok_g and ok_t for _, ok_g, ok_t in res), res
+
+
+def test_vocab_range_partitions():
+    from speculative_decoding_draft_decode_b200.sharding import vocab_range
+    for V in (1, 7, 128256, 151936):
+        for world in (1, 2, 3, 8):
+            got = [vocab_range(V, world, r) for r in range(world)]
+            assert got[0][0] == 0 and got[-1][1] == V
+            assert all(got[i][1] == got[i + 1][0] for i in range(world - 1))
+
+
+def _vocab_worker(rank, world, port, result_q):
+    """A rank of vocabulary-sharded greedy verification on CPU: its row keys
+    over its columns (the documented ordered-key format, computed here with
+    numpy in place of the rank's GPU), the gather of sharding.py, and the
+    combine -> must equal the oracle on the whole rows."""
+    import torch.distributed as dist
+    import gen
+    import oracle
+    from speculative_decoding_draft_decode_b200.sharding import gather_shard_rows, vocab_range
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        inp = gen.greedy_synthetic(seed=9, B=6, k=3, V=500, alpha=0.8)
+        v0, v1 = vocab_range(inp.V, world, rank)
+        x = inp.logits[:, :, v0:v1].reshape(-1, v1 - v0)
+
+        def key(val, idx):
+            u = np.float32(0.0 if val == 0 else val).view(np.uint32)
+            o = 0 if np.isnan(val) else (int(~u & 0xFFFFFFFF) if u & 0x80000000 else int(u | 0x80000000))
+            return (o << 32) | (~idx & 0xFFFFFFFF)
+
+        keys = np.array([max(key(x[r, j], v0 + j) for j in range(x.shape[1])) for r in range(x.shape[0])],
+                        dtype=np.uint64).view(np.int64)
+        gk, _ = gather_shard_rows(torch.from_numpy(keys))
+        g = gk.numpy().view(np.uint64)[:, :, 0]
+        best = g.max(axis=0)
+        am = (~(best & np.uint64(0xFFFFFFFF)) & np.uint64(0xFFFFFFFF)).astype(np.int64).reshape(inp.B, inp.k + 1)
+        ref = oracle.argmax_rows(inp.logits, inp.dtype)
+        result_q.put((rank, bool(np.array_equal(am, ref))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_vocab_sharded_gather_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_vocab_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(ok for _, ok in res), res
