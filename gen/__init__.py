@@ -465,6 +465,46 @@ def greedy_ragged_tiers(seed: int = 6, B: int = 64, tiers=(1, 3, 7), V: int = LL
     return r
 
 
+@dataclass
+class NgramInputs:
+    """Token histories for the n-gram proposer: tokens [B, Lmax] int32 with
+    request b's sequence in tokens[b, :lengths[b]]."""
+    name: str
+    tokens: np.ndarray
+    lengths: np.ndarray
+    B: int
+    n_min: int = 2
+    n_max: int = 5
+    k: int = 4
+
+
+def ngram_histories(seed: int = 7, B: int = 64, L: int = 4096, V: int = LLAMA3_VOCAB, repeat_frac: float = 0.5,
+                    n_min: int = 2, n_max: int = 5, k: int = 4) -> NgramInputs:
+    """Synthetic token histories shaped like the vLLM page's n-gram tasks
+    (section 3: copying a passage, continuing text that repeats its words,
+    random output): each sequence is uniform random tokens in which segments
+    copied from earlier in the same sequence make up about `repeat_frac` of
+    it; lengths vary from L/2 to L; prompt_lookup range 2..5, 4 drafts."""
+    rng = np.random.default_rng(seed)
+    tokens = np.full((B, L), -1, np.int32)
+    lengths = rng.integers(L // 2, L + 1, size=B).astype(np.int32)
+    for b in range(B):
+        n = int(lengths[b])
+        t = rng.integers(0, V, size=n).astype(np.int32)
+        pos = 64
+        while pos < n:
+            if rng.random() < repeat_frac:
+                seg = int(rng.integers(8, 128))
+                src = int(rng.integers(0, pos))
+                seg = min(seg, n - pos, pos - src)
+                t[pos:pos + seg] = t[src:src + seg]
+                pos += max(seg, 1)
+            else:
+                pos += int(rng.integers(8, 128))
+        tokens[b, :n] = t
+    return NgramInputs("ngram_histories", tokens, lengths, B, n_min, n_max, k)
+
+
 def algorithmic_bytes(inp) -> int:
     """Bytes one verify call must move: one read of every logit row the mode
     needs, the gathers, and the outputs (the rejection pass-2 row re-read is

@@ -38,7 +38,8 @@ def _bind(path):
     L.oracle_verify_rejection_parallel.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f64, u64, u64,
                                                    P, P, P, P, i32]
     L.oracle_draft_stats.argtypes = [P, i32, i64, P, i64, i32, i32, i32, f64, P, P]
-    for f in ("oracle_draft_stats", "oracle_philox4x32_10", "oracle_uniforms", "oracle_argmax_rows", "oracle_topk_rows",
+    L.oracle_ngram_propose.argtypes = [P, i64, P, i32, i32, i32, i32, P, P]
+    for f in ("oracle_ngram_propose", "oracle_draft_stats", "oracle_philox4x32_10", "oracle_uniforms", "oracle_argmax_rows", "oracle_topk_rows",
               "oracle_verify_greedy", "oracle_verify_tree", "oracle_verify_rejection",
               "oracle_verify_greedy_ragged", "oracle_verify_rejection_ragged", "oracle_verify_greedy_parallel",
               "oracle_verify_tree_parallel", "oracle_verify_rejection_parallel"):
@@ -251,3 +252,15 @@ def draft_stats(target, dtype, q, temperature):
     j = np.zeros((B, max(k, 1)), np.float64)
     lib().oracle_draft_stats(_ptr(x), DTYPE_CODE[dtype], V, _ptr(qq), V, B, k, V, float(temperature), _ptr(e), _ptr(j))
     return e[:, :k], j[:, :k]
+
+
+def ngram_propose(tokens, lengths, n_min, n_max, k):
+    """tokens [B, Lmax] int32, lengths [B] -> (drafts [B, k] -1 padded,
+    num_drafts [B]) of the n-gram (prompt-lookup) proposer."""
+    t = _c(tokens, np.int32)
+    B, Lmax = t.shape
+    ln = _c(lengths, np.int32)
+    d = np.zeros((B, max(k, 1)), np.int32)
+    n = np.zeros(B, np.int32)
+    lib().oracle_ngram_propose(_ptr(t), Lmax, _ptr(ln), B, n_min, n_max, k, _ptr(d), _ptr(n))
+    return d[:, :k], n

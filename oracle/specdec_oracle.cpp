@@ -561,6 +561,42 @@ void oracle_draft_stats(const void* target, int dtype, int64_t row_stride, const
     }
 }
 
+// N-gram (prompt-lookup) proposer ([HANDBOOK] "N-gram speculation": take a
+// suffix of the current sequence, e.g. its last two, three or four tokens;
+// search the prompt and the text generated so far for an earlier occurrence
+// of it; copy the tokens that follow that occurrence as the drafts; [VLLM]
+// section 2: prompt_lookup_min / prompt_lookup_max bound the suffix length,
+// num_speculative_tokens the drafts).  Reading: the longest suffix length n in
+// [n_min, n_max] that has an earlier occurrence wins, and among its
+// occurrences the most recent one (the largest start j with j + n < L, so at
+// least one token follows it); the drafts are the up to k tokens from j + n,
+// stopping at the end of the sequence.  No occurrence: no drafts.
+//   tokens [B, token_stride] int32, request b's sequence in tokens[b, 0..len[b])
+//   drafts [B, k] out, -1 padded; num_drafts [B] out
+void oracle_ngram_propose(const int32_t* tokens, int64_t token_stride, const int32_t* lengths, int B, int n_min,
+                          int n_max, int k, int32_t* drafts, int32_t* num_drafts) {
+    for (int b = 0; b < B; ++b) {
+        const int32_t* t = tokens + (int64_t)b * token_stride;
+        const int L = lengths[b];
+        int32_t* out = drafts + (int64_t)b * k;
+        for (int i = 0; i < k; ++i) out[i] = -1;
+        num_drafts[b] = 0;
+        bool done = false;
+        for (int n = n_max; n >= n_min && !done; --n) {
+            if (n < 1 || n >= L) continue;  // needs a suffix and an earlier place for it
+            for (int j = L - n - 1; j >= 0 && !done; --j) {  // most recent first
+                bool same = true;
+                for (int x = 0; x < n && same; ++x) same = t[j + x] == t[L - n + x];
+                if (!same) continue;
+                int c = 0;
+                for (int p = j + n; p < L && c < k; ++p) out[c++] = t[p];
+                num_drafts[b] = c;
+                done = true;
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Request-parallel drivers, for timing the oracle on all host cores.  The
 // requests of a call are independent, so `threads` std::threads each run the

@@ -19,6 +19,7 @@ from oracle import build as oracle_build
 
 import test_oracle_pins as pins
 import test_oracle_adasd as adasd
+import test_oracle_ngram as ngram
 
 TORCH_PHILOX_MAIN = r"""
 #include <ATen/core/PhiloxRNGEngine.h>
@@ -106,6 +107,14 @@ MUTANTS = [
      "ok[c] = ok[par[c]] && t >= 0 && t < V && t == am[par[c]];",
      "ok[c] = ok[par[c]] && t >= 0 && t < V && t == am[c];",
      [pins.test_tree_brute_force_small, pins.test_tree_chain_reduces_to_greedy]),
+    ("n-gram: shortest suffix tried first",
+     "for (int n = n_max; n >= n_min && !done; --n) {",
+     "for (int n = n_min; n <= n_max && !done; ++n) {",
+     [lambda: ngram.test_matches_literal_steps(0), ngram.test_known_answers]),
+    ("n-gram: oldest occurrence instead of the most recent",
+     "for (int j = L - n - 1; j >= 0 && !done; --j) {  // most recent first",
+     "for (int j = 0; j <= L - n - 1 && !done; ++j) {  // most recent first",
+     [lambda: ngram.test_matches_literal_steps(0), ngram.test_known_answers]),
     ("AdaSD: Jensen-Shannon mixture not halved",
      "const double m = 0.5 * (px + qx);",
      "const double m = (px + qx);",
