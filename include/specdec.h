@@ -323,6 +323,26 @@ specdec_status specdec_shard_greedy_combine(const uint64_t* gathered_keys, const
                                             int32_t* out_tokens, int topk, int32_t* topk_ids, float* topk_vals,
                                             struct CUstream_st* stream);
 
+/* N-gram (prompt-lookup) proposer on the GPU (handbook page, "N-gram
+ * speculation": take a suffix of the current sequence, search the prompt and
+ * the text generated so far for an earlier occurrence, copy the tokens that
+ * follow it as drafts; vLLM page, section 2: prompt_lookup_min /
+ * prompt_lookup_max and num_speculative_tokens).  The longest suffix length n
+ * in [n_min, n_max] with an earlier occurrence wins, then its most recent
+ * occurrence (start j with j + n < L); the drafts are the up to k tokens from
+ * j + n, stopping at the sequence end; no occurrence gives no drafts.
+ *   tokens        [B, token_stride] int32, device: request b's sequence in
+ *                 tokens[b, 0..lengths[b]) (lengths clamped to [0, stride])
+ *   1 <= n_min <= n_max <= 16, 0 <= k <= SPECDEC_MAX_K
+ *   drafts        [B, k] int32 out, -1 padded; num_drafts [B] int32 out
+ *   draft_offsets [B + 1] int32 out and packed_drafts [B k] int32 out, both
+ *                 or neither: the counts scanned into CSR offsets and the
+ *                 drafts packed in that order, ready for the packed-layout
+ *                 verifiers.  No workspace. */
+specdec_status specdec_ngram_propose(const int32_t* tokens, int64_t token_stride, const int32_t* lengths, int B,
+                                     int n_min, int n_max, int k, int32_t* drafts, int32_t* num_drafts,
+                                     int32_t* draft_offsets, int32_t* packed_drafts, struct CUstream_st* stream);
+
 /* Greedy verification without a caller workspace.  The pages have no
  * counterpart: this entry point exists for callers that cannot allocate
  * device memory (plug-ins and engine hooks handed only input and output

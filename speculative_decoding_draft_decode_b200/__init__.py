@@ -109,6 +109,8 @@ def lib():
         L.specdec_shard_greedy_rows.restype = i32
         L.specdec_shard_greedy_combine.argtypes = [P, P, i32, P, i32, i32, i32, P, P, i32, P, P, P]
         L.specdec_shard_greedy_combine.restype = i32
+        L.specdec_ngram_propose.argtypes = [P, i64, P, i32, i32, i32, i32, P, P, P, P, P]
+        L.specdec_ngram_propose.restype = i32
         L.specdec_tier_update.argtypes = [P, ctypes.c_double, ctypes.c_double]
         L.specdec_tier_update.restype = ctypes.c_double
         L.specdec_tier_select.argtypes = [P, i32, ctypes.c_double]
@@ -235,6 +237,33 @@ def specdec_shard_greedy_combine(gathered_keys, gathered_vals, world, draft_toke
     return lib().specdec_shard_greedy_combine(_ptr(gathered_keys), _ptr(gathered_vals), world, _ptr(draft_tokens),
                                               B, k, V, _ptr(accept_len), _ptr(out_tokens), topk, _ptr(topk_ids),
                                               _ptr(topk_vals), _stream(stream))
+
+
+def specdec_ngram_propose(tokens, token_stride, lengths, B, n_min, n_max, k, drafts, num_drafts, draft_offsets,
+                          packed_drafts, stream=None) -> int:
+    return lib().specdec_ngram_propose(_ptr(tokens), token_stride, _ptr(lengths), B, n_min, n_max, k, _ptr(drafts),
+                                       _ptr(num_drafts), _ptr(draft_offsets), _ptr(packed_drafts), _stream(stream))
+
+
+def ngram_propose(tokens, lengths, n_min: int = 2, n_max: int = 5, k: int = 4, pack: bool = True, stream=None):
+    """tokens int32 [B, Lmax] (device), lengths int32 [B] -> (drafts [B, k],
+    num_drafts [B][, draft_offsets [B+1], packed_drafts [B k]]) of the GPU
+    n-gram proposer."""
+    import torch
+    if tokens.dtype != torch.int32 or tokens.dim() != 2 or tokens.stride(1) != 1:
+        raise ValueError("tokens must be an int32 [B, Lmax] tensor with a contiguous last dimension")
+    if lengths.dtype != torch.int32 or not lengths.is_contiguous():
+        raise ValueError("lengths must be a contiguous int32 [B] tensor")
+    B, Lmax = tokens.shape
+    dev = tokens.device
+    d = torch.empty(B, max(k, 1), dtype=torch.int32, device=dev)
+    n = torch.empty(B, dtype=torch.int32, device=dev)
+    off = torch.empty(B + 1, dtype=torch.int32, device=dev) if pack else None
+    packed = torch.empty(max(B * k, 1), dtype=torch.int32, device=dev) if pack else None
+    stride = int(tokens.stride(0)) if B > 1 else max(int(Lmax), 1)
+    _check(specdec_ngram_propose(tokens, stride, lengths, B, n_min, n_max, k, d, n, off, packed, stream),
+           "ngram_propose")
+    return (d[:, :k], n, off, packed) if pack else (d[:, :k], n)
 
 
 class specdec_tier_state(ctypes.Structure):

@@ -19,6 +19,7 @@
 #include "verify_pass1.cuh"
 #include "verify_resample.cuh"
 #include "verify_stats.cuh"
+#include "verify_ngram.cuh"
 
 namespace specdec {
 namespace {
@@ -585,6 +586,35 @@ specdec_status specdec_verify_rejection_ragged(const void* target_logits, specde
     return rejection_impl(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens, draft_offsets,
                           total_drafts, B, max_k, V, temperature, seed, offset, accept_len, out_tokens, p_draft_out,
                           counters, nullptr, nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+specdec_status specdec_ngram_propose(const int32_t* tokens, int64_t token_stride, const int32_t* lengths, int B,
+                                     int n_min, int n_max, int k, int32_t* drafts, int32_t* num_drafts,
+                                     int32_t* draft_offsets, int32_t* packed_drafts, struct CUstream_st* stream) {
+    if (B < 0 || B > SPECDEC_MAX_B || n_min < 1 || n_max < n_min || n_max > kNgramMax || k < 0 ||
+        k > SPECDEC_MAX_K || token_stride < 1 || token_stride > (int64_t(1) << 31) - 1)
+        return SPECDEC_ERR_INVALID_ARG;
+    if ((draft_offsets == nullptr) != (packed_drafts == nullptr)) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    if (tokens == nullptr || lengths == nullptr || num_drafts == nullptr || (k > 0 && drafts == nullptr))
+        return SPECDEC_ERR_INVALID_ARG;
+    NgramParams P;
+    P.tokens = tokens;
+    P.stride = token_stride;
+    P.lengths = lengths;
+    P.B = B;
+    P.n_min = n_min;
+    P.n_max = n_max;
+    P.k = k;
+    P.drafts = drafts;
+    P.num_drafts = num_drafts;
+    P.offsets = draft_offsets;
+    P.packed = packed_drafts;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (launch_pdl(verify_ngram_kernel, dim3(static_cast<unsigned>(B)), 0, s, P) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    if (draft_offsets != nullptr && launch_pdl(verify_ngram_pack_kernel, dim3(1), 0, s, P) != cudaSuccess)
+        return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 
 double specdec_tier_update(specdec_tier_state* state, double accepted, double decay) {
