@@ -323,6 +323,7 @@ def run_ours(args):
     n_sets = max(2, math.ceil(4 * l2 / set_bytes) + 1) if args.sets is None else args.sets
     sets = DeviceSets(inp, n_sets, device).sets
     ver = sd.Verifier(device)
+    sd.specdec_set_prefetch_inputs(args.prefetch_inputs)
     calls, outs, kpl = setup_calls(inp, sets, ver, device)
 
     stream = torch.cuda.Stream(device)
@@ -417,7 +418,8 @@ def run_ours(args):
         "config": dict(workload=args.workload, **describe(inp), requests_per_s=inp.B * world / (ms_step / 1e3),
                        l2="rotating %d input sets, %.0f MB > 4x L2 (%d MB)" % (n_sets, n_sets * set_bytes / 1e6,
                                                                              l2 // 2**20),
-                       launch="CUDA graph of %d C-ABI calls, replayed" % per_replay,
+                       launch="CUDA graph of %d C-ABI calls, replayed%s" % (
+                           per_replay, "; prefetch_inputs on" if args.prefetch_inputs else ""),
                        parallelism="dp%d (requests per rank, no collective)" % world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
@@ -575,6 +577,9 @@ def main():
                     choices=["greedy_llama3", "greedy_tiny", "rejection_qwen", "greedy_large_batch", "tree_medusa",
                              "greedy_ragged_tiers", "rejection_qwen_adasd"])
     ap.add_argument("--sets", type=int, default=None, help="input sets in the rotation (default: > 4x L2)")
+    ap.add_argument("--prefetch-inputs", action="store_true",
+                    help="opt in to the argmax pass loading its rows before the previous kernel ends "
+                         "(safe here: the inputs are written by torch before the timed region)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
     ap.add_argument("--clock-probe-seconds", type=float, default=1.0,

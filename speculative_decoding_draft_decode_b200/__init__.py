@@ -111,6 +111,8 @@ def lib():
         L.specdec_shard_greedy_combine.restype = i32
         L.specdec_ngram_propose.argtypes = [P, i64, P, i32, i32, i32, i32, P, P, P, P, P]
         L.specdec_ngram_propose.restype = i32
+        L.specdec_set_prefetch_inputs.argtypes = [i32]
+        L.specdec_set_prefetch_inputs.restype = i32
         L.specdec_tier_update.argtypes = [P, ctypes.c_double, ctypes.c_double]
         L.specdec_tier_update.restype = ctypes.c_double
         L.specdec_tier_select.argtypes = [P, i32, ctypes.c_double]
@@ -264,6 +266,13 @@ def ngram_propose(tokens, lengths, n_min: int = 2, n_max: int = 5, k: int = 4, p
     _check(specdec_ngram_propose(tokens, stride, lengths, B, n_min, n_max, k, d, n, off, packed, stream),
            "ngram_propose")
     return (d[:, :k], n, off, packed) if pack else (d[:, :k], n)
+
+
+def specdec_set_prefetch_inputs(enable: bool) -> bool:
+    """Process-wide: let the argmax streaming pass read its logit rows before
+    the previous kernel of the stream has finished (see the header for when
+    that is safe).  Returns the previous setting."""
+    return bool(lib().specdec_set_prefetch_inputs(1 if enable else 0))
 
 
 class specdec_tier_state(ctypes.Structure):

@@ -71,6 +71,10 @@ int vec_elems(specdec_dtype dt) { return dt == SPECDEC_BF16 ? 8 : 4; }
 
 constexpr int kMaxDevices = 64;
 
+// specdec_set_prefetch_inputs: whether the argmax streaming pass may read its
+// rows before the previous kernel of the stream has finished.
+std::atomic<int> g_prefetch_inputs{0};
+
 bool vector_path_ok(const void* p, int64_t stride, int esize) {
     return (reinterpret_cast<uintptr_t>(p) % 16 == 0) && ((stride * esize) % 16 == 0);
 }
@@ -186,6 +190,7 @@ specdec_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 void fill_common(Pass1Params& P, const void* logits, int64_t row_stride, int V, const Layout& L, int64_t rows,
                  int rows_per_req, int B, void* ws) {
     memset(&P, 0, sizeof(P));
+    P.prefetch_inputs = g_prefetch_inputs.load(std::memory_order_relaxed);
     char* base = static_cast<char*>(ws);
     P.logits = logits;
     P.row_stride = row_stride;
@@ -272,6 +277,7 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     P.q = draft_probs;
     P.q_stride = q_row_stride;
     P.invT = static_cast<float>(invT_d);
+    P.log2e_invT = static_cast<float>(invT_d * 1.4426950408889634);  // log2(e) / T, rounded once
     P.invT_d = invT_d;
     P.seed = seed;
     P.offset = offset;
@@ -293,6 +299,7 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     Q.B = B;
     Q.k = k;
     Q.invT = static_cast<float>(invT_d);
+    Q.log2e_invT = P.log2e_invT;
     Q.seed = seed;
     Q.offset = offset;
     Q.state = state;
@@ -616,6 +623,8 @@ specdec_status specdec_ngram_propose(const int32_t* tokens, int64_t token_stride
         return SPECDEC_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
+
+int specdec_set_prefetch_inputs(int enable) { return g_prefetch_inputs.exchange(enable ? 1 : 0); }
 
 double specdec_tier_update(specdec_tier_state* state, double accepted, double decay) {
     if (state == nullptr || !(decay >= 0.0 && decay < 1.0) || !(accepted >= 0.0 && accepted <= SPECDEC_MAX_K))

@@ -103,12 +103,14 @@ struct Pass1Params {
     const float* q;
     int64_t q_stride;
     float invT;
+    float log2e_invT;           // log2(e) / T, for exp2
     double invT_d;
     uint64_t seed;
     uint64_t offset;
     float* p_draft_out;
     RejState* state;
     RowStat* row_stat;          // [rows] every row's (M, Z), or null
+    int prefetch_inputs;            // the argmax pass may load rows before the previous kernel ends
     // vocabulary-sharded greedy
     int vocab_offset;               // global index of this shard's column 0
     uint64_t* shard_keys;           // [R, kk] out: this shard's row keys, global indices
@@ -443,6 +445,7 @@ struct Top8Reducer {
 template <class Tag, int VEC>
 struct SoftmaxReducer {
     float invT;
+    float log2e_invT;
     double invT_d;
     __device__ __forceinline__ void begin(int64_t, const Pass1Params&, Pass1Smem&) {}
     // Warp-collective: max over the warp's part of the chunk.
@@ -451,11 +454,14 @@ struct SoftmaxReducer {
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, o));
         return m;
     }
+    // exp((x - M) / T) as exp2((x - M) * log2(e) / T): log2e_invT is the
+    // product rounded once to fp32, a relative error of 2^-24 in an exponent
+    // whose size only matters where the term itself is small.
     __device__ __forceinline__ double vec_sum(const uint4& w, bool ok, float M) const {
         if (!ok) return 0.0;
         float s = 0.0f;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) s += expf((VecOps<Tag, VEC>::elem(w, e) - M) * invT);
+        for (int e = 0; e < VEC; ++e) s += exp2f((VecOps<Tag, VEC>::elem(w, e) - M) * log2e_invT);
         return static_cast<double>(s);
     }
     // Warp-collective: store (M, S) of the warp's part of the chunk.
@@ -967,6 +973,7 @@ __device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typena
                                               int sub, int cnt, Pass1Smem& sm) {
     SoftmaxReducer<Tag, VEC> red;
     red.invT = P.invT;
+    red.log2e_invT = P.log2e_invT;
     red.invT_d = P.invT_d;
     constexpr int KEEP = UPT <= 16 ? UPT : 16;  // vectors kept in registers per batch
     float m = -FLT_MAX;
@@ -1005,7 +1012,7 @@ __device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typena
             S += red.vec_sum(x, true, M);
         }
     }
-    if (has_tail) S += static_cast<double>(expf((tail - M) * P.invT));
+    if (has_tail) S += static_cast<double>(exp2f((tail - M) * P.log2e_invT));
     red.store(M, S, static_cast<uint64_t>(r) * P.cpr + sub, P);
 }
 
@@ -1025,7 +1032,14 @@ __global__ void __launch_bounds__(NT, kMinBlocks[MODE]) verify_pass1_kernel(cons
     constexpr int BATCH = UPT < kU ? UPT : kU;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
 
-    grid_dependency_wait();
+    // Ordering with the previous kernel of the stream: by default wait before
+    // touching memory.  With prefetch_inputs (a caller promise that the
+    // logits are not written by a kernel still running ahead of this one) the
+    // argmax pass issues its loads first and waits only before it writes its
+    // partials, which the previous verify call's epilogue may still be
+    // reading.
+    const bool early = MODE == MODE_ARGMAX && P.prefetch_inputs;
+    if (!early) grid_dependency_wait();
     grid_launch_dependents();
 
     // Chunk (row blockIdx.x, sub-chunk blockIdx.y): vectors [sub*CH, ...) of
@@ -1072,6 +1086,7 @@ __global__ void __launch_bounds__(NT, kMinBlocks[MODE]) verify_pass1_kernel(cons
             red.scalar(ok ? load_scalar<Tag>(row + x) : 0.0f, x, ok, sm);
         }
     }
+    if (early) grid_dependency_wait();
     red.end(r, sub, static_cast<uint64_t>(r) * P.cpr + sub, P, sm);
     }
 }

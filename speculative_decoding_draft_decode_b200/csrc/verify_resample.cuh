@@ -56,6 +56,7 @@ struct Pass2Params {
     int B;
     int k;
     float invT;
+    float log2e_invT;  // log2(e) / T
     uint64_t seed;
     uint64_t offset;
     const RejState* state;
@@ -93,14 +94,15 @@ struct ResidualVec {
         }
     }
 
-    // p = exp((l - M)/T) / Z and r = max(0, p - q) (r = p without q).
-    __device__ __forceinline__ void values(bool has_q, float M, float invT, float invZ, float (&p)[VEC],
+    // p = exp((l - M)/T) / Z = exp2((l - M) log2(e) / T) / Z and r = max(0,
+    // p - q) (r = p without q); l2 = log2(e) / T.
+    __device__ __forceinline__ void values(bool has_q, float M, float l2, float invZ, float (&p)[VEC],
                                            float (&r)[VEC]) const {
         float lv[VEC];
         RowLoader<Tag, VEC>::unpack(l, lv);
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-            p[e] = expf((lv[e] - M) * invT) * invZ;
+            p[e] = exp2f((lv[e] - M) * l2) * invZ;
             r[e] = has_q ? fmaxf(0.0f, p[e] - qv(e)) : p[e];
         }
     }
@@ -109,9 +111,9 @@ struct ResidualVec {
 // p and r of one element of the ragged row end.
 template <class Tag>
 __device__ __forceinline__ void residual_scalar(const typename Tag::storage* row, const float* qrow, int x,
-                                                bool has_q, float M, float invT, float invZ, float& p, float& r) {
+                                                bool has_q, float M, float l2, float invZ, float& p, float& r) {
     const float l = load_scalar<Tag>(row + x);
-    p = expf((l - M) * invT) * invZ;
+    p = exp2f((l - M) * l2) * invZ;
     r = has_q ? fmaxf(0.0f, p - __ldg(qrow + x)) : p;
 }
 
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P
             double ar = 0.0, ap = 0.0;
             if (stream_pos(u0 + u, t) < cnt) {
                 float p[VEC], r[VEC];
-                v[u].values(R.has_q, st.M, P.invT, R.invZ, p, r);
+                v[u].values(R.has_q, st.M, P.log2e_invT, R.invZ, p, r);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) {
                     ar += static_cast<double>(r[e]);
@@ -228,7 +230,7 @@ __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P
         double tr = 0.0, tp = 0.0;
         if (x < P.V) {
             float p, r;
-            residual_scalar<Tag>(row, R.qrow, x, R.has_q, st.M, P.invT, R.invZ, p, r);
+            residual_scalar<Tag>(row, R.qrow, x, R.has_q, st.M, P.log2e_invT, R.invZ, p, r);
             tr = static_cast<double>(r);
             tp = static_cast<double>(p);
         }
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
             nx = x0 < P.V ? 1 : 0;
             if (nx) {
                 float p, r;
-                residual_scalar<Tag>(row, R.qrow, x0, R.has_q, st.M, P.invT, R.invZ, p, r);
+                residual_scalar<Tag>(row, R.qrow, x0, R.has_q, st.M, P.log2e_invT, R.invZ, p, r);
                 m[0] = use_p ? p : r;
             }
         } else {
@@ -412,7 +414,7 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
                 ResidualVec<Tag, VEC> v;
                 v.load(row, R.qrow, j, R.has_q);
                 float p[VEC], r[VEC];
-                v.values(R.has_q, st.M, P.invT, R.invZ, p, r);
+                v.values(R.has_q, st.M, P.log2e_invT, R.invZ, p, r);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) m[e] = use_p ? p[e] : r[e];
             }

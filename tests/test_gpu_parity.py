@@ -469,3 +469,38 @@ def test_rejection_distribution_on_gpu(V_):
         obs = np.bincount(out[sel, j], minlength=V)
         exp = _softmax64(tgt1[j]) * sel.sum()
         assert chisquare(obs, exp).pvalue > 1e-4
+
+
+def test_prefetch_inputs_mode(V_):
+    """With the opt-in early loads of the argmax pass (inputs written by
+    torch, which does not trigger programmatic launch), results stay exact,
+    including back-to-back calls on rotating inputs in a replayed graph."""
+    import torch
+    prev = sd.specdec_set_prefetch_inputs(True)
+    try:
+        check_greedy(V_, gen.greedy_llama3())
+        check_tree(V_, gen.tree_medusa())
+        inp = gen.greedy_synthetic(seed=77, B=48, k=6, V=32000, alpha=0.8, sigma=2.0, dtype="bf16")
+        sets = [inp.logits, np.roll(inp.logits, 5, axis=-1), np.roll(inp.logits, 11, axis=-1)]
+        drafts = [inp.drafts, (inp.drafts + 5) % 32000, (inp.drafts + 11) % 32000]
+        xs = [dev_logits(x, "bf16") for x in sets]
+        ds = [dev_i32(d) for d in drafts]
+        outs = [(torch.empty(48, dtype=torch.int32, device="cuda"), torch.empty(48, 7, dtype=torch.int32, device="cuda"))
+                for _ in sets]
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            for x, d, o in zip(xs, ds, outs):
+                V_.greedy(x, d, out=o)
+        s.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for x, d, o in zip(xs, ds, outs):
+                V_.greedy(x, d, out=o)
+        for _ in range(5):
+            g.replay()
+        torch.cuda.synchronize()
+        for x, d, o in zip(sets, drafts, outs):
+            al, out = oracle.verify_greedy(x, "bf16", d)
+            assert np.array_equal(host(o[0]), al) and np.array_equal(host(o[1]), out)
+    finally:
+        sd.specdec_set_prefetch_inputs(prev)
