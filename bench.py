@@ -389,6 +389,37 @@ def run_ours(args):
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
     ms_max = float(ms_t.item())
 
+    # The same steps again with the opt-in early loads of the argmax pass
+    # (specdec_set_prefetch_inputs), reported beside the default: safe here,
+    # the inputs were written by torch before any timed region.
+    prefetch = None
+    argmax_path = (isinstance(inp, gen.TreeInputs) or (isinstance(inp, (gen.GreedyInputs, gen.RaggedInputs))
+                                                        and not inp.topk))
+    if argmax_path and not args.prefetch_inputs:
+        sd.specdec_set_prefetch_inputs(True)
+        graphs.clear()  # the setting is baked into captured kernels: capture again
+        graph_of(per_replay)
+        for n in (args.warmup, args.steps):
+            if n % per_replay:
+                graph_of(n % per_replay)
+        with torch.cuda.stream(stream):
+            run_steps(args.warmup)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            run_steps(args.steps)
+            ev1.record(stream)
+        torch.cuda.synchronize(device)
+        if world > 1:
+            dist.barrier()
+        pt = torch.tensor([ev0.elapsed_time(ev1)], dtype=torch.float64, device=device)
+        if world > 1:
+            dist.all_reduce(pt, op=dist.ReduceOp.MAX)
+        sd.specdec_set_prefetch_inputs(False)
+        prefetch = float(pt.item()) / args.steps
+
     # end to end: inputs from pinned host memory, H2D + verify + D2H each step
     e2e = run_e2e(inp, ver, device, stream, args.e2e_steps) if args.e2e_steps > 0 else None
     if world > 1 and e2e is not None:
@@ -430,6 +461,13 @@ def run_ours(args):
         "gpu_launches": args.steps * kpl,
         "clocks": clocks,
     }
+    if prefetch is not None:
+        pa = alg_bytes / (prefetch / 1e3) / 1e9
+        line["prefetch_inputs"] = {
+            "note": "same steps with specdec_set_prefetch_inputs(1): the argmax pass loads its rows before the "
+                    "previous kernel ends (opt-in; the library default is off and gives `value`)",
+            "ms_per_step": prefetch, "value": rows * world / (prefetch / 1e3), "achieved_gbs": pa,
+            "frac": pa / peak}
     if e2e is not None:
         line["e2e"] = {"value": rows * world / (e2e["ms_per_step"] / 1e3), "unit": "rows/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
