@@ -393,9 +393,7 @@ def run_ours(args):
     # (specdec_set_prefetch_inputs), reported beside the default: safe here,
     # the inputs were written by torch before any timed region.
     prefetch = None
-    argmax_path = (isinstance(inp, gen.TreeInputs) or (isinstance(inp, (gen.GreedyInputs, gen.RaggedInputs))
-                                                        and not inp.topk))
-    if argmax_path and not args.prefetch_inputs:
+    if not args.prefetch_inputs:
         sd.specdec_set_prefetch_inputs(True)
         graphs.clear()  # the setting is baked into captured kernels: capture again
         graph_of(per_replay)
@@ -464,7 +462,7 @@ def run_ours(args):
     if prefetch is not None:
         pa = alg_bytes / (prefetch / 1e3) / 1e9
         line["prefetch_inputs"] = {
-            "note": "same steps with specdec_set_prefetch_inputs(1): the argmax pass loads its rows before the "
+            "note": "same steps with specdec_set_prefetch_inputs(1): the streaming pass loads its rows before the "
                     "previous kernel ends (opt-in; the library default is off and gives `value`)",
             "ms_per_step": prefetch, "value": rows * world / (prefetch / 1e3), "achieved_gbs": pa,
             "frac": pa / peak}
@@ -616,7 +614,7 @@ def main():
                              "greedy_ragged_tiers", "rejection_qwen_adasd"])
     ap.add_argument("--sets", type=int, default=None, help="input sets in the rotation (default: > 4x L2)")
     ap.add_argument("--prefetch-inputs", action="store_true",
-                    help="opt in to the argmax pass loading its rows before the previous kernel ends "
+                    help="opt in to the streaming pass loading its rows before the previous kernel ends "
                          "(safe here: the inputs are written by torch before the timed region)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)

@@ -373,11 +373,10 @@ const char* specdec_status_string(specdec_status status);
 /* Launch ordering (process-wide; returns the previous setting; default 0).
  * Every kernel of the library is enqueued with programmatic stream
  * serialisation and waits for the previous kernel of the stream before it
- * touches memory.  With enable = 1 the argmax streaming pass (greedy without
- * top-k, tree, packed greedy, vocabulary-shard rows) issues the loads of its
- * logit rows first and waits only before it writes its partial results, so
- * its loads overlap the tail of the previous kernel (for back-to-back calls,
- * the previous call's request epilogue).  Enable it only when the kernel
+ * touches memory.  With enable = 1 the streaming pass of every mode issues
+ * the loads of its first logit rows and waits only before its first
+ * workspace access, so those loads overlap the tail of the previous kernel
+ * (for back-to-back calls, the previous call's last kernel).  Enable it only when the kernel
  * enqueued just before a verify call does not write that call's logits
  * while letting its dependents start early (a kernel that executes
  * griddepcontrol.launch_dependents before its last store of the logits);

@@ -269,9 +269,9 @@ def ngram_propose(tokens, lengths, n_min: int = 2, n_max: int = 5, k: int = 4, p
 
 
 def specdec_set_prefetch_inputs(enable: bool) -> bool:
-    """Process-wide: let the argmax streaming pass read its logit rows before
-    the previous kernel of the stream has finished (see the header for when
-    that is safe).  Returns the previous setting."""
+    """Process-wide: let the streaming pass read its logit rows before the
+    previous kernel of the stream has finished (see the header for when that
+    is safe).  Returns the previous setting."""
     return bool(lib().specdec_set_prefetch_inputs(1 if enable else 0))
 
 

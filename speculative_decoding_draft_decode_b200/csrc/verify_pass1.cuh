@@ -1013,6 +1013,7 @@ __device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typena
         }
     }
     if (has_tail) S += static_cast<double>(exp2f((tail - M) * P.log2e_invT));
+    if (P.prefetch_inputs) grid_dependency_wait();  // the pass began without waiting
     red.store(M, S, static_cast<uint64_t>(r) * P.cpr + sub, P);
 }
 
@@ -1035,10 +1036,12 @@ __global__ void __launch_bounds__(NT, kMinBlocks[MODE]) verify_pass1_kernel(cons
     // Ordering with the previous kernel of the stream: by default wait before
     // touching memory.  With prefetch_inputs (a caller promise that the
     // logits are not written by a kernel still running ahead of this one) the
-    // argmax pass issues its loads first and waits only before it writes its
-    // partials, which the previous verify call's epilogue may still be
-    // reading.
-    const bool early = MODE == MODE_ARGMAX && P.prefetch_inputs;
+    // pass issues its row loads first and waits just before its first
+    // workspace access (the previous verify call's epilogue may still be
+    // reading the partials or clearing the top-8 thresholds): argmax before
+    // writing its partials, top-8 before reading the row threshold, softmax
+    // before writing its partials.
+    const bool early = P.prefetch_inputs != 0;
     if (!early) grid_dependency_wait();
     grid_launch_dependents();
 
@@ -1063,7 +1066,10 @@ __global__ void __launch_bounds__(NT, kMinBlocks[MODE]) verify_pass1_kernel(cons
             w[u] = make_uint4(0u, 0u, 0u, 0u);
             if (i < cnt) RowLoader<Tag, VEC>::raw(row, sub * CH + i, w[u]);
         }
-        if (u0 == 0) red.begin(r, sub, P, sm);  // after the loads are in flight (top-8 reads the row threshold)
+        if (u0 == 0) {
+            if (early && MODE == MODE_TOP8) grid_dependency_wait();
+            red.begin(r, sub, P, sm);  // after the loads are in flight (top-8 reads the row threshold)
+        }
         if constexpr (MODE == MODE_TOP8) {
             if (u0 == 0 && red.seed) {
                 float lm = -INFINITY;
@@ -1086,7 +1092,7 @@ __global__ void __launch_bounds__(NT, kMinBlocks[MODE]) verify_pass1_kernel(cons
             red.scalar(ok ? load_scalar<Tag>(row + x) : 0.0f, x, ok, sm);
         }
     }
-    if (early) grid_dependency_wait();
+    if (early && MODE != MODE_TOP8) grid_dependency_wait();
     red.end(r, sub, static_cast<uint64_t>(r) * P.cpr + sub, P, sm);
     }
 }

@@ -480,6 +480,14 @@ def test_prefetch_inputs_mode(V_):
     try:
         check_greedy(V_, gen.greedy_llama3())
         check_tree(V_, gen.tree_medusa())
+        for seed in (1, 2, 3):  # top-8 back to back: each call waits before reading the row thresholds
+            check_greedy(V_, gen.greedy_synthetic(seed=seed, B=20, k=8, V=60000, alpha=0.7, sigma=2.0,
+                                                  dtype="bf16"), topk=8)
+        r = gen.rejection_qwen()
+        for off in range(3):
+            got = run_rejection(V_, r, offset=off)
+            exp = oracle.verify_rejection(r.target, r.dtype, r.q, r.drafts, r.temperature, r.seed, off)
+            compare_rejection(got, exp)
         inp = gen.greedy_synthetic(seed=77, B=48, k=6, V=32000, alpha=0.8, sigma=2.0, dtype="bf16")
         sets = [inp.logits, np.roll(inp.logits, 5, axis=-1), np.roll(inp.logits, 11, axis=-1)]
         drafts = [inp.drafts, (inp.drafts + 5) % 32000, (inp.drafts + 11) % 32000]
