@@ -36,13 +36,14 @@ struct Layout {
 
 // Layout of one call.  `vec` = elements per vector (1 on the scalar path),
 // `slot1` = bytes of pass-1 partials per chunk.
-Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t slot1, bool rejection) {
+Layout make_layout(int64_t rows, int rows_per_req, int B, int V, int vec, size_t slot1, bool rejection,
+                   int u = kU) {
     Layout L;
     L.total = kPartialBase;
     if (rows <= 0 || V <= 0) return L;  // nothing streamed: only the fixed area
     L.nv = (V + vec - 1) / vec;
     L.nv_full = V / vec;
-    L.cpr = chunks_per_row(L.nv_full, vec);
+    L.cpr = chunks_per_row(L.nv_full, vec, u);
     L.NC = rows * L.cpr;
     L.partials1 = kPartialBase;
     size_t end = L.partials1 + static_cast<size_t>(L.NC) * slot1;
@@ -225,7 +226,8 @@ specdec_status greedy_impl(const void* logits, specdec_dtype dtype, int64_t row_
     if (topk > 0 && (topk_ids == nullptr || topk_vals == nullptr)) return SPECDEC_ERR_INVALID_ARG;
     const bool vec = vector_path_ok(logits, row_stride, elem_size(dtype));
     const int ve = vec ? vec_elems(dtype) : 1;
-    const Layout L = make_layout(rows, k + 1, B, V, ve, topk > 0 ? kTop8ChunkBytes : kArgmaxChunkBytes, false);
+    const Layout L = make_layout(rows, k + 1, B, V, ve, topk > 0 ? kTop8ChunkBytes : kArgmaxChunkBytes, false,
+                                 mode_u(topk > 0 ? MODE_TOP8 : MODE_ARGMAX));
     specdec_status st = check_ws(ws, ws_bytes, L.total);
     if (st != SPECDEC_OK) return st;
     Pass1Params P;
@@ -415,7 +417,8 @@ specdec_status specdec_shard_greedy_rows(const void* logits, specdec_dtype dtype
     if (logits == nullptr || row_keys == nullptr || (topk > 0 && row_vals == nullptr)) return SPECDEC_ERR_INVALID_ARG;
     const bool vec = vector_path_ok(logits, row_stride, elem_size(dtype));
     const int ve = vec ? vec_elems(dtype) : 1;
-    const Layout L = make_layout(rows, 1, 1, V_shard, ve, topk > 0 ? kTop8ChunkBytes : kArgmaxChunkBytes, false);
+    const Layout L = make_layout(rows, 1, 1, V_shard, ve, topk > 0 ? kTop8ChunkBytes : kArgmaxChunkBytes, false,
+                                 mode_u(topk > 0 ? MODE_TOP8 : MODE_ARGMAX));
     specdec_status st = check_ws(ws, ws_bytes, L.total);
     if (st != SPECDEC_OK) return st;
     Pass1Params P;
