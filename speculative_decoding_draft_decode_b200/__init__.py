@@ -51,6 +51,7 @@ SPECDEC_MODE_REJECTION = 1
 SPECDEC_MODE_TREE = 2
 
 MAX_B = 65536
+MAX_V = 1 << 24
 MAX_K = 32
 MAX_TOPK = 8
 MAX_DEPTH = 32

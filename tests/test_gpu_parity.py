@@ -512,3 +512,33 @@ def test_prefetch_inputs_mode(V_):
             assert np.array_equal(host(o[0]), al) and np.array_equal(host(o[1]), out)
     finally:
         sd.specdec_set_prefetch_inputs(prev)
+
+
+def test_maximum_batch(V_):
+    """SPECDEC_MAX_B requests (131072 rows, past the 65536 rows that get a
+    shared top-8 threshold), greedy and top-8."""
+    B, k, V = sd.MAX_B, 1, 16
+    inp = gen.greedy_synthetic(seed=91, B=B, k=k, V=V, alpha=0.5)
+    check_greedy(V_, inp)
+    check_greedy(V_, inp, topk=8, sample_topk_rows=4000)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_maximum_vocabulary(V_, dtype):
+    """V = SPECDEC_MAX_V (2^24 entries per row), greedy, top-8 and rejection."""
+    V = sd.MAX_V
+    rng = np.random.default_rng(92)
+    x = rng.standard_normal((2, 2, V), dtype=np.float32) * np.float32(2.0)
+    x[0, 0, V - 3] = 20.0          # the winner near the end of the row
+    x[1, 1, 7] = 20.0
+    logits = gen.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    am = oracle.argmax_rows(logits.reshape(-1, V), dtype).reshape(2, 2)
+    drafts = am[:, :1].copy()
+    inp = gen.GreedyInputs("maxV", dtype, logits, drafts, 2, 1, V)
+    check_greedy(V_, inp, topk=8)
+    if dtype == "f32":
+        q = np.full((2, 1, V), 1.0 / V, np.float32)
+        r = gen.RejectionInputs("maxV", "f32", x, q, drafts, 2, 1, V, seed=5)
+        got = run_rejection(V_, r)
+        exp = oracle.verify_rejection(x, "f32", q, drafts, 1.0, 5, 0)
+        compare_rejection(got, exp)
