@@ -323,6 +323,53 @@ specdec_status specdec_shard_greedy_combine(const uint64_t* gathered_keys, const
                                             int32_t* out_tokens, int topk, int32_t* topk_ids, float* topk_vals,
                                             struct CUstream_st* stream);
 
+/* Vocabulary-sharded rejection sampling (the sharded layout above; the
+ * inverse CDF needs two more exchanges than greedy).  Per call, on every
+ * rank (its columns [vocab_offset, vocab_offset + V_shard) of the target rows
+ * and of q; draft tokens are global indices; one workspace of
+ * specdec_workspace_size_shard_rejection bytes, kept across the steps):
+ *   1. specdec_shard_rejection_rows   -> row_stats [B (k+1)] of
+ *      SPECDEC_SHARD_ROW_STAT_BYTES each: the row's max logit and sum of
+ *      exp((l - M)/T) over the shard, and the logit and q of the row's draft
+ *      token when the shard holds it;
+ *   2. all-gather of row_stats in rank order -> [world, B (k+1)];
+ *   3. specdec_shard_rejection_decide -> accept_len, out_tokens (every slot but
+ *      h), p_draft_out; the same h on every rank;
+ *   4. specdec_shard_rejection_masses -> masses [B, 2] float64: the shard's
+ *      residual and target mass of row h;
+ *   5. all-gather of masses -> [world, B, 2];
+ *   6. specdec_shard_rejection_sample -> shard_tokens [B]: the drawn token
+ *      (global index) where this shard's part of row h holds the crossing of
+ *      u_res * S, else -1;
+ *   7. all-gather of shard_tokens -> [world, B];
+ *   8. specdec_shard_rejection_finish -> slot h of out_tokens.
+ * Results are those of specdec_verify_rejection on the whole rows up to the
+ * rounding of the merged sums (the same tolerance as the unsharded path). */
+#define SPECDEC_SHARD_ROW_STAT_BYTES 32
+size_t specdec_workspace_size_shard_rejection(int B, int k, int V_shard, specdec_dtype dtype);
+specdec_status specdec_shard_rejection_rows(const void* target, specdec_dtype dtype, int64_t row_stride,
+                                            const float* draft_probs, int64_t q_row_stride,
+                                            const int32_t* draft_tokens, int B, int k, int V_shard, int vocab_offset,
+                                            float temperature, void* row_stats, void* ws, size_t ws_bytes,
+                                            struct CUstream_st* stream);
+specdec_status specdec_shard_rejection_decide(const void* gathered_row_stats, int world, const int32_t* draft_tokens,
+                                              int B, int k, int V, float temperature, uint64_t seed, uint64_t offset,
+                                              int32_t* accept_len, int32_t* out_tokens, float* p_draft_out,
+                                              void* ws, size_t ws_bytes, struct CUstream_st* stream);
+specdec_status specdec_shard_rejection_masses(const void* target, specdec_dtype dtype, int64_t row_stride,
+                                              const float* draft_probs, int64_t q_row_stride, int B, int k,
+                                              int V_shard, float temperature, double* masses, void* ws,
+                                              size_t ws_bytes, struct CUstream_st* stream);
+specdec_status specdec_shard_rejection_sample(const void* target, specdec_dtype dtype, int64_t row_stride,
+                                              const float* draft_probs, int64_t q_row_stride, int B, int k,
+                                              int V_shard, int vocab_offset, float temperature, uint64_t seed,
+                                              uint64_t offset, const double* gathered_masses, int world, int rank,
+                                              int32_t* shard_tokens, void* ws, size_t ws_bytes,
+                                              struct CUstream_st* stream);
+specdec_status specdec_shard_rejection_finish(const int32_t* gathered_tokens, int world, int B, int k,
+                                              int32_t* out_tokens, void* ws, size_t ws_bytes,
+                                              struct CUstream_st* stream);
+
 /* N-gram (prompt-lookup) proposer on the GPU (handbook page, "N-gram
  * speculation": take a suffix of the current sequence, search the prompt and
  * the text generated so far for an earlier occurrence, copy the tokens that

@@ -112,6 +112,17 @@ def lib():
         L.specdec_shard_greedy_combine.restype = i32
         L.specdec_ngram_propose.argtypes = [P, i64, P, i32, i32, i32, i32, P, P, P, P, P]
         L.specdec_ngram_propose.restype = i32
+        L.specdec_workspace_size_shard_rejection.argtypes = [i32, i32, i32, i32]
+        L.specdec_workspace_size_shard_rejection.restype = sz
+        L.specdec_shard_rejection_rows.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, i32, f32, P, P, sz, P]
+        L.specdec_shard_rejection_decide.argtypes = [P, i32, P, i32, i32, i32, f32, u64, u64, P, P, P, P, sz, P]
+        L.specdec_shard_rejection_masses.argtypes = [P, i32, i64, P, i64, i32, i32, i32, f32, P, P, sz, P]
+        L.specdec_shard_rejection_sample.argtypes = [P, i32, i64, P, i64, i32, i32, i32, i32, f32, u64, u64, P, i32,
+                                                     i32, P, P, sz, P]
+        L.specdec_shard_rejection_finish.argtypes = [P, i32, i32, i32, P, P, sz, P]
+        for f in ("specdec_shard_rejection_rows", "specdec_shard_rejection_decide", "specdec_shard_rejection_masses",
+                  "specdec_shard_rejection_sample", "specdec_shard_rejection_finish"):
+            getattr(L, f).restype = i32
         L.specdec_set_prefetch_inputs.argtypes = [i32]
         L.specdec_set_prefetch_inputs.restype = i32
         L.specdec_tier_update.argtypes = [P, ctypes.c_double, ctypes.c_double]
@@ -556,6 +567,82 @@ class Verifier:
                                             draft_tokens if k > 0 else None, B, k, V, al, ot, topk, ids, vals,
                                             stream), "shard_greedy_combine")
         return (al, ot, ids, vals) if topk else (al, ot)
+
+
+class ShardRejection:
+    """One rank's side of vocabulary-sharded rejection sampling (the eight
+    steps of the C-ABI; the three all-gathers are the caller's, e.g.
+    sharding.sharded_verify_rejection).  Holds the rank's workspace between
+    the steps of one call; one object per rank and stream."""
+
+    def __init__(self, verifier, target_shard, draft_probs_shard, draft_tokens, vocab_offset: int, V: int,
+                 temperature: float, seed: int, offset: int = 0):
+        import torch
+        self.ver = verifier
+        self.x = target_shard
+        self.q = draft_probs_shard
+        self.d = draft_tokens
+        self.v0 = vocab_offset
+        self.V = V
+        self.T = temperature
+        self.seed = seed
+        self.offset = offset
+        B, k1, Vs = target_shard.shape
+        self.B, self.k, self.Vs = B, k1 - 1, Vs
+        self.dt = _dtype_code(target_shard)
+        self.rs = _row_stride(target_shard, "target_shard")
+        self.qs = _row_stride(draft_probs_shard, "draft_probs_shard") if self.k > 0 else Vs
+        need = lib().specdec_workspace_size_shard_rejection(B, self.k, Vs, self.dt)
+        self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=target_shard.device)
+        _check(specdec_workspace_init(self.ws, need), "workspace_init")
+        self.wsb = need
+        self.dev = target_shard.device
+
+    def rows(self, stream=None):
+        import torch
+        st = torch.empty(self.B * (self.k + 1), 4, dtype=torch.int64, device=self.dev)  # 32 bytes per row
+        _check(lib().specdec_shard_rejection_rows(_ptr(self.x), self.dt, self.rs, _ptr(self.q), self.qs,
+                                                  _ptr(self.d), self.B, self.k, self.Vs, self.v0, float(self.T),
+                                                  _ptr(st), _ptr(self.ws), self.wsb, _stream(stream)),
+               "shard_rejection_rows")
+        return st
+
+    def decide(self, gathered_stats, world: int, stream=None):
+        import torch
+        al = torch.empty(self.B, dtype=torch.int32, device=self.dev)
+        ot = torch.empty(self.B, self.k + 1, dtype=torch.int32, device=self.dev)
+        pd = torch.empty(self.B, max(self.k, 1), dtype=torch.float32, device=self.dev)
+        _check(lib().specdec_shard_rejection_decide(_ptr(gathered_stats.contiguous()), world, _ptr(self.d), self.B,
+                                                    self.k, self.V, float(self.T), int(self.seed) & (2**64 - 1),
+                                                    int(self.offset) & (2**64 - 1), _ptr(al), _ptr(ot), _ptr(pd),
+                                                    _ptr(self.ws), self.wsb, _stream(stream)), "shard_rejection_decide")
+        self.out = (al, ot, pd)
+        return self.out
+
+    def masses(self, stream=None):
+        import torch
+        m = torch.empty(self.B, 2, dtype=torch.float64, device=self.dev)
+        _check(lib().specdec_shard_rejection_masses(_ptr(self.x), self.dt, self.rs, _ptr(self.q), self.qs, self.B,
+                                                    self.k, self.Vs, float(self.T), _ptr(m), _ptr(self.ws),
+                                                    self.wsb, _stream(stream)), "shard_rejection_masses")
+        return m
+
+    def sample(self, gathered_masses, world: int, rank: int, stream=None):
+        import torch
+        t = torch.empty(self.B, dtype=torch.int32, device=self.dev)
+        _check(lib().specdec_shard_rejection_sample(_ptr(self.x), self.dt, self.rs, _ptr(self.q), self.qs, self.B,
+                                                    self.k, self.Vs, self.v0, float(self.T),
+                                                    int(self.seed) & (2**64 - 1), int(self.offset) & (2**64 - 1),
+                                                    _ptr(gathered_masses.contiguous()), world, rank, _ptr(t),
+                                                    _ptr(self.ws), self.wsb, _stream(stream)), "shard_rejection_sample")
+        return t
+
+    def finish(self, gathered_tokens, world: int, stream=None):
+        _check(lib().specdec_shard_rejection_finish(_ptr(gathered_tokens.contiguous()), world, self.B, self.k,
+                                                    _ptr(self.out[1]), _ptr(self.ws), self.wsb, _stream(stream)),
+               "shard_rejection_finish")
+        al, ot, pd = self.out
+        return al, ot, pd[:, :self.k]
 
 
 def specdec_verify_greedy_static_scratch(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len, out_tokens,

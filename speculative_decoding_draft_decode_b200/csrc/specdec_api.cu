@@ -349,6 +349,24 @@ specdec_status dispatch_shard_rows(specdec_dtype dt, bool vec, Pass1Params P, cu
     return vec ? launch_shard_rows<F32Tag, 4, MODE>(P, s) : launch_shard_rows<F32Tag, 1, MODE>(P, s);
 }
 
+// Vocabulary-sharded rejection: the request state sits at a fixed place
+// (every step finds it without the others' arguments), then the streaming
+// partials, then the chunk and unit masses of this shard's part of row h.
+Layout shard_rej_layout(int B, int k, int V_shard, int vec) {
+    const int64_t rows = static_cast<int64_t>(B) * (k + 1);
+    Layout L = make_layout(rows, k + 1, B, V_shard, vec, kSoftmaxChunkBytes, true);
+    const size_t state = kPartialBase, state_end = align_up(state + static_cast<size_t>(B) * sizeof(RejState), 256);
+    const size_t shift = state_end - L.partials1;  // move everything from the partials on past the state
+    L.state = state;
+    L.partials1 += shift;
+    L.masses += shift;
+    L.units += shift;
+    L.row_stat += shift;
+    L.chunk_stats += shift;
+    L.total += shift;
+    return L;
+}
+
 // Host checks of a packed-layout call.
 bool ragged_args_ok(const int32_t* offsets, int B, int total, int max_k) {
     if (offsets == nullptr || total < 0 || max_k < 0 || max_k > SPECDEC_MAX_K) return false;
@@ -463,6 +481,228 @@ specdec_status specdec_shard_greedy_combine(const uint64_t* gathered_keys, const
     cudaError_t e = topk > 0 ? launch_pdl(verify_shard_combine_kernel<MODE_TOP8>, dim3(static_cast<unsigned>(B)), 0, s, P)
                              : launch_pdl(verify_shard_combine_kernel<MODE_ARGMAX>, dim3(static_cast<unsigned>(B)), 0, s, P);
     if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+size_t specdec_workspace_size_shard_rejection(int B, int k, int V_shard, specdec_dtype dtype) {
+    if (!dtype_ok(dtype) || B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V_shard < 1 ||
+        V_shard > SPECDEC_MAX_V)
+        return 0;
+    const Layout a = shard_rej_layout(B, k, V_shard, vec_elems(dtype));
+    const Layout b = shard_rej_layout(B, k, V_shard, 1);
+    return a.total > b.total ? a.total : b.total;
+}
+
+specdec_status specdec_shard_rejection_rows(const void* target, specdec_dtype dtype, int64_t row_stride,
+                                            const float* draft_probs, int64_t q_row_stride,
+                                            const int32_t* draft_tokens, int B, int k, int V_shard, int vocab_offset,
+                                            float temperature, void* row_stats, void* ws, size_t ws_bytes,
+                                            struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V_shard < 1 || V_shard > SPECDEC_MAX_V ||
+        vocab_offset < 0 || static_cast<int64_t>(vocab_offset) + V_shard > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    const int64_t rows = static_cast<int64_t>(B) * (k + 1);
+    if (!rows_fit(rows, row_stride, V_shard)) return SPECDEC_ERR_INVALID_ARG;
+    if (target == nullptr || row_stats == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (k > 0 && (draft_tokens == nullptr || draft_probs == nullptr ||
+                  !rows_fit(static_cast<int64_t>(B) * k, q_row_stride, V_shard)))
+        return SPECDEC_ERR_INVALID_ARG;
+    const bool vec = vector_path_ok(target, row_stride, elem_size(dtype)) &&
+                     (k == 0 || vector_path_ok(draft_probs, q_row_stride, 4));
+    const Layout L = shard_rej_layout(B, k, V_shard, vec ? vec_elems(dtype) : 1);
+    specdec_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != SPECDEC_OK) return st;
+    const double invT_d = 1.0 / static_cast<double>(temperature);
+    Pass1Params P;
+    fill_common(P, target, row_stride, V_shard, L, rows, k + 1, B, ws);
+    P.drafts = draft_tokens;
+    P.k = k;
+    P.q = draft_probs;
+    P.q_stride = q_row_stride;
+    P.invT = static_cast<float>(invT_d);
+    P.log2e_invT = static_cast<float>(invT_d * 1.4426950408889634);
+    P.invT_d = invT_d;
+    P.vocab_offset = vocab_offset;
+    P.shard_stats = static_cast<ShardRowStat*>(row_stats);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (P.R > 0x7fffffff || P.cpr > 65535) return SPECDEC_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>(P.R), static_cast<unsigned>(P.cpr));
+    const dim3 grid2(static_cast<unsigned>((P.R + NWARPS - 1) / NWARPS));
+    cudaError_t e;
+    if (dtype == SPECDEC_BF16) {
+        e = vec ? launch_pdl(verify_pass1_kernel<BF16Tag, 8, MODE_SOFTMAX>, grid, 0, s, P)
+                : launch_pdl(verify_pass1_kernel<BF16Tag, 1, MODE_SOFTMAX>, grid, 0, s, P);
+        if (e == cudaSuccess) e = launch_pdl(verify_shard_softmax_rows_kernel<BF16Tag>, grid2, 0, s, P);
+    } else {
+        e = vec ? launch_pdl(verify_pass1_kernel<F32Tag, 4, MODE_SOFTMAX>, grid, 0, s, P)
+                : launch_pdl(verify_pass1_kernel<F32Tag, 1, MODE_SOFTMAX>, grid, 0, s, P);
+        if (e == cudaSuccess) e = launch_pdl(verify_shard_softmax_rows_kernel<F32Tag>, grid2, 0, s, P);
+    }
+    if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+specdec_status specdec_shard_rejection_decide(const void* gathered_row_stats, int world, const int32_t* draft_tokens,
+                                              int B, int k, int V, float temperature, uint64_t seed, uint64_t offset,
+                                              int32_t* accept_len, int32_t* out_tokens, float* p_draft_out,
+                                              void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+    if (world < 1 || world > 32 || B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V < 1 ||
+        V > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    if (gathered_row_stats == nullptr || accept_len == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (k > 0 && draft_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    specdec_status st = check_ws(ws, ws_bytes, kPartialBase + static_cast<size_t>(B) * sizeof(RejState));
+    if (st != SPECDEC_OK) return st;
+    const double invT_d = 1.0 / static_cast<double>(temperature);
+    Pass1Params P;
+    memset(&P, 0, sizeof(P));
+    P.V = V;
+    P.R = static_cast<int64_t>(B) * (k + 1);
+    P.B = B;
+    P.k = k;
+    P.drafts = draft_tokens;
+    P.accept_len = accept_len;
+    P.out_tokens = out_tokens;
+    P.p_draft_out = p_draft_out;
+    P.invT_d = invT_d;
+    P.seed = seed;
+    P.offset = offset;
+    P.world = world;
+    P.gathered_stats = static_cast<const ShardRowStat*>(gathered_row_stats);
+    P.state = reinterpret_cast<RejState*>(static_cast<char*>(ws) + kPartialBase);
+    if (launch_pdl(verify_shard_decide_kernel, dim3(static_cast<unsigned>(B)), 0, reinterpret_cast<cudaStream_t>(stream),
+                   P) != cudaSuccess)
+        return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+namespace {
+// Pass-2 parameters of a shard-rejection step (masses or token search).
+Pass2Params shard_pass2_params(const void* target, int64_t row_stride, const float* q, int64_t q_stride, int B,
+                               int k, int V_shard, float temperature, uint64_t seed, uint64_t offset, const Layout& L,
+                               void* ws) {
+    Pass2Params Q;
+    memset(&Q, 0, sizeof(Q));
+    const double invT_d = 1.0 / static_cast<double>(temperature);
+    Q.logits = target;
+    Q.row_stride = row_stride;
+    Q.q = q;
+    Q.q_stride = q_stride;
+    Q.V = V_shard;
+    Q.nv_full = static_cast<int>(L.nv_full);
+    Q.cpr = static_cast<int>(L.cpr2);
+    Q.B = B;
+    Q.k = k;
+    Q.invT = static_cast<float>(invT_d);
+    Q.log2e_invT = static_cast<float>(invT_d * 1.4426950408889634);
+    Q.seed = seed;
+    Q.offset = offset;
+    Q.state = reinterpret_cast<RejState*>(static_cast<char*>(ws) + L.state);
+    Q.chunk_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.masses);
+    Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
+    return Q;
+}
+}  // namespace
+
+specdec_status specdec_shard_rejection_masses(const void* target, specdec_dtype dtype, int64_t row_stride,
+                                              const float* draft_probs, int64_t q_row_stride, int B, int k,
+                                              int V_shard, float temperature, double* masses, void* ws,
+                                              size_t ws_bytes, struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V_shard < 1 || V_shard > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    if (target == nullptr || masses == nullptr || (k > 0 && draft_probs == nullptr)) return SPECDEC_ERR_INVALID_ARG;
+    const bool vec = vector_path_ok(target, row_stride, elem_size(dtype)) &&
+                     (k == 0 || vector_path_ok(draft_probs, q_row_stride, 4));
+    const Layout L = shard_rej_layout(B, k, V_shard, vec ? vec_elems(dtype) : 1);
+    specdec_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != SPECDEC_OK) return st;
+    Pass2Params Q = shard_pass2_params(target, row_stride, draft_probs, q_row_stride, B, k, V_shard, temperature, 0,
+                                       0, L, ws);
+    Q.shard_mass_out = reinterpret_cast<double2*>(masses);
+    if (Q.cpr > 65535) return SPECDEC_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid(static_cast<unsigned>(B), static_cast<unsigned>(Q.cpr));
+    const dim3 grid2(static_cast<unsigned>((B + NWARPS - 1) / NWARPS));
+    cudaError_t e;
+    if (dtype == SPECDEC_BF16)
+        e = vec ? launch_pdl(verify_resample_kernel<BF16Tag, 8>, grid, 0, s, Q)
+                : launch_pdl(verify_resample_kernel<BF16Tag, 1>, grid, 0, s, Q);
+    else
+        e = vec ? launch_pdl(verify_resample_kernel<F32Tag, 4>, grid, 0, s, Q)
+                : launch_pdl(verify_resample_kernel<F32Tag, 1>, grid, 0, s, Q);
+    if (e == cudaSuccess)
+        e = launch_pdl(verify_shard_mass_totals_kernel, grid2, 0, s, Q);
+    if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+specdec_status specdec_shard_rejection_sample(const void* target, specdec_dtype dtype, int64_t row_stride,
+                                              const float* draft_probs, int64_t q_row_stride, int B, int k,
+                                              int V_shard, int vocab_offset, float temperature, uint64_t seed,
+                                              uint64_t offset, const double* gathered_masses, int world, int rank,
+                                              int32_t* shard_tokens, void* ws, size_t ws_bytes,
+                                              struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V_shard < 1 || V_shard > SPECDEC_MAX_V ||
+        world < 1 || world > 32 || rank < 0 || rank >= world || vocab_offset < 0 ||
+        static_cast<int64_t>(vocab_offset) + V_shard > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    if (target == nullptr || gathered_masses == nullptr || shard_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    const bool vec = vector_path_ok(target, row_stride, elem_size(dtype)) &&
+                     (k == 0 || vector_path_ok(draft_probs, q_row_stride, 4));
+    const Layout L = shard_rej_layout(B, k, V_shard, vec ? vec_elems(dtype) : 1);
+    specdec_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != SPECDEC_OK) return st;
+    Pass2Params Q = shard_pass2_params(target, row_stride, draft_probs, q_row_stride, B, k, V_shard, temperature,
+                                       seed, offset, L, ws);
+    Q.shard_totals = reinterpret_cast<const double2*>(gathered_masses);
+    Q.world = world;
+    Q.rank = rank;
+    Q.vocab_offset = vocab_offset;
+    Q.shard_token = shard_tokens;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid(static_cast<unsigned>((B + NWARPS - 1) / NWARPS));
+    cudaError_t e;
+    if (dtype == SPECDEC_BF16)
+        e = vec ? launch_pdl(verify_resample_epilogue_kernel<BF16Tag, 8>, grid, 0, s, Q)
+                : launch_pdl(verify_resample_epilogue_kernel<BF16Tag, 1>, grid, 0, s, Q);
+    else
+        e = vec ? launch_pdl(verify_resample_epilogue_kernel<F32Tag, 4>, grid, 0, s, Q)
+                : launch_pdl(verify_resample_epilogue_kernel<F32Tag, 1>, grid, 0, s, Q);
+    if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
+
+specdec_status specdec_shard_rejection_finish(const int32_t* gathered_tokens, int world, int B, int k,
+                                              int32_t* out_tokens, void* ws, size_t ws_bytes,
+                                              struct CUstream_st* stream) {
+    if (world < 1 || world > 32 || B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    if (gathered_tokens == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    specdec_status st = check_ws(ws, ws_bytes, kPartialBase + static_cast<size_t>(B) * sizeof(RejState));
+    if (st != SPECDEC_OK) return st;
+    Pass1Params P;
+    memset(&P, 0, sizeof(P));
+    P.B = B;
+    P.k = k;
+    P.out_tokens = out_tokens;
+    P.world = world;
+    P.gathered_tokens = gathered_tokens;
+    P.state = reinterpret_cast<RejState*>(static_cast<char*>(ws) + kPartialBase);
+    if (launch_pdl(verify_shard_finish_kernel, dim3(static_cast<unsigned>((B + NT - 1) / NT)), 0,
+                   reinterpret_cast<cudaStream_t>(stream), P) != cudaSuccess)
+        return SPECDEC_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
 }
 

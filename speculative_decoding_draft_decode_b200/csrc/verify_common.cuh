@@ -30,6 +30,19 @@ struct RowStat {
     double Z;
 };
 
+// Vocabulary-sharded rejection: one row's statistics over one shard's
+// columns, exchanged between the ranks: the max logit and sum exp((l - M)/T)
+// of the shard, and, when the shard holds the row's draft token, its logit
+// and q value.
+struct ShardRowStat {
+    float M;
+    float l_draft;
+    float q_draft;
+    int32_t owned;  // 1: this shard holds the draft token of the row
+    double S;
+    double pad;
+};
+
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialisation may start while the previous kernel of the stream finishes;
 // griddepcontrol.wait blocks until that kernel has completed and its memory

@@ -131,6 +131,10 @@ struct Pass1Params {
     const uint64_t* gathered_keys;  // [world, R, kk] every shard's row keys
     const float* gathered_vals;     // [world, R, 8] (top-8)
     int world;
+    // vocabulary-sharded rejection
+    ShardRowStat* shard_stats;               // [R] out: this shard's row statistics
+    const ShardRowStat* gathered_stats;      // [world, R] every shard's
+    const int32_t* gathered_tokens;          // [world, B] the drawn token from its owner, -1 elsewhere
 };
 
 // Static shared memory of the pass-1 kernel.
@@ -1288,6 +1292,170 @@ __global__ void __launch_bounds__(NT) verify_shard_combine_kernel(const Pass1Par
     if (static_cast<int>(threadIdx.x) < k) sm.drafts[threadIdx.x] = dr;
     __syncthreads();
     greedy_accept(P, b, g, sm.drafts, sm.am);
+}
+
+// ---------------------------------------------------------------------------
+// Vocabulary-sharded rejection sampling: three exchanges between the ranks.
+//   1. verify_shard_softmax_rows_kernel (after the softmax pass over this
+//      shard's columns): every row's (M, S) over the shard and, for the row's
+//      draft token if the shard holds it, its logit and q value.
+//   2. verify_shard_decide_kernel (every rank, on the gathered statistics):
+//      M = max M_r, Z = sum S_r exp((M_r - M)/T), p_i(d_i) from the owner's
+//      logit, the Philox accept test and h, as the unsharded epilogue; every
+//      rank reaches the same h.  Then each shard's (residual, target) mass of
+//      row h is exchanged, and the shard whose running mass crosses u_res * S
+//      draws the token (verify_resample_epilogue_kernel in shard mode).
+//   3. verify_shard_finish_kernel: the owner's token into its output slot.
+// ---------------------------------------------------------------------------
+template <class Tag>
+__global__ void __launch_bounds__(NT) verify_shard_softmax_rows_kernel(const Pass1Params P) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * NWARPS + wp;  // a warp per row
+    if (r >= P.R) return;  // warp-uniform
+    const int np = P.cpr * NWARPS;
+    const SoftmaxPartial* p = static_cast<const SoftmaxPartial*>(P.partials) + r * np;
+    MaxSum acc;
+    acc.M = -FLT_MAX;
+    acc.S = 0.0;
+    constexpr int kPB = 8;
+    for (int i0 = lane; i0 < np; i0 += 32 * kPB) {
+        MaxSum x[kPB];
+#pragma unroll
+        for (int j = 0; j < kPB; ++j) {
+            const int i = i0 + 32 * j;
+            x[j].M = i < np ? __ldcg(&p[i].M) : -FLT_MAX;
+            x[j].S = i < np ? __ldcg(&p[i].S) : 0.0;
+        }
+#pragma unroll
+        for (int j = 0; j < kPB; ++j) acc = maxsum_merge(acc, x[j], P.invT_d);
+    }
+    acc = warp_maxsum(acc, P.invT_d);
+    if (lane == 0) {
+        ShardRowStat st = {};
+        st.M = acc.M;
+        st.S = acc.S;
+        const int64_t b = r / (P.k + 1);
+        const int i = static_cast<int>(r % (P.k + 1));
+        if (i < P.k) {
+            const int d = P.drafts[b * P.k + i] - P.vocab_offset;  // the draft as a column of this shard
+            if (d >= 0 && d < P.V) {
+                st.owned = 1;
+                st.l_draft = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride + d);
+                st.q_draft = __ldg(P.q + (b * P.k + i) * P.q_stride + d);
+            }
+        }
+        P.shard_stats[r] = st;
+    }
+}
+
+// One CTA per request over the gathered statistics (P.V is the global
+// vocabulary size here).
+__global__ void __launch_bounds__(NT) verify_shard_decide_kernel(const Pass1Params P) {
+    __shared__ Pass1Smem sm;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int64_t b = blockIdx.x;
+    const int k = P.k;
+    for (int t = wp; t <= k; t += NWARPS) {
+        const int64_t r = b * (k + 1) + t;
+        MaxSum acc;
+        acc.M = -FLT_MAX;
+        acc.S = 0.0;
+        float ld = 0.0f, qd = 0.0f;
+        int owned = 0;
+        if (lane < P.world) {  // shard `lane`
+            const ShardRowStat s = P.gathered_stats[static_cast<int64_t>(lane) * P.R + r];
+            acc.M = s.M;
+            acc.S = s.S;
+            owned = s.owned;
+            ld = s.l_draft;
+            qd = s.q_draft;
+        }
+        acc = warp_maxsum(acc, P.invT_d);
+        const unsigned who = __ballot_sync(FULL_MASK, lane < P.world && owned);
+        const int src = who ? __ffs(who) - 1 : 0;
+        ld = __shfl_sync(FULL_MASK, ld, src);
+        qd = __shfl_sync(FULL_MASK, qd, src);
+        if (lane == 0) {
+            sm.rowM[t] = acc.M;
+            sm.rowZ[t] = acc.S;
+            if (t < k) {  // the draft's logit and q, or a marker that no shard holds it
+                sm.am[t] = who ? 1 : 0;
+                reinterpret_cast<float*>(sm.stage)[2 * t] = ld;
+                reinterpret_cast<float*>(sm.stage)[2 * t + 1] = qd;
+            }
+        }
+    }
+    __syncthreads();
+    int bad = 0;
+    for (int t = threadIdx.x; t <= k; t += NT) {
+        const double z = sm.rowZ[t];
+        if (!(z > 0.0 && z <= DBL_MAX)) bad = 1;
+    }
+    bad = __syncthreads_or(bad);
+    if (bad) {
+        for (int i = threadIdx.x; i <= k; i += NT) P.out_tokens[b * (k + 1) + i] = -1;
+        if (P.p_draft_out)
+            for (int i = threadIdx.x; i < k; i += NT) P.p_draft_out[b * k + i] = __uint_as_float(0x7fc00000u);
+        if (threadIdx.x == 0) {
+            P.accept_len[b] = -1;
+            RejState st = {};
+            P.state[b] = st;
+        }
+        return;
+    }
+    if (wp == 0) {
+        bool accept = false;
+        int d = -1;
+        if (lane < k) {
+            d = P.drafts[b * k + lane];
+            const bool in = d >= 0 && d < P.V && sm.am[lane];
+            double p = 0.0, q = 0.0;
+            if (in) {
+                const float ld = reinterpret_cast<const float*>(sm.stage)[2 * lane];
+                p = exp((static_cast<double>(ld) - static_cast<double>(sm.rowM[lane])) * P.invT_d) / sm.rowZ[lane];
+                q = static_cast<double>(reinterpret_cast<const float*>(sm.stage)[2 * lane + 1]);
+            }
+            if (P.p_draft_out) P.p_draft_out[b * k + lane] = static_cast<float>(p);
+            const double2 u = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(lane));
+            accept = in && (u.x * q < p);
+        }
+        const unsigned rej = __ballot_sync(FULL_MASK, lane < k && !accept);
+        const int h = rej ? __ffs(rej) - 1 : k;
+        if (lane < h) P.out_tokens[b * (k + 1) + lane] = d;
+        else if (lane > h && lane <= k) P.out_tokens[b * (k + 1) + lane] = -1;
+        if (k == 32 && lane == 0 && h < 32) P.out_tokens[b * (k + 1) + 32] = -1;
+        if (lane == 0) {
+            P.accept_len[b] = h;
+            RejState st = {};
+            st.h = h;
+            st.valid = 1;
+            st.M = sm.rowM[h];
+            st.Z = sm.rowZ[h];
+            st.row = b * (k + 1) + h;
+            st.qrow = h < k ? b * k + h : -1;
+            P.state[b] = st;
+        }
+    }
+}
+
+// The drawn token from the shard that holds it, into slot h of each request.
+__global__ void __launch_bounds__(NT) verify_shard_finish_kernel(const Pass1Params P) {
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * NT + threadIdx.x;
+    if (b >= P.B) return;
+    const RejState st = P.state[b];
+    if (!st.valid) return;
+    int token = -1;
+    for (int w = 0; w < P.world; ++w) {
+        const int t = __ldcg(&P.gathered_tokens[static_cast<int64_t>(w) * P.B + b]);
+        token = t > token ? t : token;
+    }
+    P.out_tokens[st.row] = token;
 }
 
 }  // namespace specdec

@@ -63,6 +63,13 @@ struct Pass2Params {
     double2* chunk_mass;  // [B, cpr] (residual mass, target mass) of row h
     double2* unit_mass;   // [B, cpr, units_per_chunk] likewise per unit
     int32_t* out_tokens;
+    // vocabulary-sharded rejection (shard_totals null: the whole row is here)
+    const double2* shard_totals;  // [world, B] every shard's (residual, target) mass of row h
+    int world;
+    int rank;
+    int vocab_offset;             // global index of this shard's column 0
+    int32_t* shard_token;         // [B] out: the drawn token (global index) if this shard holds it, else -1
+    double2* shard_mass_out;      // [B] out: this shard's (residual, target) mass of row h
 };
 
 // One vector of row h: the raw logits and the matching q words.
@@ -358,7 +365,10 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
     const int64_t b = static_cast<int64_t>(blockIdx.x) * NWARPS + (threadIdx.x >> 5);
     if (b >= P.B) return;  // warp-uniform
     const RejState st = P.state[b];
-    if (!st.valid) return;  // the statistics pass already wrote -1 everywhere
+    if (!st.valid) {  // the statistics pass already wrote -1 everywhere
+        if (P.shard_totals != nullptr && lane == 0) P.shard_token[b] = -1;
+        return;
+    }
     const int64_t out_at = st.row;  // the drawn token's slot is row h's
 
     // Totals of r and p over the chunk masses, then u_res * S.
@@ -374,17 +384,59 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
         tr += __shfl_xor_sync(FULL_MASK, tr, o);
         tp += __shfl_xor_sync(FULL_MASK, tp, o);
     }
-    const bool use_p = !(tr > 0.0);
-    const double S = use_p ? tp : tr;
-    const double2 uu = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(st.h));
-    const double target = uu.y * S;
+    bool found = true;
+    double start = 0.0;  // mass before this part of the row
+    bool use_p;
+    double target;
+    if (P.shard_totals == nullptr) {
+        use_p = !(tr > 0.0);
+        const double S = use_p ? tp : tr;
+        const double2 uu = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(st.h));
+        target = uu.y * S;
+    } else {
+        // Vocabulary shards in rank order are the row in index order: the
+        // shard whose running mass first exceeds u_res * S draws the token
+        // (the last shard with mass if rounding leaves none).
+        double2 m = make_double2(0.0, 0.0);
+        if (lane < P.world) m = __ldcg(&P.shard_totals[static_cast<int64_t>(lane) * P.B + b]);
+        double ar = m.x, ap = m.y;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ar += __shfl_xor_sync(FULL_MASK, ar, o);
+            ap += __shfl_xor_sync(FULL_MASK, ap, o);
+        }
+        use_p = !(ar > 0.0);
+        const double S = use_p ? ap : ar;
+        const double2 uu = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(st.h));
+        target = uu.y * S;
+        const double mine = use_p ? m.y : m.x;
+        double incl = mine;
+        // fixed order: the running sum over shards 0..lane
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double w = __shfl_up_sync(FULL_MASK, incl, o);
+            if (lane >= o) incl += w;
+        }
+        const double excl = incl - mine;
+        const unsigned cross = __ballot_sync(FULL_MASK, lane < P.world && mine > 0.0 && incl > target);
+        const unsigned pos = __ballot_sync(FULL_MASK, lane < P.world && mine > 0.0);
+        const int owner = cross ? __ffs(cross) - 1 : (pos ? 31 - __clz(pos) : P.world - 1);
+        found = cross != 0u;
+        start = __shfl_sync(FULL_MASK, excl, owner);
+        if (owner != P.rank) {
+            if (lane == 0) P.shard_token[b] = -1;
+            return;
+        }
+    }
 
     // 1. the chunk, 2. the unit within it, 3. the element within the unit.
-    bool found = true;
     double before = 0.0;
-    const int chunk = warp_find_level(cm, P.cpr, use_p, 0.0, target, found, before);
+    const int chunk = warp_find_level(cm, P.cpr, use_p, start, target, found, before);
     if (chunk < 0) {  // no mass anywhere (cannot happen for a valid row)
-        if (lane == 0) P.out_tokens[out_at] = P.V - 1;
+        if (lane == 0) {
+            if (P.shard_totals == nullptr) P.out_tokens[out_at] = P.V - 1;
+            else P.shard_token[b] = P.vocab_offset + P.V - 1;
+        }
         return;
     }
     const bool has_tail = chunk == P.cpr - 1 && P.nv_full * VEC < P.V;
@@ -449,7 +501,34 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
         }
         token = hit != INT_MAX ? hit : (last >= 0 ? last : P.V - 1);
     }
-    if (lane == 0) P.out_tokens[out_at] = token;
+    if (lane == 0) {
+        if (P.shard_totals == nullptr) P.out_tokens[out_at] = token;
+        else P.shard_token[b] = P.vocab_offset + token;
+    }
+}
+
+// Vocabulary-sharded rejection: this shard's total (residual, target) mass
+// of each request's row h, a warp per request over its chunk masses.
+__global__ void __launch_bounds__(NT) verify_shard_mass_totals_kernel(const Pass2Params P) {
+    const int lane = threadIdx.x & 31;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * NWARPS + (threadIdx.x >> 5);
+    if (b >= P.B) return;  // warp-uniform
+    double tr = 0.0, tp = 0.0;
+    if (P.state[b].valid) {
+        for (int c = lane; c < P.cpr; c += 32) {
+            const double2 x = __ldcg(&P.chunk_mass[b * P.cpr + c]);
+            tr += x.x;
+            tp += x.y;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tr += __shfl_xor_sync(FULL_MASK, tr, o);
+        tp += __shfl_xor_sync(FULL_MASK, tp, o);
+    }
+    if (lane == 0) P.shard_mass_out[b] = make_double2(tr, tp);
 }
 
 }  // namespace specdec

@@ -88,3 +88,29 @@ def sharded_verify_greedy(verifier, logits_shard, vocab_offset: int, V: int, dra
     keys, vals = (res if topk else (res, None))
     gk, gv = gather_shard_rows(keys, vals, group)
     return verifier.shard_greedy_combine(gk, gv, draft_tokens, V, topk)
+
+
+def _gather_stack(t, group=None):
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    bufs = [torch.empty_like(t) for _ in range(world)]
+    dist.all_gather(bufs, t.contiguous(), group=group)
+    return torch.stack(bufs)
+
+
+def sharded_verify_rejection(verifier, target_shard, draft_probs_shard, draft_tokens, vocab_offset: int, V: int,
+                             temperature: float, seed: int, offset: int = 0, group=None):
+    """Rejection-sampling verification with the vocabulary sharded over the
+    ranks of `group`: row statistics, all-gather, the accept decision (the
+    same on every rank), the shards' masses of row h, all-gather, the draw on
+    the shard holding the crossing, all-gather of the token.  Every rank
+    returns (accept_len, out_tokens, p_draft)."""
+    import torch.distributed as dist
+    import speculative_decoding_draft_decode_b200 as sd
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    sr = sd.ShardRejection(verifier, target_shard, draft_probs_shard, draft_tokens, vocab_offset, V, temperature,
+                           seed, offset)
+    sr.decide(_gather_stack(sr.rows(), group), world)
+    tokens = sr.sample(_gather_stack(sr.masses(), group), world, rank)
+    return sr.finish(_gather_stack(tokens, group), world)

@@ -77,3 +77,63 @@ def test_sharded_special_values(V_, dtype):
     for world in (2, 3, 7):
         check(V_, inp, world, 8)
         check(V_, inp, world, 0)
+
+
+def run_sharded_rejection(r, world):
+    """The eight steps on `world` emulated ranks (column slices, separate
+    workspaces), the all-gathers as stacks."""
+    import torch
+    import speculative_decoding_draft_decode_b200 as sd
+    x = dev_logits(r.target, r.dtype)
+    q = torch.from_numpy(np.ascontiguousarray(r.q, dtype=np.float32)).cuda()
+    d = dev_i32(r.drafts)
+    ranks = []
+    for w in range(world):
+        v0, v1 = vocab_range(r.V, world, w)
+        ranks.append(sd.ShardRejection(sd.Verifier(torch.device("cuda", 0)), x[:, :, v0:v1], q[:, :, v0:v1], d, v0,
+                                       r.V, r.temperature, r.seed, r.offset))
+    stats = torch.stack([s.rows() for s in ranks])
+    for s in ranks:
+        s.decide(stats, world)
+    masses = torch.stack([s.masses() for s in ranks])
+    tokens = torch.stack([s.sample(masses, world, w) for w, s in enumerate(ranks)])
+    outs = [[host(t) for t in s.finish(tokens, world)] for s in ranks]
+    for o in outs[1:]:  # every rank holds the same results (NaN p_draft of invalid requests included)
+        assert all(np.array_equal(a, b, equal_nan=a.dtype.kind == "f") for a, b in zip(o, outs[0]))
+    return outs[0]
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 8])
+def test_sharded_rejection_qwen(world):
+    require_cuda()
+    from test_gpu_parity import compare_rejection, EXEMPT_FRACTION
+    r = gen.rejection_qwen()
+    n, ex = 0, 0
+    for off in range(3):
+        r.offset = off
+        got = run_sharded_rejection(r, world)
+        exp = oracle.verify_rejection(r.target, r.dtype, r.q, r.drafts, r.temperature, r.seed, off)
+        a, b = compare_rejection(got, exp)
+        n, ex = n + a, ex + b
+    assert ex <= max(1, EXEMPT_FRACTION * n)
+
+
+def test_sharded_rejection_special_rows():
+    require_cuda()
+    from test_gpu_parity import compare_rejection
+    rng = np.random.default_rng(3)
+    B, k, V = 24, 4, 2003
+    tgt = (rng.standard_normal((B, k + 1, V)) * 1.5).astype(np.float32)
+    noisy = tgt[:, :k].astype(np.float64) + rng.standard_normal((B, k, V))
+    q = np.exp(noisy - noisy.max(-1, keepdims=True))
+    q = (q / q.sum(-1, keepdims=True)).astype(np.float32)
+    drafts = np.argmax(q, axis=-1).astype(np.int32)
+    drafts[1, 1] = V + 5                   # out of range: rejected
+    drafts[2, 0] = V - 1                   # the last column (last shard)
+    tgt[3, 2, 1500] = np.nan               # invalid request
+    tgt[4, :, :1200] = -np.inf             # whole shards of -inf
+    r = gen.RejectionInputs("special", "f32", tgt, q, drafts, B, k, V, temperature=0.8, seed=11, offset=4)
+    for world in (2, 5):
+        got = run_sharded_rejection(r, world)
+        exp = oracle.verify_rejection(tgt, "f32", q, drafts, 0.8, 11, 4)
+        compare_rejection(got, exp)
