@@ -1,9 +1,9 @@
-// verify_common.cuh — pieces shared by the two verify kernels: the state the
-// rejection pass hands to the resample pass, the programmatic-launch
-// controls, and the ordered-atomic helpers.
+// verify_common.cuh — pieces shared by the verify kernels: the state the
+// rejection pass hands to the resample pass, the row statistics kept or
+// exchanged for the draft statistics and the vocabulary-sharded path, and
+// the programmatic-launch controls.
 #pragma once
 
-#include <cuda/atomic>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -51,14 +51,6 @@ struct ShardRowStat {
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-}
-
-// Request counters: a release-acquire increment at device scope.  The
-// release publishes every write the CTA made before its preceding barrier;
-// the acquire lets the CTA that sees the final count read all of them.
-__device__ __forceinline__ unsigned ticket_add(unsigned* p) {
-    cuda::atomic_ref<unsigned, cuda::thread_scope_device> a(*p);
-    return a.fetch_add(1u, cuda::memory_order_acq_rel);
 }
 
 }  // namespace specdec

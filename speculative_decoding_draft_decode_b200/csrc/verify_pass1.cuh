@@ -1,17 +1,19 @@
 // verify_pass1.cuh — the streaming verify pass (greedy, top-8, tree, and the
-// rejection statistics).
+// rejection statistics) and the request epilogues that follow it.
 //
-// Work unit: a chunk of kChunk 16-byte vectors of ONE logit row (rows are cut
-// into cpr chunks; the last one is shorter and carries the ragged row end).
-// One CTA per chunk, on a (row, sub-chunk) grid scheduled sub-chunk-major
-// (all rows' first chunks, then all rows' second chunks, ...).  The grid is many times larger
-// than what the GPU keeps resident, so the hardware block scheduler hands
-// chunks to SMs as they free up and no SM waits for a slower one.  Every
-// thread issues all its loads of the chunk at once; each warp reduces its
-// part (argmax key, top-8 keys, or softmax max/sum) and stores one partial
-// per (chunk, warp).  The CTA then takes a ticket for its request; the CTA
-// that takes a request's last ticket merges that request's partials (one
-// warp per row) and runs the request epilogue:
+// Work unit: a chunk of 16-byte vectors of ONE logit row (rows are cut into
+// cpr chunks; the last one is shorter and carries the ragged row end).  One
+// CTA per chunk, on a (row, sub-chunk) grid scheduled sub-chunk-major (all
+// rows' first chunks, then all rows' second chunks, ...).  The grid is many
+// times larger than what the GPU keeps resident, so the hardware block
+// scheduler hands chunks to SMs as they free up and no SM waits for a slower
+// one.  Every thread issues its loads of the chunk at once; each warp reduces
+// its part (argmax key, top-8 keys, or softmax max/sum) and stores one
+// partial per (chunk, warp).
+//
+// The request epilogues run as a second kernel (one CTA per request,
+// launched with programmatic stream serialisation so it is resident before
+// the pass drains); each merges its rows' partials and runs:
 //
 //   greedy     accept-prefix scan and correction/bonus token (Arctic page,
 //              "Verifier optimisation"; handbook, "How does speculative
@@ -21,10 +23,10 @@
 //              path and bonus (handbook, "Medusa" and "EAGLE");
 //   rejection  p_i(d_i), Philox accept test, accepted length h (vLLM page,
 //              section 1: rejection sampling keeps the target distribution);
-//              the resample of row h is the second kernel.
+//              the resample of row h follows (verify_resample.cuh).
 //
-// No CTA ever waits for another: the last ticket holder does the merge and
-// resets what it used (its ticket, its rows' top-8 thresholds), so the next
+// No CTA waits for another; the only words that must be zero when a call
+// starts (the top-8 row thresholds) are cleared by the epilogue, so the next
 // call (or a graph replay) starts from zero.
 #pragma once
 
@@ -661,7 +663,7 @@ __device__ void row_top8_warp(const Pass1Params& P, int64_t r, uint64_t* surv, u
 }
 
 // ---------------------------------------------------------------------------
-// Request epilogues (every thread of the last-ticket CTA).
+// Request epilogues (every thread of the request's CTA).
 // ---------------------------------------------------------------------------
 // Where request b's rows, drafts and outputs are.  Fixed layout: k drafts
 // per request, rows b*(k+1) ...  Packed layout (variable speculation length,
