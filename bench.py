@@ -325,6 +325,10 @@ def run_ours(args):
     ver = sd.Verifier(device)
     sd.specdec_set_prefetch_inputs(args.prefetch_inputs)
     calls, outs, kpl = setup_calls(inp, sets, ver, device)
+    # The input sets and outputs were made on the default stream (the rolled
+    # sets by kernels still queued there, and the outputs may reuse blocks of
+    # its freed temporaries); the calls run on a stream of their own.
+    torch.cuda.synchronize(device)
 
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
@@ -487,6 +491,7 @@ def run_e2e(inp, ver, device, stream, steps):
     d = {k: torch.empty_like(v, device=device) for k, v in h.items()}
     calls, outs, _ = setup_calls(inp, [d], ver, device)
     res_h = [torch.empty_like(o, device="cpu").pin_memory() for o in outs[:2]]
+    stream.wait_stream(torch.cuda.current_stream(device))  # buffers made on the default stream
     h2d = sum(v.numel() * v.element_size() for v in h.values())
     d2h = sum(o.numel() * o.element_size() for o in res_h)
 

@@ -56,22 +56,29 @@ enum Pass1Mode { MODE_ARGMAX = 0, MODE_TOP8 = 1, MODE_TREE = 2, MODE_SOFTMAX = 3
 #define SPECDEC_MINB_ARGMAX 6
 #endif
 #ifndef SPECDEC_MINB_TOP8
-#define SPECDEC_MINB_TOP8 4
+#define SPECDEC_MINB_TOP8 6
 #endif
 #ifndef SPECDEC_MINB_SOFTMAX
 #define SPECDEC_MINB_SOFTMAX 5
 #endif
 constexpr int kMinBlocks[4] = {SPECDEC_MINB_ARGMAX, SPECDEC_MINB_TOP8, SPECDEC_MINB_ARGMAX, SPECDEC_MINB_SOFTMAX};
 
-// 16-byte vectors per thread per chunk, per mode (loaded kU at a time): the
-// top-8 pass takes chunks twice as large, spreading its per-chunk work (the
-// end-of-chunk merge, the threshold publication) over twice the elements and
-// publishing a tighter row threshold from the first chunk (2 % faster on the
-// B=256, k=8 Llama-3 top-8 batch than 8; 12 and 24 are no better).
+// 16-byte vectors per thread per chunk, per mode: the top-8 pass takes
+// chunks twice as large, spreading its per-chunk work (the end-of-chunk
+// merge, the threshold publication) over twice the elements and publishing a
+// tighter row threshold from the first chunk (2 % faster on the B=256, k=8
+// Llama-3 top-8 batch than 8; 12 and 24 are no better).  It loads them
+// kTop8Batch at a time: batches of 4 keep it within 40 registers, so 6 CTAs
+// are resident per SM as in the argmax pass (2-3 % faster on that batch than
+// batches of 8 at 4 CTAs per SM).
 #ifndef SPECDEC_TOP8_U
 #define SPECDEC_TOP8_U 16
 #endif
+#ifndef SPECDEC_TOP8_BATCH
+#define SPECDEC_TOP8_BATCH 4
+#endif
 constexpr int kUTop8 = SPECDEC_TOP8_U;
+constexpr int kTop8Batch = SPECDEC_TOP8_BATCH;
 __host__ __device__ constexpr int mode_u(int mode) { return mode == MODE_TOP8 ? kUTop8 : kU; }
 // Workspace sizes count chunks at kU per thread, an upper bound for every mode.
 static_assert(kUTop8 >= kU, "the top-8 chunks must not be smaller than the others");
@@ -1040,8 +1047,8 @@ __device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typena
 // Pass-1 kernel: one CTA per chunk.  The grid holds many more CTAs than the
 // GPU keeps resident, so the hardware block scheduler hands chunks to SMs as
 // they free up (faster SMs take more chunks) and no counter is shared.  Every
-// thread issues all its loads of the chunk at once (kU x 16 bytes in flight
-// per thread), then its warp reduces.
+// thread issues its loads a batch at a time (kU x 16 bytes in flight per
+// thread; kTop8Batch in the top-8 pass), then its warp reduces the batch.
 // ---------------------------------------------------------------------------
 template <class Tag, int VEC, int MODE>
 __global__ void __launch_bounds__(NT, kMinBlocks[MODE]) verify_pass1_kernel(const Pass1Params P) {
@@ -1049,7 +1056,8 @@ __global__ void __launch_bounds__(NT, kMinBlocks[MODE]) verify_pass1_kernel(cons
     using Elem = typename Tag::storage;
     constexpr int CH = chunk_vecs(VEC, mode_u(MODE));  // vectors per chunk
     constexpr int UPT = CH / NT;                       // vectors per thread
-    constexpr int BATCH = UPT < kU ? UPT : kU;
+    constexpr int kB = MODE == MODE_TOP8 ? kTop8Batch : kU;  // loads in flight per thread
+    constexpr int BATCH = UPT < kB ? UPT : kB;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
 
     // Ordering with the previous kernel of the stream: by default wait before

@@ -496,6 +496,7 @@ def test_prefetch_inputs_mode(V_):
         outs = [(torch.empty(48, dtype=torch.int32, device="cuda"), torch.empty(48, 7, dtype=torch.int32, device="cuda"))
                 for _ in sets]
         s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())  # inputs and outputs made on the default stream
         with torch.cuda.stream(s):
             for x, d, o in zip(xs, ds, outs):
                 V_.greedy(x, d, out=o)

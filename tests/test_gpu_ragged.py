@@ -114,6 +114,7 @@ def test_counters_accumulate_and_replay(V_):
     al = torch.empty(24, dtype=torch.int32, device="cuda")
     ot = torch.empty(24 + T, dtype=torch.int32, device="cuda")
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())  # inputs and outputs made on the default stream
     with torch.cuda.stream(s):
         V_.greedy_ragged(x, d, o, T, 7, counters=ctr, out=(al, ot))  # workspace sized before capture
     s.synchronize()
