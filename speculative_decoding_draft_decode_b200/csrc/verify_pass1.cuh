@@ -49,11 +49,12 @@ constexpr int kThetaRows = 65536;   // rows with a shared top-8 threshold
 enum Pass1Mode { MODE_ARGMAX = 0, MODE_TOP8 = 1, MODE_TREE = 2, MODE_SOFTMAX = 3 };
 
 // Resident CTAs per SM the streaming pass is compiled for (a register cap;
-// more resident CTAs keep more loads in flight), per mode: argmax, top-8,
-// tree (streams as argmax), softmax.  Measured on B200: argmax 6 (40
-// registers) beats 5 by 4 %, softmax 5 beats 4 by 2.5 %.
+// more resident warps hide more of the load latency), per mode: argmax,
+// top-8, tree (streams as argmax), softmax.  Measured on B200: argmax 8 (32
+// registers, loads in batches of 4) beats 6 (40 registers, batches of 8) by
+// 1-2 % and 6 beat 5 by 4 %; softmax 5 beats 4 by 2.5 %.
 #ifndef SPECDEC_MINB_ARGMAX
-#define SPECDEC_MINB_ARGMAX 6
+#define SPECDEC_MINB_ARGMAX 8
 #endif
 #ifndef SPECDEC_MINB_TOP8
 #define SPECDEC_MINB_TOP8 6
@@ -77,8 +78,13 @@ constexpr int kMinBlocks[4] = {SPECDEC_MINB_ARGMAX, SPECDEC_MINB_TOP8, SPECDEC_M
 #ifndef SPECDEC_TOP8_BATCH
 #define SPECDEC_TOP8_BATCH 4
 #endif
+// 16-byte loads in flight per thread in the argmax pass (chunks of kU).
+#ifndef SPECDEC_ARGMAX_BATCH
+#define SPECDEC_ARGMAX_BATCH 4
+#endif
 constexpr int kUTop8 = SPECDEC_TOP8_U;
 constexpr int kTop8Batch = SPECDEC_TOP8_BATCH;
+constexpr int kArgmaxBatch = SPECDEC_ARGMAX_BATCH;
 __host__ __device__ constexpr int mode_u(int mode) { return mode == MODE_TOP8 ? kUTop8 : kU; }
 // Workspace sizes count chunks at kU per thread, an upper bound for every mode.
 static_assert(kUTop8 >= kU, "the top-8 chunks must not be smaller than the others");
@@ -1047,8 +1053,8 @@ __device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typena
 // Pass-1 kernel: one CTA per chunk.  The grid holds many more CTAs than the
 // GPU keeps resident, so the hardware block scheduler hands chunks to SMs as
 // they free up (faster SMs take more chunks) and no counter is shared.  Every
-// thread issues its loads a batch at a time (kU x 16 bytes in flight per
-// thread; kTop8Batch in the top-8 pass), then its warp reduces the batch.
+// thread issues its loads a batch at a time (kArgmaxBatch or kTop8Batch
+// 16-byte loads in flight per thread), then its warp reduces the batch.
 // ---------------------------------------------------------------------------
 template <class Tag, int VEC, int MODE>
 __global__ void __launch_bounds__(NT, kMinBlocks[MODE]) verify_pass1_kernel(const Pass1Params P) {
@@ -1056,7 +1062,7 @@ __global__ void __launch_bounds__(NT, kMinBlocks[MODE]) verify_pass1_kernel(cons
     using Elem = typename Tag::storage;
     constexpr int CH = chunk_vecs(VEC, mode_u(MODE));  // vectors per chunk
     constexpr int UPT = CH / NT;                       // vectors per thread
-    constexpr int kB = MODE == MODE_TOP8 ? kTop8Batch : kU;  // loads in flight per thread
+    constexpr int kB = MODE == MODE_TOP8 ? kTop8Batch : kArgmaxBatch;  // loads in flight per thread
     constexpr int BATCH = UPT < kB ? UPT : kB;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
 
