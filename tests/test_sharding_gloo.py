@@ -1,8 +1,13 @@
-"""Request sharding across ranks: world-size-2 gloo process groups on the CPU.
+"""Sharding across ranks: gloo process groups on the CPU.
 
-Each rank verifies its slice of one global batch (here with the CPU oracle
-standing in for a rank's GPU) and the gathered outputs must equal the
-unsharded verification exactly, for greedy and tree mode."""
+By request: each rank verifies its slice of one global batch (here with the
+CPU oracle standing in for a rank's GPU) and the gathered outputs must equal
+the unsharded verification exactly, for greedy and tree mode.
+
+By vocabulary: each rank holds a column slice of every row; the exchanges of
+sharding.py (greedy: one all-gather of row keys; rejection: row statistics,
+masses of row h, the drawn token) must reproduce the unsharded result, with
+numpy standing in for a rank's kernels."""
 import os
 import socket
 
@@ -129,3 +134,104 @@ def test_vocab_sharded_gather_gloo():
     for p in procs:
         p.join(timeout=60)
     assert all(ok for _, ok in res), res
+
+
+def _rejection_worker(rank, world, port, result_q):
+    """A rank of vocabulary-sharded rejection verification on CPU, with numpy
+    in fp64 in place of the rank's kernels, through the three exchanges of
+    sharding.py: its row statistics (max and sum of exp of l/T over its
+    columns, and the draft's l/T and q where it holds the draft), the same
+    accept decision on every rank, its residual and target masses of row h,
+    the draw on the shard holding the crossing, and the token.  The result
+    must equal the oracle on the whole rows (up to decisions within 1e-6 of
+    a boundary)."""
+    import torch.distributed as dist
+    import gen
+    import oracle
+    from speculative_decoding_draft_decode_b200.sharding import _gather_stack, vocab_range
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        r = gen.rejection_qwen(seed=5, B=12, k=3, V=700, temperature=0.8)
+        B, k, V, T = r.B, r.k, r.V, r.temperature
+        v0, v1 = vocab_range(V, world, rank)
+        x = r.target.astype(np.float64)[:, :, v0:v1] / T
+        q = r.q.astype(np.float64)[:, :, v0:v1]
+        # exchange 1: per row (M, S, l_d/T, q_d, holds the draft)
+        st = np.zeros((B, k + 1, 5))
+        st[..., 0] = x.max(axis=-1)
+        st[..., 1] = np.exp(x - st[..., 0][..., None]).sum(axis=-1)
+        for b in range(B):
+            for i in range(k):
+                d = int(r.drafts[b, i])
+                if v0 <= d < v1:
+                    st[b, i, 2:] = (x[b, i, d - v0], q[b, i, d - v0], 1.0)
+        g = _gather_stack(torch.from_numpy(st)).numpy()  # [world, B, k+1, 5]
+        M = g[..., 0].max(axis=0)
+        Z = (g[..., 1] * np.exp(g[..., 0] - M)).sum(axis=0)
+        h = np.full(B, k)
+        for b in range(B):
+            for i in range(k):
+                own = np.nonzero(g[:, b, i, 4] > 0)[0]
+                if own.size == 0:  # the draft is outside the vocabulary
+                    h[b] = i
+                    break
+                ld, qd = g[own[0], b, i, 2], g[own[0], b, i, 3]
+                ua, _ = oracle.uniforms(r.seed, r.offset, b, i)
+                if not (ua * qd < np.exp(ld - M[b, i]) / Z[b, i]):
+                    h[b] = i
+                    break
+        # exchange 2: this shard's (residual, target) mass of row h
+        res = []
+        for b in range(B):
+            p = np.exp(x[b, h[b]] - M[b, h[b]]) / Z[b, h[b]]
+            rr = np.maximum(0.0, p - q[b, h[b]]) if h[b] < k else p
+            res.append((rr, p))
+        masses = np.array([(rr.sum(), p.sum()) for rr, p in res])
+        mg = _gather_stack(torch.from_numpy(masses)).numpy()  # [world, B, 2]
+        # the shard whose running mass first exceeds u_res * S draws
+        tok = np.full(B, -1, np.int64)
+        for b in range(B):
+            use_p = not (mg[:, b, 0].sum() > 0.0)
+            col = 1 if use_p else 0
+            _, ur = oracle.uniforms(r.seed, r.offset, b, int(h[b]))
+            target = ur * mg[:, b, col].sum()
+            run = np.cumsum(mg[:, b, col])
+            cross = np.nonzero((mg[:, b, col] > 0) & (run > target))[0]
+            owner = cross[0] if cross.size else np.nonzero(mg[:, b, col] > 0)[0][-1]
+            if owner != rank:
+                continue
+            start = run[owner] - mg[owner, b, col]
+            m = res[b][1] if use_p else res[b][0]
+            c = start + np.cumsum(m)
+            hit = np.nonzero((m > 0) & (c > target))[0]
+            tok[b] = v0 + (hit[0] if hit.size else np.nonzero(m > 0)[0][-1])
+        # exchange 3: the owner's token
+        tg = _gather_stack(torch.from_numpy(tok)).numpy().max(axis=0)
+        out = np.full((B, k + 1), -1, np.int32)
+        for b in range(B):
+            out[b, :h[b]] = r.drafts[b, :h[b]]
+            out[b, h[b]] = tg[b]
+        al, eo, _, margin = oracle.verify_rejection(r.target, r.dtype, r.q, r.drafts, T, r.seed, r.offset)
+        bad = [(b, int(h[b]), int(al[b])) for b in range(B)
+               if (h[b] != al[b] or not np.array_equal(out[b], eo[b])) and not margin[b] < 1e-6]
+        result_q.put((rank, bad, int((h < k).sum())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_vocab_sharded_rejection_exchanges_gloo(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rejection_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(p.exitcode == 0 for p in procs)
+    assert all(not bad for _, bad, _ in res), res
+    assert res[0][2] > 0, "some request must reject a draft, so the residual draw is exercised"
