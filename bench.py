@@ -254,10 +254,11 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
+    def __init__(self, index, log_dir=None):
+        import tempfile
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % index)
+        self.path = os.path.join(log_dir or tempfile.gettempdir(), "specdec_clocks_rank%d.csv" % index)
 
     def start(self):
         try:
@@ -366,7 +367,7 @@ def run_ours(args):
     stream.synchronize()
 
     # clocks: sample across a 1 s burst of the same steps and the timed region
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(local, args.clock_log_dir)
     sampler.start()
     t_probe = time.time()
     with torch.cuda.stream(stream):
@@ -614,6 +615,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--clock-log-dir", default=None,
+                    help="directory for the raw nvidia-smi clock samples (default: the system temp directory)")
     ap.add_argument("--workload", default="greedy_llama3",
                     choices=["greedy_llama3", "greedy_tiny", "rejection_qwen", "greedy_large_batch", "tree_medusa",
                              "greedy_ragged_tiers", "rejection_qwen_adasd"])
