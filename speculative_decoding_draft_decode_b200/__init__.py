@@ -137,10 +137,16 @@ def lib():
 # Argument marshalling
 # ---------------------------------------------------------------------------
 def _ptr(x):
+    """Device address of a tensor argument (an int is taken as a raw device
+    pointer).  Host tensors are refused before anything is launched: a kernel
+    given a host address would fault."""
     if x is None:
         return None
     if isinstance(x, int):
         return x
+    if not getattr(x, "is_cuda", False):
+        raise ValueError("verifier arrays must be CUDA device tensors, got one on %s"
+                         % getattr(x, "device", type(x).__name__))
     return x.data_ptr()
 
 
@@ -352,6 +358,18 @@ class Verifier:
         self._ws = None
         self._ws_bytes = 0
 
+    def _on_device(self, *tensors):
+        """Every tensor argument must live on this verifier's CUDA device (any
+        CUDA device when the verifier's has no index)."""
+        want = self.device
+        for t in tensors:
+            if t is None:
+                continue
+            dv = getattr(t, "device", None)
+            if dv is None or dv.type != "cuda" or (want.index is not None and dv.index != want.index):
+                raise ValueError("verifier arrays must be on %s, got one on %s"
+                                 % (want, dv if dv is not None else type(t).__name__))
+
     def workspace(self, nbytes: int, stream=None):
         import torch
         if nbytes > self._ws_bytes:
@@ -365,6 +383,7 @@ class Verifier:
         """logits [B, k+1, V] (bf16/f32), draft_tokens [B, k] int32 ->
         (accept_len [B], out_tokens [B, k+1][, topk_ids, topk_vals])."""
         import torch
+        self._on_device(logits, draft_tokens if logits.shape[1] > 1 else None, *(out or ()))
         B, k1, V = logits.shape
         k = k1 - 1
         dt = _dtype_code(logits)
@@ -390,6 +409,7 @@ class Verifier:
         """logits [B, N+1, V], parents/node_tokens [B, N+1] int32 ->
         (accept_len [B], accept_nodes [B, max_depth], out_tokens [B, max_depth+1])."""
         import torch
+        self._on_device(logits, parents, node_tokens, *(out or ()))
         B, n1, V = logits.shape
         dt = _dtype_code(logits)
         stride = _row_stride(logits, "logits")
@@ -416,6 +436,7 @@ class Verifier:
         with stats=True also (draft_entropy [B, k], js_distance [B, k]) float64
         (AdaSD's statistics; `out` then holds five tensors)."""
         import torch
+        self._on_device(target_logits, draft_probs if target_logits.shape[1] > 1 else None, draft_tokens if target_logits.shape[1] > 1 else None, *(out or ()))
         B, k1, V = target_logits.shape
         k = k1 - 1
         dt = _dtype_code(target_logits)
@@ -474,6 +495,7 @@ class Verifier:
         off[b] + b) -> (accept_len [B], out_tokens [B + T][, topk_ids,
         topk_vals]); `counters` (int64 [3 + max_k]) accumulates."""
         import torch
+        self._on_device(logits, draft_tokens if total_drafts > 0 else None, draft_offsets, counters, *(out or ()))
         B, rs = self._ragged_args(logits, draft_offsets, draft_tokens, total_drafts, max_k)
         R, V = logits.shape
         dt = _dtype_code(logits)
@@ -499,6 +521,7 @@ class Verifier:
         int32, draft_offsets [B+1] int32 -> (accept_len [B], out_tokens
         [B + T], p_draft [T])."""
         import torch
+        self._on_device(target_logits, draft_probs if total_drafts > 0 else None, draft_tokens if total_drafts > 0 else None, draft_offsets, counters, *(out or ()))
         B, rs = self._ragged_args(target_logits, draft_offsets, draft_tokens, total_drafts, max_k)
         R, V = target_logits.shape
         dt = _dtype_code(target_logits)
@@ -531,6 +554,7 @@ class Verifier:
         (topk == 0) or [B (k+1), 8] with row_vals float32 [B (k+1), 8]:
         ordered keys with global indices (bit patterns of uint64)."""
         import torch
+        self._on_device(logits_shard, *(out or ()))
         B, k1, Vs = logits_shard.shape
         rows = B * k1
         dt = _dtype_code(logits_shard)
@@ -553,6 +577,7 @@ class Verifier:
         """gathered_keys int64 [world, B (k+1), kk], gathered_vals float32
         [world, B (k+1), 8] (topk > 0), draft_tokens [B, k] -> as greedy()."""
         import torch
+        self._on_device(gathered_keys, gathered_vals, draft_tokens, *(out or ()))
         world = gathered_keys.shape[0]
         B, k = draft_tokens.shape
         dev = gathered_keys.device
@@ -578,6 +603,9 @@ class ShardRejection:
     def __init__(self, verifier, target_shard, draft_probs_shard, draft_tokens, vocab_offset: int, V: int,
                  temperature: float, seed: int, offset: int = 0):
         import torch
+        has_drafts = target_shard.shape[1] > 1
+        verifier._on_device(target_shard, draft_probs_shard if has_drafts else None,
+                            draft_tokens if has_drafts else None)
         self.ver = verifier
         self.x = target_shard
         self.q = draft_probs_shard

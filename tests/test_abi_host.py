@@ -139,3 +139,32 @@ def test_workspace_init_rejects_bad_pointer(L):
     assert sd.specdec_workspace_init(None, 100, 0) == sd.SPECDEC_ERR_WORKSPACE
     assert sd.specdec_workspace_init(FAKE + 8, 100, 0) == sd.SPECDEC_ERR_WORKSPACE
     assert sd.specdec_workspace_init(FAKE, 0, 0) == sd.SPECDEC_OK
+
+
+def test_host_tensors_are_refused_before_any_launch(L):
+    """A kernel handed a host address would fault: every entry of the binding
+    refuses host tensors (and tensors of another device) up front."""
+    import torch
+    x = torch.zeros(2, 3, 64, dtype=torch.float32)
+    d = torch.zeros(2, 2, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        sd._ptr(x)
+    ver = sd.Verifier(torch.device("cuda", 0))
+    with pytest.raises(ValueError):
+        ver.greedy(x, d)
+    with pytest.raises(ValueError):
+        ver.rejection(x, torch.zeros(2, 2, 64), d, 1.0, 1)
+    with pytest.raises(ValueError):
+        ver.tree(x, torch.zeros(2, 3, dtype=torch.int32), torch.zeros(2, 3, dtype=torch.int32), 4)
+    off = torch.tensor([0, 1, 2], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        ver.greedy_ragged(torch.zeros(4, 64), torch.zeros(2, dtype=torch.int32), off, 2, 2)
+    with pytest.raises(ValueError):
+        ver.shard_greedy_rows(x, 0)
+    with pytest.raises(ValueError):
+        sd.ShardRejection(ver, x, torch.zeros(2, 2, 64), d, 0, 128, 1.0, 1)
+    with pytest.raises(ValueError):
+        sd.ngram_propose(torch.zeros(2, 16, dtype=torch.int32), torch.tensor([16, 16], dtype=torch.int32))
+    with pytest.raises(ValueError):
+        sd.specdec_verify_greedy(x, sd.SPECDEC_F32, 64, d, 2, 2, 64, torch.zeros(2, dtype=torch.int32),
+                                 torch.zeros(2, 3, dtype=torch.int32), 0, None, None, 0, 0, None)
