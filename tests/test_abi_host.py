@@ -168,3 +168,17 @@ def test_host_tensors_are_refused_before_any_launch(L):
     with pytest.raises(ValueError):
         sd.specdec_verify_greedy(x, sd.SPECDEC_F32, 64, d, 2, 2, 64, torch.zeros(2, dtype=torch.int32),
                                  torch.zeros(2, 3, dtype=torch.int32), 0, None, None, 0, 0, None)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No CPU fallback: without the CUDA library every call raises."""
+    saved_lib, saved_path = sd._lib, sd.library_path
+    try:
+        sd._lib = None
+        sd.library_path = str(tmp_path / "libspecdec.so")
+        with pytest.raises(Exception, match="no CPU fallback"):
+            sd.lib()
+        with pytest.raises(Exception, match="no CPU fallback"):
+            sd.specdec_abi_version()
+    finally:
+        sd._lib, sd.library_path = saved_lib, saved_path
