@@ -127,6 +127,18 @@ MUTANTS = [
      "if (qx > 0.0) H -= qx * std::log(qx);",
      "if (px > 0.0) H -= px * std::log(px);",
      [lambda: adasd.test_matches_scipy(1.0), adasd.test_closed_forms]),
+    ("margin: sample distance not divided by S",
+     "mg = std::min(mg, std::min(t - prev, c - t) / S);",
+     "mg = std::min(mg, std::min(t - prev, c - t));",
+     [pins.test_rejection_margin_sample_distance_over_S]),
+    ("margin: accept test measured at the rejecting position only",
+     "mg = std::min(mg, qd > 0.0 ? std::fabs(ua - p / qd) : p);\n        if (!(ua * qd < p)) break;",
+     "if (!(ua * qd < p)) { mg = std::min(mg, qd > 0.0 ? std::fabs(ua - p / qd) : p); break; }",
+     [pins.test_rejection_margin_accept_distance, pins.test_rejection_margin_zero_q_draft]),
+    ("margin: residual mass S left out",
+     "        mg = std::min(mg, S);\n",
+     "",
+     [pins.test_rejection_margin_residual_mass]),
 ]
 
 

@@ -553,3 +553,104 @@ def test_rejection_invalid_rows():
     al, out, pd, _ = oracle.verify_rejection(t, "f32", q, np.array([[6, 7]], np.int32), 1.0, 0, 0)
     assert al[0] >= 0 and (out[0, : al[0] + 1] >= 5).all()
     assert abs(pd[0, 0] - 0.2) < 1e-15
+
+
+# ---------------------------------------------------------------------------
+# The rejection margin: how far a request's decisions sit from a boundary
+# (the accept test's uniform against p/q, the residual's total mass S, and
+# u_res * S against the edges of the chosen bin, over S).  It only decides
+# which rows the sampling tolerance exempts, so each case below fixes it by
+# construction: the rows are built so that one term equals a chosen delta
+# and every other term is at least ten times larger.
+# ---------------------------------------------------------------------------
+NEG = np.float32(-1e4)  # exp(-1e4 - m) is exactly 0 in fp64: probability 0
+DELTA = 1e-3
+
+
+def _seed_where(pred, positions):
+    """The first seed whose uniforms (request 0, offset 0) at `positions`
+    satisfy pred([(u_acc, u_res), ...])."""
+    for seed in range(1, 100000):
+        us = [oracle.uniforms(seed, 0, 0, i) for i in positions]
+        if pred(us):
+            return seed, us
+    raise AssertionError("no seed found")
+
+
+def _log_row(p):
+    """float32 logits whose softmax is p (entries 0 get probability 0)."""
+    p = np.asarray(p, np.float64)
+    return np.where(p > 0, np.log(np.where(p > 0, p, 1.0)), NEG).astype(np.float32)
+
+
+def test_rejection_margin_accept_distance():
+    """An accepted draft whose p/q sits DELTA above the accept uniform: the
+    margin is DELTA, though no position rejects."""
+    seed, ((ua0, _), (_, ur1)) = _seed_where(
+        lambda us: 0.1 < us[0][0] < 0.85 and min(us[1][1], 1 - us[1][1]) > 10 * DELTA, (0, 1))
+    a = 0.5 * (ua0 + DELTA)  # p_0(d) with q_0(d) = 1/2: p/q = ua0 + DELTA
+    target = np.stack([_log_row([a, 1 - a, 0, 0]), _log_row([1, 0, 0, 0])])[None]
+    q = np.array([[[0.5, 0.5, 0, 0]]], np.float32)
+    al, out, pd, mg = oracle.verify_rejection(target, "f32", q, np.array([[0]], np.int32), 1.0, seed, 0)
+    assert al[0] == 1 and out[0].tolist() == [0, 0]
+    assert abs(mg[0] - DELTA) < 1e-6, mg[0]
+
+
+def test_rejection_margin_sample_distance_over_S():
+    """A rejection whose residual has total mass S = 1/2 and whose chosen bin
+    starts DELTA * S below u_res * S: the margin is DELTA (the distance
+    divided by S), not DELTA * S."""
+    seed, ((ua0, ur0),) = _seed_where(
+        lambda us: us[0][0] > 0.5 + 10 * DELTA and 10 * DELTA < us[0][1] < 1 - 10 * DELTA, (0,))
+    p0 = [0.5, 0.5 * (ur0 - DELTA), 0.5 * (1 - ur0 + DELTA), 0]
+    # q one-hot on the draft: p/q = 1/2 <= ua0 rejects; r = max(0, p - q) = p on tokens 1..3, S = 1/2
+    target = np.stack([_log_row(p0), _log_row([1, 0, 0, 0])])[None]
+    q = np.array([[[1, 0, 0, 0]]], np.float32)
+    al, out, pd, mg = oracle.verify_rejection(target, "f32", q, np.array([[0]], np.int32), 1.0, seed, 0)
+    assert al[0] == 0 and out[0].tolist() == [2, -1]
+    assert abs(mg[0] - DELTA) < 1e-6, mg[0]
+
+
+def test_rejection_margin_residual_mass():
+    """A rejection whose residual max(0, p - q) holds only eps of mass: the
+    margin is eps (a residual this small is a near-tie between resampling
+    from it and falling back to p)."""
+    seed, ((ua0, ur0),) = _seed_where(lambda us: us[0][0] > 0.01 and 0.01 < us[0][1] < 0.99, (0,))
+    qrow = np.array([1e-4, 1 - 1e-4, 0, 0], np.float32)
+    eps = 1.0 - float(qrow[1])  # S = 1 - q(1): p is one-hot on token 1
+    target = np.stack([_log_row([0, 1, 0, 0]), _log_row([1, 0, 0, 0])])[None]
+    al, out, pd, mg = oracle.verify_rejection(target, "f32", qrow[None, None], np.array([[0]], np.int32), 1.0,
+                                              seed, 0)
+    assert al[0] == 0 and out[0].tolist() == [1, -1]
+    assert abs(mg[0] / eps - 1) < 1e-9, (mg[0], eps)
+
+
+def test_rejection_margin_zero_q_draft():
+    """A draft q gives no mass is accepted iff p(d) > 0, whatever the uniform:
+    its distance from the boundary is p(d) itself."""
+    seed, (_, (_, ur1)) = _seed_where(lambda us: min(us[1][1], 1 - us[1][1]) > 0.1, (0, 1))
+    target = np.stack([_log_row([0.01, 0.99, 0, 0]), _log_row([1, 0, 0, 0])])[None]
+    q = np.array([[[0, 1, 0, 0]]], np.float32)
+    al, out, pd, mg = oracle.verify_rejection(target, "f32", q, np.array([[0]], np.int32), 1.0, seed, 0)
+    assert al[0] == 1 and out[0].tolist() == [0, 0]
+    assert abs(mg[0] - 0.01) < 1e-6, mg[0]
+
+
+def test_rejection_margin_bonus_only_and_invalid():
+    """k = 0: only the bonus draw from p_0; with p uniform over n tokens the
+    bins are 1/n wide and the margin is u_res's distance to the nearest
+    multiple of 1/n.  An invalid request has no decision: margin +inf."""
+    n = 8
+    for seed in (3, 4, 5):
+        _, ur = oracle.uniforms(seed, 0, 0, 0)
+        target = np.zeros((1, 1, n), np.float32)
+        al, out, pd, mg = oracle.verify_rejection(target, "f32", np.zeros((1, 0, n), np.float32),
+                                                  np.zeros((1, 0), np.int32), 1.0, seed, 0)
+        x = ur * n
+        assert al[0] == 0 and out[0, 0] == int(math.floor(x))
+        assert abs(mg[0] - min(x - math.floor(x), math.ceil(x) - x) / n) < 1e-12
+    t = np.zeros((1, 2, 4), np.float32)
+    t[0, 1, 2] = np.nan
+    _, _, _, mg = oracle.verify_rejection(t, "f32", np.full((1, 1, 4), 0.25, np.float32),
+                                          np.array([[1]], np.int32), 1.0, 1, 0)
+    assert mg[0] == math.inf
