@@ -47,9 +47,20 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     directly).
     """
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    lsb = (u >> np.uint32(16)) & np.uint32(1)
-    r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
-    return r.astype(np.uint16)
+    out = np.empty(u.shape, dtype=np.uint16)
+    flat_u, flat_o = u.reshape(-1), out.reshape(-1)
+    step = 1 << 20  # in slices, so the temporaries stay in cache
+    t = np.empty(min(step, flat_u.size), dtype=np.uint32)
+    for i in range(0, flat_u.size, step):
+        src = flat_u[i:i + step]
+        w = t[:src.size]
+        np.right_shift(src, np.uint32(16), out=w)
+        np.bitwise_and(w, np.uint32(1), out=w)
+        np.add(w, np.uint32(0x7FFF), out=w)
+        np.add(w, src, out=w)
+        np.right_shift(w, np.uint32(16), out=w)
+        flat_o[i:i + step] = w
+    return out
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

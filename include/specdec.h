@@ -404,9 +404,15 @@ specdec_status specdec_ngram_propose(const int32_t* tokens, int64_t token_stride
  *     a top-8 call clears its threshold words on `stream` first.  Calls that
  *     may overlap on the GPU (other streams, other threads) race: serialise
  *     them or use specdec_verify_greedy with separate workspaces.
- *   - A call whose workspace need (specdec_workspace_size) exceeds
- *     SPECDEC_STATIC_SCRATCH_BYTES returns SPECDEC_ERR_WORKSPACE and launches
- *     nothing. */
+ *   - Arguments are checked before any CUDA call: a rejected call returns
+ *     its status and enqueues nothing.  A call whose workspace need
+ *     (specdec_workspace_size) exceeds SPECDEC_STATIC_SCRATCH_BYTES returns
+ *     SPECDEC_ERR_WORKSPACE.
+ *   - The kernels run on the CURRENT device: `stream` and every pointer must
+ *     belong to it.
+ *   - The scratch address is cached per device for the life of the process;
+ *     do not use this entry point across a cudaDeviceReset (the module, and
+ *     with it the array, may be loaded at another address afterwards). */
 #define SPECDEC_STATIC_SCRATCH_BYTES (8u << 20)
 specdec_status specdec_verify_greedy_static_scratch(const void* logits, specdec_dtype dtype, int64_t row_stride,
                                                     const int32_t* draft_tokens, int B, int k, int V,

@@ -150,6 +150,25 @@ def _ptr(x):
     return x.data_ptr()
 
 
+def _on_current_device(*tensors, stream=None):
+    """The entry points without a Verifier launch on the current CUDA device:
+    tensor arguments (and a torch stream) on another device are refused
+    before anything is launched (a kernel would read another GPU's memory)."""
+    import torch
+    cur = None
+    for t in tensors + ((stream,) if stream is not None and not isinstance(stream, int) else ()):
+        if t is None or isinstance(t, int):
+            continue
+        dv = getattr(t, "device", None)
+        if dv is None or dv.type != "cuda":
+            raise ValueError("verifier arrays must be CUDA device tensors, got one on %s"
+                             % (dv if dv is not None else type(t).__name__))
+        if cur is None:
+            cur = torch.cuda.current_device()
+        if dv.index is not None and dv.index != cur:
+            raise ValueError("arguments must be on the current device cuda:%d, got one on %s" % (cur, dv))
+
+
 def _stream(s):
     if s is None:
         import torch
@@ -678,6 +697,7 @@ def specdec_verify_greedy_static_scratch(logits, dtype, row_stride, draft_tokens
     """Greedy verification using the library's fixed device scratch instead of
     a caller workspace (for callers that cannot allocate device memory).
     Calls that may overlap on the GPU race on that scratch."""
+    _on_current_device(logits, draft_tokens, accept_len, out_tokens, topk_ids, topk_vals, stream=stream)
     fn = lib().specdec_verify_greedy_static_scratch
     if fn.argtypes is None:  # declare the C signature once (64-bit pointers and strides)
         P, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64

@@ -212,6 +212,24 @@ void fill_common(Pass1Params& P, const void* logits, int64_t row_stride, int V, 
 namespace specdec {
 namespace {
 
+// Every check specdec_verify_greedy makes before it launches anything, the
+// workspace's aside (B == 0 passes: such a call does nothing).
+specdec_status greedy_args_status(const void* logits, specdec_dtype dtype, int64_t row_stride,
+                                  const int32_t* draft_tokens, int B, int k, int V, const int32_t* accept_len,
+                                  const int32_t* out_tokens, int topk, const int32_t* topk_ids,
+                                  const float* topk_vals) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V < 1 || V > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (topk < 0 || topk > SPECDEC_MAX_TOPK) return SPECDEC_ERR_INVALID_ARG;
+    if (B == 0) return SPECDEC_OK;
+    if (!rows_fit(static_cast<int64_t>(B) * (k + 1), row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
+    if (logits == nullptr || accept_len == nullptr || out_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (k > 0 && draft_tokens == nullptr) return SPECDEC_ERR_INVALID_ARG;
+    if (topk > 0 && (topk_ids == nullptr || topk_vals == nullptr)) return SPECDEC_ERR_INVALID_ARG;
+    return SPECDEC_OK;
+}
+
 // Greedy verification over `rows` logit rows: the fixed layout (offsets null,
 // k drafts per request, rows = B (k + 1)) or the packed one (offsets [B+1],
 // k = the bound on every request's count, rows = B + total drafts).
@@ -728,11 +746,9 @@ specdec_status specdec_verify_greedy(const void* logits, specdec_dtype dtype, in
                                      int32_t* accept_len, int32_t* out_tokens,
                                      int topk, int32_t* topk_ids, float* topk_vals,
                                      void* ws, size_t ws_bytes, struct CUstream_st* stream) {
-    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
-    if (B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V < 1 || V > SPECDEC_MAX_V)
-        return SPECDEC_ERR_INVALID_ARG;
-    if (topk < 0 || topk > SPECDEC_MAX_TOPK) return SPECDEC_ERR_INVALID_ARG;
-    if (B == 0) return SPECDEC_OK;
+    const specdec_status st = greedy_args_status(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len,
+                                                 out_tokens, topk, topk_ids, topk_vals);
+    if (st != SPECDEC_OK || B == 0) return st;
     return greedy_impl(logits, dtype, row_stride, draft_tokens, nullptr, static_cast<int64_t>(B) * k, B, k, V,
                        accept_len, out_tokens, topk, topk_ids, topk_vals, nullptr, ws, ws_bytes,
                        reinterpret_cast<cudaStream_t>(stream));
@@ -939,23 +955,26 @@ extern "C" specdec_status specdec_verify_greedy_static_scratch(
     const void* logits, specdec_dtype dtype, int64_t row_stride, const int32_t* draft_tokens, int B, int k, int V,
     int32_t* accept_len, int32_t* out_tokens, int topk, int32_t* topk_ids, float* topk_vals,
     struct CUstream_st* stream) {
+    // Every argument check comes before the first CUDA call, so a rejected
+    // call enqueues nothing (not even the threshold clear below).
+    specdec_status st = specdec::greedy_args_status(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len,
+                                                    out_tokens, topk, topk_ids, topk_vals);
+    if (st != SPECDEC_OK || B == 0) return st;
     const size_t need = specdec_workspace_size(SPECDEC_MODE_GREEDY, B, k, V, dtype);
     if (need > SPECDEC_STATIC_SCRATCH_BYTES) return SPECDEC_ERR_WORKSPACE;  // beyond the fixed scratch
     void* scratch = nullptr;
-    if (B > 0 && need > 0) {
-        if (specdec::static_scratch_address(&scratch) != cudaSuccess) return SPECDEC_ERR_CUDA;
-        // The top-8 row thresholds must start at zero.  Every completed call
-        // leaves them so, but the array keeps whatever a call that failed
-        // half-way left: clear this call's words first.
-        if (topk > 0 && k >= 0 && k <= SPECDEC_MAX_K) {
-            int64_t rows = static_cast<int64_t>(B) * (k + 1);
-            if (rows > specdec::kThetaRows) rows = specdec::kThetaRows;
-            if (cudaMemsetAsync(static_cast<char*>(scratch) + specdec::kThetaBase, 0,
-                                static_cast<size_t>(rows) * sizeof(unsigned),
-                                reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-                return SPECDEC_ERR_CUDA;
-        }
+    if (specdec::static_scratch_address(&scratch) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    // The top-8 row thresholds must start at zero.  Every completed call
+    // leaves them so, but the array keeps whatever a call that failed
+    // half-way left: clear this call's words first.
+    if (topk > 0) {
+        int64_t rows = static_cast<int64_t>(B) * (k + 1);
+        if (rows > specdec::kThetaRows) rows = specdec::kThetaRows;
+        if (cudaMemsetAsync(static_cast<char*>(scratch) + specdec::kThetaBase, 0,
+                            static_cast<size_t>(rows) * sizeof(unsigned),
+                            reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return SPECDEC_ERR_CUDA;
     }
     return specdec_verify_greedy(logits, dtype, row_stride, draft_tokens, B, k, V, accept_len, out_tokens, topk,
-                                 topk_ids, topk_vals, scratch, scratch ? SPECDEC_STATIC_SCRATCH_BYTES : 0, stream);
+                                 topk_ids, topk_vals, scratch, SPECDEC_STATIC_SCRATCH_BYTES, stream);
 }
