@@ -2,15 +2,23 @@
 """Throughput of the B200 speculative-decoding verifier.
 
 One step = one verify call over one batch of B requests (B*(k+1) logit rows
-of V entries), inputs already resident in HBM.  Default workload: greedy
-verification at the Llama-3 vocabulary, B=64, k=5, V=128256, bf16.
+of V entries), inputs already resident in HBM.  The headline workload
+(`value`) is greedy verification at the Llama-3 vocabulary, B=64, k=5,
+V=128256, bf16; the default run then times the other four verify
+configurations the same way and reports each under `workloads`: the tiny
+fp32 greedy batch, rejection sampling at the Qwen vocabulary, the large
+batch with per-position top-8, and the 64-node draft trees.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference]
+                    [--also A,B,...] [--intervals I] [--impl ours|reference]
 
-Prints one JSON line.  Multi-GPU: launched with torch.distributed.run, one
-rank per GPU; every rank verifies its own batch (requests are independent;
-no collective on the data path) and the time is the max over ranks.
+Prints one JSON line.  Every workload is timed as I regions of exactly K
+calls (a synchronize on both sides of each; a barrier too with N > 1); the
+median region gives the figure and the min and max are reported beside it.
+Multi-GPU: one rank per GPU (started here under torch.distributed.run when
+--gpus N > 1 is given without a launcher); every rank verifies its own
+batch (requests are independent; no collective on the data path) and each
+time is the max over ranks.
 
 The timed steps replay a CUDA graph of the C-ABI calls over a rotation of
 input sets whose total exceeds 4x the L2 cache, so every step streams its
@@ -110,6 +118,16 @@ def describe(inp):
         if inp.stats:
             d["adasd_stats"] = "draft entropy and Jensen-Shannon distance per draft position"
     return d
+
+
+L2_POLICY = "inputs rotate over device copies totalling more than 4x the L2 cache, so every call reads HBM"
+
+
+def line_config(name, inp, world):
+    """The `config` of a JSON line: the workload and its shape.  Both arms
+    (ours and the reference) emit the same dict for the same workload."""
+    return dict(workload=name, **describe(inp), l2=L2_POLICY,
+                parallelism="dp%d (requests per rank, no collective)" % world)
 
 
 def rows_of(inp, req=None):
@@ -299,38 +317,38 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def run_ours(args):
+def dist_max(values, device, world):
+    """Element-wise max over ranks of a list of floats (the list itself at one rank)."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def measure(name, args, world, rank, local, device, cpu_seconds):
+    """Times one workload on this rank's GPU and returns its entry of the JSON
+    line: `intervals` timed regions of exactly `steps` calls each (a barrier
+    and a synchronize on both sides of each), their median as the figure, the
+    min and max beside it, all maxed over ranks."""
     import torch
     import torch.distributed as dist
     import speculative_decoding_draft_decode_b200 as sd
-    from speculative_decoding_draft_decode_b200 import build as sd_build
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    if rank == 0 or world == 1:
-        sd_build.build()
-    if world > 1:
-        dist.barrier()
-
-    inp = make_workload(args.workload, seed_offset=rank)
+    inp = make_workload(name, seed_offset=rank)
     set_bytes = gen.algorithmic_bytes(inp)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     n_sets = max(2, math.ceil(4 * l2 / set_bytes) + 1) if args.sets is None else args.sets
     sets = DeviceSets(inp, n_sets, device).sets
     ver = sd.Verifier(device)
-    sd.specdec_set_prefetch_inputs(args.prefetch_inputs)
+    sd.specdec_set_prefetch_inputs(False)
     calls, outs, kpl = setup_calls(inp, sets, ver, device)
     # The input sets and outputs were made on the default stream (the rolled
     # sets by kernels still queued there, and the outputs may reuse blocks of
     # its freed temporaries); the calls run on a stream of their own.
     torch.cuda.synchronize(device)
-
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
         for c in calls:  # allocates the workspace, loads the kernels
@@ -349,10 +367,12 @@ def run_ours(args):
             graphs[n] = g
         return graphs[n]
 
-    graph_of(per_replay)
-    for n in (args.warmup, args.steps):
-        if n % per_replay:
-            graph_of(n % per_replay)
+    def capture_all():
+        graphs.clear()  # the prefetch setting is baked into captured kernels
+        graph_of(per_replay)
+        for n in (args.warmup, args.steps):
+            if n % per_replay:
+                graph_of(n % per_replay)
 
     def run_steps(n):
         # exactly n calls, all from captured graphs
@@ -362,11 +382,31 @@ def run_ours(args):
         if rest:
             graph_of(rest).replay()
 
-    with torch.cuda.stream(stream):
-        run_steps(args.warmup)
-    stream.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
 
-    # clocks: sample across a 1 s burst of the same steps and the timed region
+    def timed_intervals():
+        with torch.cuda.stream(stream):
+            run_steps(args.warmup)
+        stream.synchronize()
+        ms = []
+        for _ in range(args.intervals):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(device)
+            with torch.cuda.stream(stream):
+                ev0.record(stream)
+                run_steps(args.steps)
+                ev1.record(stream)
+            torch.cuda.synchronize(device)
+            ms.append(ev0.elapsed_time(ev1))
+        if world > 1:
+            dist.barrier()
+        med, lo, hi = dist_max([statistics.median(ms), min(ms), max(ms)], device, world)
+        return med / args.steps, lo / args.steps, hi / args.steps
+
+    capture_all()
+    # clocks: sampled across a short untimed burst of the same steps and the timed region
     sampler = ClockSampler(local, args.clock_log_dir)
     sampler.start()
     t_probe = time.time()
@@ -374,112 +414,119 @@ def run_ours(args):
         while time.time() - t_probe < args.clock_probe_seconds:
             run_steps(per_replay * 50)
             stream.synchronize()
-
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(device)
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        run_steps(args.steps)
-        ev1.record(stream)
-    torch.cuda.synchronize(device)
-    if world > 1:
-        dist.barrier()
-    ms = ev0.elapsed_time(ev1)
+    ms_step, ms_lo, ms_hi = timed_intervals()
     clocks = sampler.stop()
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
 
-    # The same steps again with the opt-in early loads of the argmax pass
+    # The same steps with the opt-in early loads of the streaming pass
     # (specdec_set_prefetch_inputs), reported beside the default: safe here,
     # the inputs were written by torch before any timed region.
     prefetch = None
-    if not args.prefetch_inputs:
+    if not args.no_prefetch_leg:
         sd.specdec_set_prefetch_inputs(True)
-        graphs.clear()  # the setting is baked into captured kernels: capture again
-        graph_of(per_replay)
-        for n in (args.warmup, args.steps):
-            if n % per_replay:
-                graph_of(n % per_replay)
-        with torch.cuda.stream(stream):
-            run_steps(args.warmup)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(device)
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            run_steps(args.steps)
-            ev1.record(stream)
-        torch.cuda.synchronize(device)
-        if world > 1:
-            dist.barrier()
-        pt = torch.tensor([ev0.elapsed_time(ev1)], dtype=torch.float64, device=device)
-        if world > 1:
-            dist.all_reduce(pt, op=dist.ReduceOp.MAX)
+        capture_all()
+        prefetch = timed_intervals()
         sd.specdec_set_prefetch_inputs(False)
-        prefetch = float(pt.item()) / args.steps
 
     # end to end: inputs from pinned host memory, H2D + verify + D2H each step
     e2e = run_e2e(inp, ver, device, stream, args.e2e_steps) if args.e2e_steps > 0 else None
-    if world > 1 and e2e is not None:
-        t = torch.tensor([e2e["ms_per_step"]], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["ms_per_step"] = float(t.item())
+    if e2e is not None:
+        e2e["ms_per_step"] = dist_max([e2e["ms_per_step"]], device, world)[0]
 
     rows = rows_of(inp)
-    ms_step = ms_max / args.steps
-    value = rows * world / (ms_step / 1e3)
     peak, peak_kind = measured_peak()
     alg_bytes = set_bytes + resample_bytes(inp, outs)
     achieved = alg_bytes / (ms_step / 1e3) / 1e9
+    res = {
+        "value": rows * world / (ms_step / 1e3),
+        "unit": "rows/s",
+        "ms_per_step": ms_step,
+        "us_per_call": ms_step * 1e3,
+        "requests_per_s": inp.B * world / (ms_step / 1e3),
+        "intervals": {"n": args.intervals, "steps_each": args.steps, "ms_per_step_median": ms_step,
+                      "ms_per_step_min": ms_lo, "ms_per_step_max": ms_hi},
+        "dtype": inp.dtype,
+        "config": line_config(name, inp, world),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                     % peak_kind if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "algorithmic_bytes_per_launch": alg_bytes, "traffic": recorded_traffic(name),
+                     "duration_us": ms_step * 1e3, "kernels_per_step": kpl,
+                     "note": "one call of every kernel of the step; duration = median timed region / steps "
+                             "(launch gaps included)"},
+        "timing": {"input_sets": n_sets, "input_bytes": n_sets * set_bytes, "l2_bytes": l2,
+                   "launch": "CUDA graph of %d C-ABI calls, replayed" % per_replay},
+        "gpu_launches": args.intervals * args.steps * kpl,
+        "clocks": clocks,
+    }
+    if inp.B * (getattr(inp, "k", 0) + 1) * inp.V < 4_000_000:
+        res["roofline"]["note"] += "; latency-bound at this size (report the time per call)"
+    if prefetch is not None:
+        pa = alg_bytes / (prefetch[0] / 1e3) / 1e9
+        res["prefetch_inputs"] = {
+            "note": "same steps with specdec_set_prefetch_inputs(1): the streaming pass loads its rows before the "
+                    "previous kernel ends (opt-in; the library default is off and gives `value`)",
+            "ms_per_step": prefetch[0], "ms_per_step_min": prefetch[1], "ms_per_step_max": prefetch[2],
+            "value": rows * world / (prefetch[0] / 1e3), "achieved_gbs": pa, "frac": pa / peak}
+    if e2e is not None:
+        res["e2e"] = {"value": rows * world / (e2e["ms_per_step"] / 1e3), "unit": "rows/s",
+                      "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                      "ms_per_step": e2e["ms_per_step"]}
+    if rank == 0 and cpu_seconds > 0:
+        res["cpu_baseline"] = cpu_baseline(inp, cpu_seconds)
+    graphs.clear()
+    del sets, calls, outs, ver
+    torch.cuda.synchronize(device)
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_draft_decode_b200 import build as sd_build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if rank == 0 or world == 1:
+        sd_build.build()
+    if world > 1:
+        dist.barrier()
+
+    head = measure(args.workload, args, world, rank, local, device, args.cpu_baseline_seconds)
+    others = {}
+    for name in args.also:
+        if name != args.workload:
+            others[name] = measure(name, args, world, rank, local, device, args.cpu_baseline_seconds / 3)
     line = {
         "metric": METRIC,
-        "value": value,
+        "value": head["value"],
         "unit": "rows/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms_step,
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": inp.dtype,
+        "dtype": head["dtype"],
         "data": "synthetic",
-        "config": dict(workload=args.workload, **describe(inp), requests_per_s=inp.B * world / (ms_step / 1e3),
-                       l2="rotating %d input sets, %.0f MB > 4x L2 (%d MB)" % (n_sets, n_sets * set_bytes / 1e6,
-                                                                             l2 // 2**20),
-                       launch="CUDA graph of %d C-ABI calls, replayed%s" % (
-                           per_replay, "; prefetch_inputs on" if args.prefetch_inputs else ""),
-                       parallelism="dp%d (requests per rank, no collective)" % world),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-                     % peak_kind if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "algorithmic_bytes_per_launch": alg_bytes, "traffic": recorded_traffic(args.workload),
-                     "duration_us": ms_step * 1e3, "kernels_per_step": kpl,
-                     "note": "duration = timed region / steps (launch gaps included)"},
-        "gpu_launches": args.steps * kpl,
-        "clocks": clocks,
+        "config": head["config"],
     }
-    if prefetch is not None:
-        pa = alg_bytes / (prefetch / 1e3) / 1e9
-        line["prefetch_inputs"] = {
-            "note": "same steps with specdec_set_prefetch_inputs(1): the streaming pass loads its rows before the "
-                    "previous kernel ends (opt-in; the library default is off and gives `value`)",
-            "ms_per_step": prefetch, "value": rows * world / (prefetch / 1e3), "achieved_gbs": pa,
-            "frac": pa / peak}
-    if e2e is not None:
-        line["e2e"] = {"value": rows * world / (e2e["ms_per_step"] / 1e3), "unit": "rows/s",
-                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                       "ms_per_step": e2e["ms_per_step"]}
-    if rank == 0 and args.cpu_baseline_seconds > 0:
-        line["cpu_baseline"] = cpu_baseline(inp, args.cpu_baseline_seconds)
+    for key in ("requests_per_s", "intervals", "roofline", "gpu_launches", "clocks", "timing", "prefetch_inputs",
+                "e2e", "cpu_baseline"):
+        if key in head:
+            line[key] = head[key]
+    if others:
+        line["workloads"] = others
+        line["gpu_launches_all_workloads"] = head["gpu_launches"] + sum(o["gpu_launches"] for o in others.values())
     if world > 1:
         dist.barrier()
-        graphs.clear()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -600,42 +647,93 @@ def run_reference(args):
     el = time.perf_counter() - t0
     value = rows_of(inp, req) * args.steps / el
     sample = "first %d of %d requests per step, fp64 C++ oracle on %d threads" % (req, inp.B, th)
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus or 1)))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype,
-            "data": "synthetic", "config": dict(workload=args.workload, **describe(inp)),
+            "data": "synthetic", "config": line_config(args.workload, inp, world),
             "cpu_baseline": {"value": value, "unit": "rows/s", "cores": th, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def main():
+SUITE = ("greedy_llama3", "greedy_tiny", "rejection_qwen", "greedy_large_batch", "tree_medusa")
+WORKLOADS = SUITE + ("greedy_ragged_tiers", "rejection_qwen_adasd")
+
+
+def relaunch_under_torchrun(args):
+    """`--gpus N` (N > 1) without a torch.distributed launcher: start N ranks
+    here, one per GPU, and return their exit status."""
+    import signal
+    import socket
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=%d" % args.gpus,
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    proc = subprocess.Popen(cmd, start_new_session=True)
+    try:
+        return proc.wait(timeout=args.launch_timeout)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGTERM)
+        try:
+            proc.wait(timeout=60)
+        except subprocess.TimeoutExpired:
+            os.killpg(proc.pid, signal.SIGKILL)
+        print("bench: the %d ranks did not finish within %d s" % (args.gpus, args.launch_timeout), file=sys.stderr)
+        return 1
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=None,
+                    help="GPUs (one rank each); without a torch.distributed launcher N > 1 starts the ranks itself")
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--clock-log-dir", default=None,
                     help="directory for the raw nvidia-smi clock samples (default: the system temp directory)")
-    ap.add_argument("--workload", default="greedy_llama3",
-                    choices=["greedy_llama3", "greedy_tiny", "rejection_qwen", "greedy_large_batch", "tree_medusa",
-                             "greedy_ragged_tiers", "rejection_qwen_adasd"])
+    ap.add_argument("--workload", default="greedy_llama3", choices=WORKLOADS,
+                    help="the headline workload (`value` of the line)")
+    ap.add_argument("--also", default=",".join(w for w in SUITE if w != "greedy_llama3"),
+                    help="comma-separated workloads timed after the headline one and reported under `workloads` "
+                         "(default: the rest of the five verify configurations; '' for none)")
+    ap.add_argument("--intervals", type=int, default=30, help="timed regions of exactly --steps calls per workload")
     ap.add_argument("--sets", type=int, default=None, help="input sets in the rotation (default: > 4x L2)")
-    ap.add_argument("--prefetch-inputs", action="store_true",
-                    help="opt in to the streaming pass loading its rows before the previous kernel ends "
-                         "(safe here: the inputs are written by torch before the timed region)")
+    ap.add_argument("--no-prefetch-leg", action="store_true",
+                    help="skip timing the opt-in early-load mode beside the default")
     ap.add_argument("--e2e-steps", type=int, default=20)
-    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0,
+                    help="oracle time for the headline workload's CPU baseline (a third of it for each other one)")
     ap.add_argument("--clock-probe-seconds", type=float, default=1.0,
                     help="untimed burst of the same steps while nvidia-smi samples clocks")
-    args = ap.parse_args()
+    ap.add_argument("--launch-timeout", type=int, default=1800, help="seconds for ranks started by --gpus N")
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.steps < 1 or args.intervals < 1:
+        ap.error("--steps and --intervals must be positive")
+    args.also = [w for w in args.also.split(",") if w]
+    bad = [w for w in args.also if w not in WORKLOADS]
+    if bad:
+        ap.error("unknown workloads in --also: %s" % ", ".join(bad))
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is not None and args.gpus is not None and int(env_world) != args.gpus:
+        ap.error("--gpus %d but the launcher started WORLD_SIZE=%s ranks" % (args.gpus, env_world))
+    return args
+
+
+def main():
+    args = parse_args()
     if args.impl == "reference":
         run_reference(args)
-    else:
-        run_ours(args)
+        return 0
+    if os.environ.get("WORLD_SIZE") is None and (args.gpus or 1) > 1:
+        return relaunch_under_torchrun(args)
+    run_ours(args)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

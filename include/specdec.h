@@ -155,6 +155,22 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
                                         int32_t* accept_len, int32_t* out_tokens, float* p_draft_out,
                                         void* ws, size_t ws_bytes, struct CUstream_st* stream);
 
+/* Rejection-sampling verification of a slice of a larger batch: requests
+ * request_base .. request_base + B - 1 of it (vLLM page, section 1, as
+ * specdec_verify_rejection).  Request b of this call draws the Philox
+ * uniforms of global request request_base + b (counter (request_base + b, i,
+ * offset_lo, offset_hi)), so a batch split by request over several calls or
+ * ranks, each passing the index of its first request, gives exactly the
+ * results of one call over the whole batch.  Every other argument and result
+ * as specdec_verify_rejection; request_base + B must not exceed 2^32
+ * (SPECDEC_ERR_INVALID_ARG).  request_base = 0 is specdec_verify_rejection. */
+specdec_status specdec_verify_rejection_slice(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
+                                              const float* draft_probs, int64_t q_row_stride,
+                                              const int32_t* draft_tokens, int B, int k, int V, float temperature,
+                                              uint64_t seed, uint64_t offset, uint32_t request_base,
+                                              int32_t* accept_len, int32_t* out_tokens, float* p_draft_out,
+                                              void* ws, size_t ws_bytes, struct CUstream_st* stream);
+
 /* Tree verification (handbook, "Medusa": candidates form a tree and the
  * longest accepted candidate prefix is kept; "EAGLE": EAGLE-2 draft trees).
  *   logits       [B, N+1, V]; row c scores the children of node c; row 0 is

@@ -30,6 +30,8 @@ def _bind(path):
     L.oracle_verify_tree.argtypes = [P, i32, i64, P, P, i32, i32, i32, i32, P, P, P]
     L.oracle_verify_rejection.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f64, u64, u64,
                                           P, P, P, P]
+    L.oracle_verify_rejection_slice.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f64, u64, u64, u32,
+                                                P, P, P, P]
     L.oracle_verify_greedy_ragged.argtypes = [P, i32, i64, P, P, i32, i64, i32, i32, P, P, i32, P, P, P]
     L.oracle_verify_rejection_ragged.argtypes = [P, i32, i64, P, i64, P, P, i32, i64, i32, i32, f64, u64, u64,
                                                  P, P, P, P, P]
@@ -40,7 +42,7 @@ def _bind(path):
     L.oracle_draft_stats.argtypes = [P, i32, i64, P, i64, i32, i32, i32, f64, P, P]
     L.oracle_ngram_propose.argtypes = [P, i64, P, i32, i32, i32, i32, P, P]
     for f in ("oracle_ngram_propose", "oracle_draft_stats", "oracle_philox4x32_10", "oracle_uniforms", "oracle_argmax_rows", "oracle_topk_rows",
-              "oracle_verify_greedy", "oracle_verify_tree", "oracle_verify_rejection",
+              "oracle_verify_greedy", "oracle_verify_tree", "oracle_verify_rejection", "oracle_verify_rejection_slice",
               "oracle_verify_greedy_ragged", "oracle_verify_rejection_ragged", "oracle_verify_greedy_parallel",
               "oracle_verify_tree_parallel", "oracle_verify_rejection_parallel"):
         getattr(L, f).restype = None
@@ -160,8 +162,10 @@ def verify_tree(logits, dtype, parents, node_tokens, max_depth, threads=1):
     return al, nodes, out
 
 
-def verify_rejection(target, dtype, q, drafts, temperature, seed, offset, threads=1):
-    """target [B, k+1, V]; q [B, k, V] float32 -> (accept_len, out_tokens, p_draft, margin)."""
+def verify_rejection(target, dtype, q, drafts, temperature, seed, offset, threads=1, request_base=0):
+    """target [B, k+1, V]; q [B, k, V] float32 -> (accept_len, out_tokens, p_draft, margin).
+    With request_base, the arrays are requests request_base .. of a larger
+    batch and draw that batch's uniforms."""
     x = _logit_array(target, dtype)
     B, k1, V = x.shape
     k = k1 - 1
@@ -171,6 +175,11 @@ def verify_rejection(target, dtype, q, drafts, temperature, seed, offset, thread
     out = np.zeros((B, k1), np.int32)
     pd = np.zeros((B, max(k, 1)), np.float64)
     mg = np.zeros(B, np.float64)
+    if request_base:
+        lib().oracle_verify_rejection_slice(_ptr(x), DTYPE_CODE[dtype], V, _ptr(qq), V, _ptr(d), B, k, V,
+                                            float(temperature), int(seed), int(offset), int(request_base),
+                                            _ptr(al), _ptr(out), _ptr(pd), _ptr(mg))
+        return al, out, pd[:, :k], mg
     fn = lib().oracle_verify_rejection_parallel if threads > 1 else lib().oracle_verify_rejection
     extra = (threads,) if threads > 1 else ()
     fn(_ptr(x), DTYPE_CODE[dtype], V, _ptr(qq), V, _ptr(d), B, k, V, float(temperature), int(seed), int(offset),

@@ -476,6 +476,20 @@ void oracle_verify_rejection(const void* target, int dtype, int64_t row_stride,
                           out_tokens + (int64_t)b * (k + 1), p_draft + (int64_t)b * k, &margin[b]);
 }
 
+// The same for requests base .. base + B - 1 of a larger batch: request b of
+// the arrays draws the uniforms of request index base + b, so the requests
+// of one batch give the same results in one call or split over several.
+void oracle_verify_rejection_slice(const void* target, int dtype, int64_t row_stride,
+                                   const float* q, int64_t q_row_stride, const int32_t* drafts,
+                                   int B, int k, int V, double temperature, uint64_t seed, uint64_t offset,
+                                   uint32_t base, int32_t* accept_len, int32_t* out_tokens, double* p_draft,
+                                   double* margin) {
+    for (int b = 0; b < B; ++b)
+        rejection_request(target, dtype, row_stride, (int64_t)b * (k + 1), q, q_row_stride, (int64_t)b * k,
+                          drafts + (int64_t)b * k, k, V, temperature, seed, offset, base + (uint32_t)b,
+                          &accept_len[b], out_tokens + (int64_t)b * (k + 1), p_draft + (int64_t)b * k, &margin[b]);
+}
+
 // Rejection-sampling verification in the packed layout of
 // oracle_verify_greedy_ragged: request b's k_b + 1 target rows and output
 // slots start at row off[b] + b, its q rows and p_draft entries at off[b];

@@ -28,7 +28,7 @@ __all__ = [
     "SPECDEC_OK", "SPECDEC_F32", "SPECDEC_BF16", "SPECDEC_MODE_GREEDY", "SPECDEC_MODE_REJECTION",
     "SPECDEC_MODE_TREE", "SpecdecError", "lib", "library_path", "header_path",
     "specdec_workspace_size", "specdec_workspace_init", "specdec_verify_greedy",
-    "specdec_verify_rejection", "specdec_verify_tree", "specdec_status_string", "specdec_abi_version",
+    "specdec_verify_rejection", "specdec_verify_rejection_slice", "specdec_verify_tree", "specdec_status_string", "specdec_abi_version",
     "Verifier",
 ]
 
@@ -91,6 +91,9 @@ def lib():
         L.specdec_verify_rejection.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f32, u64, u64,
                                                P, P, P, P, sz, P]
         L.specdec_verify_rejection.restype = i32
+        L.specdec_verify_rejection_slice.argtypes = [P, i32, i64, P, i64, P, i32, i32, i32, f32, u64, u64,
+                                                     ctypes.c_uint32, P, P, P, P, sz, P]
+        L.specdec_verify_rejection_slice.restype = i32
         L.specdec_verify_tree.argtypes = [P, i32, i64, P, P, i32, i32, i32, i32, P, P, P, P, sz, P]
         L.specdec_verify_tree.restype = i32
         L.specdec_workspace_size_ragged.argtypes = [i32, i32, i32, i32, i32]
@@ -212,6 +215,16 @@ def specdec_verify_rejection(target_logits, dtype, row_stride, draft_probs, q_ro
                                           int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
                                           _ptr(accept_len), _ptr(out_tokens), _ptr(p_draft_out),
                                           _ptr(ws), ws_bytes, _stream(stream))
+
+
+def specdec_verify_rejection_slice(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens,
+                                   B, k, V, temperature, seed, offset, request_base, accept_len, out_tokens,
+                                   p_draft_out, ws, ws_bytes, stream=None) -> int:
+    return lib().specdec_verify_rejection_slice(_ptr(target_logits), dtype, row_stride, _ptr(draft_probs),
+                                                q_row_stride, _ptr(draft_tokens), B, k, V, float(temperature),
+                                                int(seed) & (2**64 - 1), int(offset) & (2**64 - 1),
+                                                int(request_base), _ptr(accept_len), _ptr(out_tokens),
+                                                _ptr(p_draft_out), _ptr(ws), ws_bytes, _stream(stream))
 
 
 def specdec_verify_rejection_stats(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens,
@@ -449,11 +462,15 @@ class Verifier:
         return al, nodes, ot
 
     def rejection(self, target_logits, draft_probs, draft_tokens, temperature: float, seed: int, offset: int = 0,
-                  stream=None, out=None, want_p_draft: bool = True, stats: bool = False):
+                  stream=None, out=None, want_p_draft: bool = True, stats: bool = False, request_base: int = 0):
         """target_logits [B, k+1, V], draft_probs [B, k, V] f32, draft_tokens
         [B, k] int32 -> (accept_len [B], out_tokens [B, k+1], p_draft [B, k]);
         with stats=True also (draft_entropy [B, k], js_distance [B, k]) float64
-        (AdaSD's statistics; `out` then holds five tensors)."""
+        (AdaSD's statistics; `out` then holds five tensors).  request_base:
+        these are requests request_base .. of a larger batch, drawing that
+        batch's uniforms (specdec_verify_rejection_slice)."""
+        if request_base and stats:
+            raise ValueError("request_base is not supported together with stats")
         import torch
         self._on_device(target_logits, draft_probs if target_logits.shape[1] > 1 else None, draft_tokens if target_logits.shape[1] > 1 else None, *(out or ()))
         B, k1, V = target_logits.shape
@@ -485,8 +502,13 @@ class Verifier:
                                                   seed, offset, al, ot, pd, ent, js, ws, wsb, stream),
                    "verify_rejection_stats")
             return al, ot, (pd[:, :k] if pd is not None else None), ent[:, :k], js[:, :k]
-        _check(specdec_verify_rejection(target_logits, dt, stride, q, q_stride, d, B, k, V, temperature, seed,
-                                        offset, al, ot, pd, ws, wsb, stream), "verify_rejection")
+        if request_base:
+            _check(specdec_verify_rejection_slice(target_logits, dt, stride, q, q_stride, d, B, k, V, temperature,
+                                                  seed, offset, request_base, al, ot, pd, ws, wsb, stream),
+                   "verify_rejection_slice")
+        else:
+            _check(specdec_verify_rejection(target_logits, dt, stride, q, q_stride, d, B, k, V, temperature, seed,
+                                            offset, al, ot, pd, ws, wsb, stream), "verify_rejection")
         return al, ot, (pd[:, :k] if pd is not None else None)
 
 

@@ -270,7 +270,7 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
                               const int32_t* offsets, int64_t total, int B, int k, int V, float temperature,
                               uint64_t seed, uint64_t offset, int32_t* accept_len, int32_t* out_tokens,
                               float* p_draft_out, int64_t* counters, double* entropy, double* js, void* ws,
-                              size_t ws_bytes, cudaStream_t s) {
+                              size_t ws_bytes, cudaStream_t s, uint32_t req_base = 0) {
     if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
     const int64_t rows = offsets ? B + total : static_cast<int64_t>(B) * (k + 1);
     if (!rows_fit(rows, row_stride, V)) return SPECDEC_ERR_INVALID_ARG;
@@ -303,6 +303,7 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     P.offset = offset;
     P.p_draft_out = p_draft_out;
     P.state = state;
+    P.req_base = req_base;
     const bool stats = entropy != nullptr && offsets == nullptr && k > 0;
     P.row_stat = stats ? reinterpret_cast<RowStat*>(static_cast<char*>(ws) + L.row_stat) : nullptr;
     st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
@@ -322,6 +323,7 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     Q.log2e_invT = P.log2e_invT;
     Q.seed = seed;
     Q.offset = offset;
+    Q.req_base = req_base;
     Q.state = state;
     Q.chunk_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.masses);
     Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
@@ -816,6 +818,25 @@ specdec_status specdec_verify_rejection(const void* target_logits, specdec_dtype
                           static_cast<int64_t>(B) * k, B, k, V, temperature, seed, offset, accept_len, out_tokens,
                           p_draft_out, nullptr, nullptr, nullptr, ws, ws_bytes,
                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+specdec_status specdec_verify_rejection_slice(const void* target_logits, specdec_dtype dtype, int64_t row_stride,
+                                              const float* draft_probs, int64_t q_row_stride,
+                                              const int32_t* draft_tokens, int B, int k, int V, float temperature,
+                                              uint64_t seed, uint64_t offset, uint32_t request_base,
+                                              int32_t* accept_len, int32_t* out_tokens, float* p_draft_out,
+                                              void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+    if (!dtype_ok(dtype)) return SPECDEC_ERR_UNSUPPORTED;
+    if (B < 0 || B > SPECDEC_MAX_B || k < 0 || k > SPECDEC_MAX_K || V < 1 || V > SPECDEC_MAX_V)
+        return SPECDEC_ERR_INVALID_ARG;
+    if (!(isnormal(temperature) && temperature > 0.0f)) return SPECDEC_ERR_INVALID_ARG;
+    if (static_cast<uint64_t>(request_base) + static_cast<uint64_t>(B) > (uint64_t(1) << 32))
+        return SPECDEC_ERR_INVALID_ARG;  // a request index past 2^32 - 1
+    if (B == 0) return SPECDEC_OK;
+    return rejection_impl(target_logits, dtype, row_stride, draft_probs, q_row_stride, draft_tokens, nullptr,
+                          static_cast<int64_t>(B) * k, B, k, V, temperature, seed, offset, accept_len, out_tokens,
+                          p_draft_out, nullptr, nullptr, nullptr, ws, ws_bytes,
+                          reinterpret_cast<cudaStream_t>(stream), request_base);
 }
 
 specdec_status specdec_verify_rejection_stats(const void* target_logits, specdec_dtype dtype, int64_t row_stride,

@@ -138,6 +138,7 @@ struct Pass1Params {
     float* p_draft_out;
     RejState* state;
     RowStat* row_stat;          // [rows] every row's (M, Z), or null
+    uint32_t req_base;          // Philox request index of request 0 (a slice of a larger batch)
     int prefetch_inputs;            // the argmax pass may load rows before the previous kernel ends
     // vocabulary-sharded greedy
     int vocab_offset;               // global index of this shard's column 0
@@ -967,7 +968,8 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
                 qd = static_cast<double>(qf);
             }
             if (P.p_draft_out) P.p_draft_out[g.d0 + lane] = static_cast<float>(p);
-            const double2 u = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(lane));
+            const double2 u = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b) + P.req_base,
+                                              static_cast<uint32_t>(lane));
             accept = in && (u.x * qd < p);
         }
         const unsigned rej = __ballot_sync(FULL_MASK, lane < k && !accept);

@@ -59,6 +59,7 @@ struct Pass2Params {
     float log2e_invT;  // log2(e) / T
     uint64_t seed;
     uint64_t offset;
+    uint32_t req_base;    // Philox request index of request 0 (a slice of a larger batch)
     const RejState* state;
     double2* chunk_mass;  // [B, cpr] (residual mass, target mass) of row h
     double2* unit_mass;   // [B, cpr, units_per_chunk] likewise per unit
@@ -391,7 +392,8 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
     if (P.shard_totals == nullptr) {
         use_p = !(tr > 0.0);
         const double S = use_p ? tp : tr;
-        const double2 uu = verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b), static_cast<uint32_t>(st.h));
+        const double2 uu =
+            verify_uniforms(P.seed, P.offset, static_cast<uint32_t>(b) + P.req_base, static_cast<uint32_t>(st.h));
         target = uu.y * S;
     } else {
         // Vocabulary shards in rank order are the row in index order: the

@@ -4,9 +4,10 @@ By request: requests are independent, so a batch shards by request with no
 exchange on the data path: rank i verifies requests [start_i, stop_i) of the
 global batch and the per-request outputs are concatenated in rank order.
 Greedy and tree results are identical to the unsharded call.  In rejection
-mode the Philox counter uses the request index *within the call*, so a
-sharded call draws other (equally valid) uniforms than an unsharded one
-unless every rank passes a distinct `offset`.
+mode every rank passes the global index of its first request
+(specdec_verify_rejection_slice), so each request draws the same Philox
+uniforms as in one call over the whole batch and the results are identical
+too (sharded_verify_rejection_requests).
 
 By vocabulary (Arctic page, "Speculator optimisation": with the scorer's
 tensor parallelism each GPU holds a slice of the vocabulary of every logit
@@ -50,6 +51,24 @@ def gather_requests(local, B: int, group=None):
         dist.all_gather(bufs, pad, group=group)
         out.append(torch.cat([b[: e - s] for b, (s, e) in zip(bufs, counts)], dim=0))
     return out
+
+
+def sharded_verify_rejection_requests(verifier, target, draft_probs, draft_tokens, temperature: float, seed: int,
+                                      offset: int = 0, group=None):
+    """Rejection-sampling verification of one global batch split by request:
+    this rank verifies its range [start, stop) of target [B, k+1, V],
+    draft_probs [B, k, V] and draft_tokens [B, k] (its CUDA kernels, keyed by
+    the global request index), and the outputs are all-gathered in batch
+    order.  Every rank returns (accept_len [B], out_tokens [B, k+1], p_draft
+    [B, k]), equal to the unsharded call's."""
+    import torch.distributed as dist
+    B = target.shape[0]
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    s, e = request_range(B, world, rank)
+    k = target.shape[1] - 1
+    q = draft_probs[s:e] if k > 0 else draft_probs
+    al, ot, pd = verifier.rejection(target[s:e], q, draft_tokens[s:e], temperature, seed, offset, request_base=s)
+    return gather_requests([al, ot, pd], B, group)
 
 
 def vocab_range(V: int, world: int, rank: int):

@@ -182,3 +182,19 @@ def test_missing_library_fails_loudly(tmp_path):
             sd.specdec_abi_version()
     finally:
         sd._lib, sd.library_path = saved_lib, saved_path
+
+
+def test_rejection_slice_argument_checks(L):
+    """request_base + B past 2^32 and the usual argument errors return before
+    any CUDA call."""
+    f = sd.specdec_verify_rejection_slice
+    F = FAKE
+    assert f(F, sd.SPECDEC_F32, 64, F, 64, F, 4, 2, 64, 1.0, 1, 0, 2**32 - 3, F, F, None, F, 1 << 20, 0) == \
+        sd.SPECDEC_ERR_INVALID_ARG
+    assert f(F, sd.SPECDEC_F32, 64, F, 64, F, 4, 2, 64, 0.0, 1, 0, 7, F, F, None, F, 1 << 20, 0) == \
+        sd.SPECDEC_ERR_INVALID_ARG
+    assert f(F, 9, 64, F, 64, F, 4, 2, 64, 1.0, 1, 0, 7, F, F, None, F, 1 << 20, 0) == sd.SPECDEC_ERR_UNSUPPORTED
+    assert f(None, sd.SPECDEC_F32, 64, None, 64, None, 0, 2, 64, 1.0, 1, 0, 2**32 - 1, None, None, None, None, 0,
+             0) == sd.SPECDEC_OK  # B = 0
+    assert f(F, sd.SPECDEC_F32, 64, F, 64, F, 4, 2, 64, 1.0, 1, 0, 7, F, F, None, F, 16, 0) == \
+        sd.SPECDEC_ERR_WORKSPACE

@@ -36,6 +36,8 @@ def test_reference_arm_line():
     assert d["data"] == "synthetic" and d["dtype"] == "bf16"
     assert d["config"]["workload"] == "greedy_llama3"
     assert (d["config"]["B"], d["config"]["k"], d["config"]["V"]) == (64, 5, 128256)
+    # the same config dict as our arm's line for the same workload
+    assert d["config"] == bench.line_config("greedy_llama3", bench.make_workload("greedy_llama3"), 1)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
@@ -44,6 +46,47 @@ def test_reference_arm_line():
 def test_reference_arm_other_ranks_do_nothing():
     res = _run(["--impl", "reference", "--steps", "1", "--warmup", "3"], env={"RANK": "1", "WORLD_SIZE": "2"})
     assert res.returncode == 0 and res.stdout.strip() == ""
+
+
+def test_argument_rules():
+    a = bench.parse_args([])
+    assert a.workload == "greedy_llama3" and a.intervals >= 30 and a.gpus is None
+    assert set(a.also) == set(bench.SUITE) - {"greedy_llama3"}
+    assert bench.parse_args(["--also", ""]).also == []
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--also", "greedy_tiny,nonsense"])
+
+
+def test_gpus_must_match_the_launcher():
+    """Under a launcher, --gpus N must equal the ranks it started."""
+    res = _run(["--gpus", "1", "--steps", "1", "--warmup", "3"], env={"WORLD_SIZE": "2", "RANK": "0"})
+    assert res.returncode != 0 and "WORLD_SIZE" in res.stderr
+
+
+def test_gpus_without_a_launcher_starts_the_ranks(monkeypatch):
+    """`--gpus N` (N > 1) with no launcher starts N ranks under
+    torch.distributed.run on 127.0.0.1 instead of timing one GPU."""
+    seen = {}
+
+    class FakeProc:
+        pid = 0
+
+        def wait(self, timeout=None):
+            return 0
+
+    def fake_popen(cmd, start_new_session=False):
+        seen["cmd"], seen["session"] = cmd, start_new_session
+        return FakeProc()
+
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(bench.subprocess, "Popen", fake_popen)
+    monkeypatch.setattr(bench, "run_ours", lambda a: pytest.fail("timed one GPU instead of starting the ranks"))
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "4", "--steps", "3", "--warmup", "3"])
+    assert bench.main() == 0
+    cmd = seen["cmd"]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"] and "--nproc-per-node=4" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1" and seen["session"]
+    assert cmd[-6:] == ["--gpus", "4", "--steps", "3", "--warmup", "3"]
 
 
 def test_warmup_floor():

@@ -235,3 +235,56 @@ def test_vocab_sharded_rejection_exchanges_gloo(world):
     assert all(p.exitcode == 0 for p in procs)
     assert all(not bad for _, bad, _ in res), res
     assert res[0][2] > 0, "some request must reject a draft, so the residual draw is exercised"
+
+
+class _OracleVerifier:
+    """Stands in for a rank's CUDA verifier on CPU: Verifier.rejection with
+    the oracle computing the request slice (keyed by the global request
+    index, as specdec_verify_rejection_slice is)."""
+
+    def rejection(self, target, q, drafts, temperature, seed, offset=0, request_base=0):
+        import oracle
+        al, out, pd, _ = oracle.verify_rejection(target.numpy(), "f32", q.numpy(), drafts.numpy(), temperature, seed,
+                                                 offset, request_base=request_base)
+        return torch.from_numpy(al), torch.from_numpy(out), torch.from_numpy(pd.astype(np.float32))
+
+
+def _request_rejection_worker(rank, world, port, result_q):
+    """Request-sharded rejection through sharding.py: every rank verifies its
+    request range with the global request index, and the gathered results
+    must equal one unsharded call exactly (same uniforms, same arithmetic)."""
+    import torch.distributed as dist
+    import gen
+    import oracle
+    from speculative_decoding_draft_decode_b200.sharding import sharded_verify_rejection_requests
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        r = gen.rejection_qwen(seed=6, B=11, k=3, V=900, temperature=1.0)
+        al, out, pd = sharded_verify_rejection_requests(_OracleVerifier(), torch.from_numpy(r.target),
+                                                        torch.from_numpy(r.q), torch.from_numpy(r.drafts),
+                                                        r.temperature, r.seed, r.offset)
+        ral, rout, rpd, _ = oracle.verify_rejection(r.target, r.dtype, r.q, r.drafts, r.temperature, r.seed,
+                                                    r.offset)
+        ok = (np.array_equal(al.numpy(), ral) and np.array_equal(out.numpy(), rout)
+              and np.array_equal(pd.numpy(), rpd.astype(np.float32)))
+        result_q.put((rank, ok, int((ral < r.k).sum())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_request_sharded_rejection_matches_unsharded_gloo(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_request_rejection_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+    assert all(p.exitcode == 0 for p in procs)
+    assert all(ok for _, ok, _ in res), res
+    assert res[0][2] > 0, "some request must reject a draft"
