@@ -532,6 +532,127 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
+def run_vocab_shard(args):
+    """Vocabulary-sharded greedy verification (Arctic page, "Speculator
+    optimisation": each GPU holds a column slice of every logit row, takes its
+    TopK, the results are all-gathered and the global TopK taken from them):
+    one step = this rank's streaming pass over its columns, the all-gather of
+    the row keys (NCCL over NVLink), and the combine with the accept scan.
+    Every step verifies the one batch across all ranks (strong scaling).
+    Launched eagerly on one stream per rank; also times the rank-local
+    kernels alone."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import speculative_decoding_draft_decode_b200 as sd
+    from speculative_decoding_draft_decode_b200 import build as sd_build
+    from speculative_decoding_draft_decode_b200.sharding import vocab_range
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    if rank == 0 or world == 1:
+        sd_build.build()
+    if world > 1:
+        dist.barrier()
+    inp = make_workload(args.workload)  # the same batch on every rank
+    if not isinstance(inp, gen.GreedyInputs):
+        raise SystemExit("--shard vocab times greedy workloads only")
+    B, k, V, topk = inp.B, inp.k, inp.V, inp.topk
+    R = B * (k + 1)
+    v0, v1 = vocab_range(V, world, rank)
+    full = host_tensors(inp)
+    shard = full["logits"][:, :, v0:v1].contiguous()
+    es = shard.element_size()
+    shard_bytes = shard.numel() * es
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    n_sets = max(2, math.ceil(4 * l2 / shard_bytes) + 1) if args.sets is None else args.sets
+    sets = [shard.to(device) for _ in range(n_sets)]  # same values, separate memory
+    drafts = full["drafts"].to(device)
+    ver = sd.Verifier(device)
+    kk = 8 if topk else 1
+    keys = torch.empty(R, kk, dtype=torch.int64, device=device)
+    vals = torch.empty(R, 8, dtype=torch.float32, device=device) if topk else None
+    gk = torch.empty(world, R, kk, dtype=torch.int64, device=device)
+    gv = torch.empty(world, R, 8, dtype=torch.float32, device=device) if topk else None
+    outs = (torch.empty(B, dtype=torch.int32, device=device), torch.empty(B, k + 1, dtype=torch.int32, device=device),
+            torch.empty(B, k + 1, max(topk, 1), dtype=torch.int32, device=device),
+            torch.empty(B, k + 1, max(topk, 1), dtype=torch.float32, device=device))
+    torch.cuda.synchronize(device)
+
+    def step(i, exchange=True):
+        ver.shard_greedy_rows(sets[i % n_sets], v0, topk, out=(keys, vals))
+        if exchange and world > 1:
+            dist.all_gather_into_tensor(gk, keys)
+            if topk:
+                dist.all_gather_into_tensor(gv, vals)
+        else:
+            gk[rank].copy_(keys)
+            if topk:
+                gv[rank].copy_(vals)
+        ver.shard_greedy_combine(gk, gv, drafts, V, topk, out=outs)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(exchange):
+        for i in range(args.warmup):
+            step(i, exchange)
+        ms = []
+        for _ in range(args.intervals):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(device)
+            ev0.record()
+            for i in range(args.steps):
+                step(i, exchange)
+            ev1.record()
+            torch.cuda.synchronize(device)
+            ms.append(ev0.elapsed_time(ev1))
+        med, lo, hi = dist_max([statistics.median(ms), min(ms), max(ms)], device, world)
+        return med / args.steps, lo / args.steps, hi / args.steps
+
+    sampler = ClockSampler(local, args.clock_log_dir)
+    sampler.start()
+    ms_step, ms_lo, ms_hi = timed(True)
+    clocks = sampler.stop()
+    local_ms = timed(False)
+    peak, peak_kind = measured_peak()
+    alg_local = shard_bytes + R * kk * 8 + (R * 32 if topk else 0)  # this rank's columns, its row keys and values
+    achieved_local = alg_local / (local_ms[0] / 1e3) / 1e9
+    xbytes = (world - 1) * R * (kk * 8 + (32 if topk else 0))  # what one rank receives per step
+    line = {
+        "metric": METRIC, "value": R / (ms_step / 1e3), "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": inp.dtype, "data": "synthetic",
+        "config": dict(workload=args.workload, **describe(inp), l2=L2_POLICY,
+                       parallelism="vocabulary split over %d ranks (one all-gather of row keys per step)" % world),
+        "intervals": {"n": args.intervals, "steps_each": args.steps, "ms_per_step_median": ms_step,
+                      "ms_per_step_min": ms_lo, "ms_per_step_max": ms_hi},
+        "rank_local": {"ms_per_step": local_ms[0], "ms_per_step_min": local_ms[1], "ms_per_step_max": local_ms[2],
+                       "note": "streaming pass over this rank's columns, row keys and combine, without the all-gather",
+                       "achieved_gbs": achieved_local, "frac": achieved_local / peak,
+                       "algorithmic_bytes_per_rank": alg_local},
+        "exchange": {"bytes_received_per_rank_per_step": xbytes,
+                     "ms_per_step": max(0.0, ms_step - local_ms[0]),
+                     "note": "all-gather time = step time minus rank-local time"},
+        "roofline": {"bound": "hbm", "achieved": achieved_local, "peak": peak, "unit": "GB/s",
+                     "frac": achieved_local / peak, "traffic": None,
+                     "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" % peak_kind,
+                     "note": "rank-local kernels: this rank's column bytes over their time"},
+        "gpu_launches": args.intervals * args.steps * 3, "clocks": clocks,
+        "timing": {"input_sets": n_sets, "launch": "eager C-ABI calls and NCCL all-gathers on one stream"},
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_e2e(inp, ver, device, stream, steps):
     """Public API end to end: pinned host inputs -> device, verify, result -> host."""
     import torch
@@ -709,6 +830,9 @@ def parse_args(argv=None):
     ap.add_argument("--clock-probe-seconds", type=float, default=1.0,
                     help="untimed burst of the same steps while nvidia-smi samples clocks")
     ap.add_argument("--launch-timeout", type=int, default=1800, help="seconds for ranks started by --gpus N")
+    ap.add_argument("--shard", choices=["requests", "vocab"], default="requests",
+                    help="requests: every rank verifies its own batch (default); vocab: one batch with its "
+                         "vocabulary split over the ranks (greedy workloads)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -731,7 +855,10 @@ def main():
         return 0
     if os.environ.get("WORLD_SIZE") is None and (args.gpus or 1) > 1:
         return relaunch_under_torchrun(args)
-    run_ours(args)
+    if args.shard == "vocab":
+        run_vocab_shard(args)
+    else:
+        run_ours(args)
     return 0
 
 

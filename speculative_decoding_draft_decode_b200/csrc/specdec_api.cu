@@ -5,6 +5,9 @@
 // starts sit at a fixed place, so a workspace initialised once serves calls
 // of any shape; each call returns those words to zero before it ends.
 //   [0, 256 KiB)            top-8 thresholds, one word per row (first 65536 rows)
+//   then                    control words of the fused rejection kernel
+//                           (index counter, error word, per-request counters
+//                           and flags for up to kFusedMaxB requests)
 //   then                    streaming-pass partials, one slot per chunk
 //   then (rejection only)   per-request RejState, per-chunk and per-unit masses
 //                           of row h
@@ -20,12 +23,14 @@
 #include "verify_resample.cuh"
 #include "verify_stats.cuh"
 #include "verify_ngram.cuh"
+#include "verify_fused.cuh"
 
 namespace specdec {
 namespace {
 
 constexpr size_t kThetaBase = 0;
-constexpr size_t kPartialBase = kThetaBase + static_cast<size_t>(kThetaRows) * sizeof(unsigned);
+constexpr size_t kCtlBase = kThetaBase + static_cast<size_t>(kThetaRows) * sizeof(unsigned);
+constexpr size_t kPartialBase = (kCtlBase + kCtlWords * sizeof(unsigned) + 255) / 256 * 256;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -75,6 +80,16 @@ constexpr int kMaxDevices = 64;
 // specdec_set_prefetch_inputs: whether the argmax streaming pass may read its
 // rows before the previous kernel of the stream has finished.
 std::atomic<int> g_prefetch_inputs{0};
+
+// specdec_set_rejection_fused: fixed-layout rejection calls of up to
+// kFusedMaxB requests run as the one fused kernel (1) or as the four kernels
+// (0).
+std::atomic<int> g_rejection_fused{1};
+
+// Clock cycles a CTA of the fused rejection kernel waits for a request's
+// decision before it gives up (about a second at B200 clocks; a decision
+// normally comes within microseconds).
+constexpr long long kWaitBudgetCycles = 2000000000LL;
 
 bool vector_path_ok(const void* p, int64_t stride, int esize) {
     return (reinterpret_cast<uintptr_t>(p) % 16 == 0) && ((stride * esize) % 16 == 0);
@@ -306,8 +321,14 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     P.req_base = req_base;
     const bool stats = entropy != nullptr && offsets == nullptr && k > 0;
     P.row_stat = stats ? reinterpret_cast<RowStat*>(static_cast<char*>(ws) + L.row_stat) : nullptr;
-    st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
-    if (st != SPECDEC_OK) return st;
+    const uint64_t n_pass1 = static_cast<uint64_t>(L.NC);
+    const uint64_t n_total = n_pass1 + static_cast<uint64_t>(B) * static_cast<uint64_t>(L.cpr2);
+    const bool fused = g_rejection_fused.load(std::memory_order_relaxed) != 0 && offsets == nullptr && !stats &&
+                       B <= kFusedMaxB && n_total < 0x7fffffffull;
+    if (!fused) {
+        st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
+        if (st != SPECDEC_OK) return st;
+    }
     Pass2Params Q;
     memset(&Q, 0, sizeof(Q));
     Q.logits = target_logits;
@@ -328,6 +349,32 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     Q.chunk_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.masses);
     Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
     Q.out_tokens = out_tokens;
+    if (fused) {
+        FusedParams F;
+        memset(&F, 0, sizeof(F));
+        F.p1 = P;
+        F.p1.prefetch_inputs = 0;  // the kernel waits for the previous one before its first access
+        F.p2 = Q;
+        unsigned* ctl = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kCtlBase);
+        F.next = ctl;
+        F.error = ctl + 1;
+        F.req_ticket = ctl + kCtlHeadWords;
+        F.decided = F.req_ticket + kFusedMaxB;
+        F.res_ticket = F.decided + kFusedMaxB;
+        F.n_pass1 = static_cast<unsigned>(n_pass1);
+        F.n_total = static_cast<unsigned>(n_total);
+        F.wait_budget = kWaitBudgetCycles;
+        const dim3 grid(static_cast<unsigned>(n_total));
+        cudaError_t e;
+        if (dtype == SPECDEC_BF16)
+            e = vec ? launch_pdl(verify_rejection_fused_kernel<BF16Tag, 8>, grid, 0, s, F)
+                    : launch_pdl(verify_rejection_fused_kernel<BF16Tag, 1>, grid, 0, s, F);
+        else
+            e = vec ? launch_pdl(verify_rejection_fused_kernel<F32Tag, 4>, grid, 0, s, F)
+                    : launch_pdl(verify_rejection_fused_kernel<F32Tag, 1>, grid, 0, s, F);
+        if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
+        return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+    }
     st = dispatch_pass2(dtype, vec, Q, s);
     if (st != SPECDEC_OK || !stats) return st;
     StatsParams S;
@@ -905,6 +952,36 @@ specdec_status specdec_ngram_propose(const int32_t* tokens, int64_t token_stride
 }
 
 int specdec_set_prefetch_inputs(int enable) { return g_prefetch_inputs.exchange(enable ? 1 : 0); }
+
+int specdec_set_rejection_fused(int enable) { return g_rejection_fused.exchange(enable ? 1 : 0); }
+
+specdec_status specdec_workspace_check(const void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+    if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % 16 != 0 || ws_bytes < kPartialBase)
+        return SPECDEC_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SPECDEC_ERR_CUDA;
+    unsigned err = 0;
+    if (cudaMemcpy(&err, static_cast<const char*>(ws) + kCtlBase + sizeof(unsigned), sizeof(err),
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SPECDEC_ERR_CUDA;
+    return err != 0u ? SPECDEC_ERR_TIMEOUT : SPECDEC_OK;
+}
+
+specdec_status specdec_selftest_wait_timeout(void* ws, size_t ws_bytes, long long budget_cycles,
+                                             struct CUstream_st* stream) {
+    if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % 16 != 0 || ws_bytes < kPartialBase)
+        return SPECDEC_ERR_WORKSPACE;
+    if (budget_cycles < 1 || budget_cycles > kWaitBudgetCycles) return SPECDEC_ERR_INVALID_ARG;
+    unsigned* ctl = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kCtlBase);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(32);
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaLaunchKernelEx(&cfg, verify_wait_selftest_kernel, static_cast<const unsigned*>(ctl + 2), ctl + 1,
+                           budget_cycles) != cudaSuccess)
+        return SPECDEC_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+}
 
 double specdec_tier_update(specdec_tier_state* state, double accepted, double decay) {
     if (state == nullptr || !(decay >= 0.0 && decay < 1.0) || !(accepted >= 0.0 && accepted <= SPECDEC_MAX_K))
