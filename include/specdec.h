@@ -470,8 +470,18 @@ int specdec_set_prefetch_inputs(int enable);
  * enqueued. */
 int specdec_set_rejection_fused(int enable);
 
+/* How the argmax and top-8 streaming passes (greedy, top-8, tree) read their
+ * chunks on the 16-byte vector path (process-wide; returns the previous
+ * setting; default 0): 0 = each thread loads its vectors into registers, a
+ * batch at a time; 1 = one thread of each CTA hands the chunk to the
+ * bulk-copy engine (1-D cp.async.bulk copies into the CTA's shared memory,
+ * one mbarrier per 8 KB piece) and the warps reduce the pieces as they land.
+ * Results are identical.  The setting is read when a call is enqueued. */
+int specdec_set_stream_bulk(int enable);
+
 /* Synchronises `stream`, then reads the workspace's error word: SPECDEC_OK,
- * or SPECDEC_ERR_TIMEOUT when a wait of the fused rejection kernel gave up
+ * or SPECDEC_ERR_TIMEOUT when a wait of the fused rejection kernel (or of a
+ * bulk-copy streaming pass for its copies) gave up
  * since the workspace was last initialised (the results of that call are
  * undefined, and the workspace must be initialised again with
  * specdec_workspace_init before its next use).  SPECDEC_ERR_WORKSPACE for a

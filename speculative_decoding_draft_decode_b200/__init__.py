@@ -128,6 +128,8 @@ def lib():
             getattr(L, f).restype = i32
         L.specdec_set_prefetch_inputs.argtypes = [i32]
         L.specdec_set_prefetch_inputs.restype = i32
+        L.specdec_set_stream_bulk.argtypes = [i32]
+        L.specdec_set_stream_bulk.restype = i32
         L.specdec_set_rejection_fused.argtypes = [i32]
         L.specdec_set_rejection_fused.restype = i32
         L.specdec_workspace_check.argtypes = [P, sz, P]
@@ -331,11 +333,18 @@ def specdec_set_prefetch_inputs(enable: bool) -> bool:
     return bool(lib().specdec_set_prefetch_inputs(1 if enable else 0))
 
 
-def specdec_set_rejection_fused(enable: bool) -> bool:
+def specdec_set_rejection_fused(enable) -> int:
     """Process-wide: fixed-layout rejection calls of up to 8192 requests run as
     the one request-by-request kernel (default) or as four kernels.  Returns
     the previous setting."""
-    return bool(lib().specdec_set_rejection_fused(1 if enable else 0))
+    return lib().specdec_set_rejection_fused(int(enable))
+
+
+def specdec_set_stream_bulk(enable: bool) -> bool:
+    """Process-wide: the argmax and top-8 streaming passes stage each chunk in
+    shared memory with bulk copies (True) or load into registers (False,
+    default).  Returns the previous setting."""
+    return bool(lib().specdec_set_stream_bulk(1 if enable else 0))
 
 
 def specdec_workspace_check(ws, nbytes: int, stream=None) -> int:

@@ -24,6 +24,7 @@
 #include "verify_stats.cuh"
 #include "verify_ngram.cuh"
 #include "verify_fused.cuh"
+#include "verify_bulk.cuh"
 
 namespace specdec {
 namespace {
@@ -81,6 +82,10 @@ constexpr int kMaxDevices = 64;
 // rows before the previous kernel of the stream has finished.
 std::atomic<int> g_prefetch_inputs{0};
 
+// specdec_set_stream_bulk: the argmax and top-8 streaming passes stage their
+// chunks in shared memory with bulk copies (1) or load into registers (0).
+std::atomic<int> g_stream_bulk{0};
+
 // specdec_set_rejection_fused: fixed-layout rejection calls of up to
 // kFusedMaxB requests run as the one fused kernel (1) or as the four kernels
 // (0).
@@ -98,6 +103,18 @@ bool vector_path_ok(const void* p, int64_t stride, int esize) {
 bool rows_fit(int64_t rows, int64_t row_stride, int V) {
     // Every element offset must fit comfortably in 63 bits.
     return row_stride >= V && row_stride <= (int64_t(1) << 40) && rows * row_stride < (int64_t(1) << 52);
+}
+
+// CTAs of a persistent kernel: as many as the current device keeps resident.
+template <class Kernel>
+cudaError_t persistent_ctas(Kernel fn, unsigned* out) {
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NT, 0);
+    if (e != cudaSuccess) return e;
+    *out = static_cast<unsigned>((per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1));
+    return cudaSuccess;
 }
 
 // Launch with programmatic stream serialisation: the kernel may be scheduled
@@ -118,6 +135,30 @@ cudaError_t launch_pdl(Kernel fn, dim3 grid, int dyn, cudaStream_t stream, const
     return cudaLaunchKernelEx(&cfg, fn, P);
 }
 
+// The bulk-copy streaming kernel of a mode: its shared-memory ring (the
+// chunk) exceeds the default 48 KB for top-8, so the limit is raised once per
+// device.
+template <class Tag, int VEC, int MODE>
+cudaError_t launch_bulk_pass(const Pass1Params& P, dim3 grid, cudaStream_t stream) {
+    constexpr int CH = chunk_vecs(VEC, mode_u(MODE));
+    constexpr int kBytes = CH * 16;
+    static std::atomic<unsigned long long> ready{0};  // bit d: device d set up
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(ready.load(std::memory_order_acquire) & bit)) {
+        e = cudaFuncSetAttribute(verify_pass1_bulk_kernel<Tag, VEC, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(verify_pass1_bulk_kernel<Tag, VEC, MODE>,
+                                     cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
+        ready.fetch_or(bit, std::memory_order_release);
+    }
+    return launch_pdl(verify_pass1_bulk_kernel<Tag, VEC, MODE>, grid, kBytes, stream, P);
+}
+
 // The streaming pass (one CTA per chunk; trees stream like greedy argmax),
 // then the request epilogues (one CTA per request).
 template <class Tag, int VEC, int MODE>
@@ -125,8 +166,15 @@ specdec_status launch_pass1(Pass1Params P, cudaStream_t stream) {
     constexpr int STREAM_MODE = MODE == MODE_TREE ? MODE_ARGMAX : MODE;
     if (P.R > 0x7fffffff || P.cpr > 65535) return SPECDEC_ERR_UNSUPPORTED;  // grid limits
     const dim3 grid(static_cast<unsigned>(P.R), static_cast<unsigned>(P.cpr));
-    if (launch_pdl(verify_pass1_kernel<Tag, VEC, STREAM_MODE>, grid, 0, stream, P) != cudaSuccess)
-        return SPECDEC_ERR_CUDA;
+    cudaError_t e;
+    if constexpr (VEC > 1 && STREAM_MODE != MODE_SOFTMAX) {
+        e = g_stream_bulk.load(std::memory_order_relaxed) ? launch_bulk_pass<Tag, VEC, STREAM_MODE>(P, grid, stream)
+                                                           : launch_pdl(verify_pass1_kernel<Tag, VEC, STREAM_MODE>,
+                                                                        grid, 0, stream, P);
+    } else {
+        e = launch_pdl(verify_pass1_kernel<Tag, VEC, STREAM_MODE>, grid, 0, stream, P);
+    }
+    if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
     if constexpr (MODE == MODE_TOP8) {
         const int rows = P.k + 1 < kTop8EpiWarps ? P.k + 1 : kTop8EpiWarps;  // a warp per row
         if (launch_pdl(verify_top8_epilogue_kernel<Tag>, dim3(static_cast<unsigned>(P.B)), 0, stream, P, 32 * rows) !=
@@ -186,11 +234,11 @@ specdec_status dispatch_stats(specdec_dtype dt, bool vec, StatsParams S, cudaStr
 
 bool dtype_ok(specdec_dtype dt) { return dt == SPECDEC_F32 || dt == SPECDEC_BF16; }
 
-// Pass-1 partial bytes per chunk: one argmax key per warp, 8 keys per warp
-// (top-8), or one (max, sum) pair per warp (softmax).
-constexpr size_t kArgmaxChunkBytes = NWARPS * sizeof(uint64_t);
-constexpr size_t kTop8ChunkBytes = NWARPS * 8 * sizeof(uint64_t);
-constexpr size_t kSoftmaxChunkBytes = NWARPS * sizeof(SoftmaxPartial);
+// Pass-1 partial bytes per chunk: one argmax key, 8 keys (top-8), or one
+// (max, sum) pair (softmax).
+constexpr size_t kArgmaxChunkBytes = kPartsPerChunk * sizeof(uint64_t);
+constexpr size_t kTop8ChunkBytes = kPartsPerChunk * 8 * sizeof(uint64_t);
+constexpr size_t kSoftmaxChunkBytes = kPartsPerChunk * sizeof(SoftmaxPartial);
 size_t slot_bytes(specdec_mode mode) {
     if (mode == SPECDEC_MODE_GREEDY) return kArgmaxChunkBytes > kTop8ChunkBytes ? kArgmaxChunkBytes : kTop8ChunkBytes;
     if (mode == SPECDEC_MODE_REJECTION) return kSoftmaxChunkBytes;
@@ -218,6 +266,7 @@ void fill_common(Pass1Params& P, const void* logits, int64_t row_stride, int V, 
     P.rows_per_req = rows_per_req;
     P.B = B;
     P.theta_row = reinterpret_cast<unsigned*>(base + kThetaBase);
+    P.bulk_error = reinterpret_cast<unsigned*>(base + kCtlBase) + 1;
     P.partials = base + L.partials1;
 }
 
@@ -323,8 +372,10 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     P.row_stat = stats ? reinterpret_cast<RowStat*>(static_cast<char*>(ws) + L.row_stat) : nullptr;
     const uint64_t n_pass1 = static_cast<uint64_t>(L.NC);
     const uint64_t n_total = n_pass1 + static_cast<uint64_t>(B) * static_cast<uint64_t>(L.cpr2);
-    const bool fused = g_rejection_fused.load(std::memory_order_relaxed) != 0 && offsets == nullptr && !stats &&
-                       B <= kFusedMaxB && n_total < 0x7fffffffull;
+    const int fused_mode = g_rejection_fused.load(std::memory_order_relaxed);
+    const uint64_t n_total_p = n_pass1 + 2ull * static_cast<uint64_t>(B) + static_cast<uint64_t>(B) * L.cpr2;
+    const bool fused = fused_mode != 0 && offsets == nullptr && !stats && B <= kFusedMaxB &&
+                       n_total_p < 0x7fffffffull;
     if (!fused) {
         st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
         if (st != SPECDEC_OK) return st;
@@ -362,16 +413,36 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
         F.decided = F.req_ticket + kFusedMaxB;
         F.res_ticket = F.decided + kFusedMaxB;
         F.n_pass1 = static_cast<unsigned>(n_pass1);
-        F.n_total = static_cast<unsigned>(n_total);
         F.wait_budget = kWaitBudgetCycles;
-        const dim3 grid(static_cast<unsigned>(n_total));
+        F.exits = ctl + 3;
         cudaError_t e;
-        if (dtype == SPECDEC_BF16)
-            e = vec ? launch_pdl(verify_rejection_fused_kernel<BF16Tag, 8>, grid, 0, s, F)
-                    : launch_pdl(verify_rejection_fused_kernel<BF16Tag, 1>, grid, 0, s, F);
-        else
-            e = vec ? launch_pdl(verify_rejection_fused_kernel<F32Tag, 4>, grid, 0, s, F)
-                    : launch_pdl(verify_rejection_fused_kernel<F32Tag, 1>, grid, 0, s, F);
+        if (fused_mode == 2) {
+            F.n_total = static_cast<unsigned>(n_total_p);
+            unsigned ctas = 0;
+            if (dtype == SPECDEC_BF16)
+                e = vec ? persistent_ctas(verify_rejection_persistent_kernel<BF16Tag, 8>, &ctas)
+                        : persistent_ctas(verify_rejection_persistent_kernel<BF16Tag, 1>, &ctas);
+            else
+                e = vec ? persistent_ctas(verify_rejection_persistent_kernel<F32Tag, 4>, &ctas)
+                        : persistent_ctas(verify_rejection_persistent_kernel<F32Tag, 1>, &ctas);
+            if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
+            const dim3 grid(ctas < F.n_total ? ctas : F.n_total);
+            if (dtype == SPECDEC_BF16)
+                e = vec ? launch_pdl(verify_rejection_persistent_kernel<BF16Tag, 8>, grid, 0, s, F)
+                        : launch_pdl(verify_rejection_persistent_kernel<BF16Tag, 1>, grid, 0, s, F);
+            else
+                e = vec ? launch_pdl(verify_rejection_persistent_kernel<F32Tag, 4>, grid, 0, s, F)
+                        : launch_pdl(verify_rejection_persistent_kernel<F32Tag, 1>, grid, 0, s, F);
+        } else {
+            F.n_total = static_cast<unsigned>(n_total);
+            const dim3 grid(static_cast<unsigned>(n_total));
+            if (dtype == SPECDEC_BF16)
+                e = vec ? launch_pdl(verify_rejection_fused_kernel<BF16Tag, 8>, grid, 0, s, F)
+                        : launch_pdl(verify_rejection_fused_kernel<BF16Tag, 1>, grid, 0, s, F);
+            else
+                e = vec ? launch_pdl(verify_rejection_fused_kernel<F32Tag, 4>, grid, 0, s, F)
+                        : launch_pdl(verify_rejection_fused_kernel<F32Tag, 1>, grid, 0, s, F);
+        }
         if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
         return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
     }
@@ -953,7 +1024,9 @@ specdec_status specdec_ngram_propose(const int32_t* tokens, int64_t token_stride
 
 int specdec_set_prefetch_inputs(int enable) { return g_prefetch_inputs.exchange(enable ? 1 : 0); }
 
-int specdec_set_rejection_fused(int enable) { return g_rejection_fused.exchange(enable ? 1 : 0); }
+int specdec_set_stream_bulk(int enable) { return g_stream_bulk.exchange(enable ? 1 : 0); }
+
+int specdec_set_rejection_fused(int enable) { return g_rejection_fused.exchange(enable < 0 || enable > 2 ? 1 : enable); }
 
 specdec_status specdec_workspace_check(const void* ws, size_t ws_bytes, struct CUstream_st* stream) {
     if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % 16 != 0 || ws_bytes < kPartialBase)

@@ -56,6 +56,7 @@ constexpr int kFusedMaxB = 8192;
 //   word 1           error word (1: a wait gave up; 2: the index counter was
 //                    not zero when a call started)
 //   word 2           a flag nothing sets (the wait self-test)
+//   word 3           CTAs of the persistent kernel that have finished
 //   [64, +B)         pass-1 chunks finished per request
 //   [.., +B)         decision published per request
 //   [.., +B)         resample chunks finished per request
@@ -71,8 +72,9 @@ struct FusedParams {
     unsigned* decided;     // [kFusedMaxB]
     unsigned* res_ticket;  // [kFusedMaxB]
     unsigned n_pass1;      // R * cpr
-    unsigned n_total;      // n_pass1 + B * cpr2
+    unsigned n_total;      // n_pass1 + B * cpr2 (one item per CTA); n_pass1 + B + B * cpr2 + B (persistent)
     long long wait_budget;  // clock64 cycles a CTA waits for a decision
+    unsigned* exits;       // persistent kernel: CTAs that have drawn past the end
 };
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
@@ -194,6 +196,131 @@ __global__ void __launch_bounds__(NT, SPECDEC_MINB_FUSED) verify_rejection_fused
     if (s_last && ok && threadIdx.x < 32) {
         __threadfence();
         token_search<Tag, VEC>(Q, load_state_cg(Q.state + b), b);
+    }
+}
+
+__device__ __forceinline__ void red_release_add_u32(unsigned* p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Waits until *word == want (one thread), bounded as wait_flag_bounded.
+__device__ __noinline__ bool wait_count_bounded(const unsigned* word, unsigned want, long long budget,
+                                                unsigned* error) {
+    if (ld_acquire_u32(word) == want) return true;
+    const long long t0 = clock64();
+    unsigned ns = 32;
+    while (ld_acquire_u32(word) != want) {
+        if (clock64() - t0 > budget) {
+            atomicOr(error, 1u);
+            return false;
+        }
+        __nanosleep(ns);
+        if (ns < 256) ns <<= 1;
+    }
+    return true;
+}
+
+// The same dataflow on a persistent grid (as many CTAs as are resident):
+// each CTA draws its next index while it works on the current one, and the
+// per-request steps are items of their own, so a streaming item never waits
+// for an atomic's answer:
+//   [0, nA)                      softmax chunk; then a release add to its
+//                                request's chunk count
+//   [nA, nA + B)                 decision of request b, once its count is
+//                                (k + 1) cpr; then a release store of its flag
+//   [nA + B, nA + B + B cpr2)    resample chunk of row h, once the flag is up;
+//                                then a release add to the request's count
+//   [.., + B)                    token of request b, once that count is cpr2;
+//                                returns the request's words to zero
+// Every item waits only on items with smaller indices, and a CTA holds at
+// most its current index and the next one, so the waits end.
+template <class Tag, int VEC>
+__global__ void __launch_bounds__(NT, SPECDEC_MINB_FUSED) verify_rejection_persistent_kernel(const FusedParams F) {
+    __shared__ Pass1Smem sm;
+    __shared__ double red2[2][NWARPS];
+    __shared__ unsigned s_next, s_ok;
+    using Elem = typename Tag::storage;
+    constexpr int CH = chunk_vecs(VEC, kU);
+    constexpr int UPT = CH / NT;
+    const Pass1Params& P = F.p1;
+    const Pass2Params& Q = F.p2;
+    const unsigned nA = F.n_pass1, B = static_cast<unsigned>(P.B), cpr2 = static_cast<unsigned>(Q.cpr);
+    const unsigned nD = nA + B, nM = nD + B * cpr2;
+
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    if (threadIdx.x == 0) s_next = atomicAdd(F.next, 1u);
+    __syncthreads();
+    unsigned item = s_next;
+    __syncthreads();
+    while (item < F.n_total) {
+        unsigned nxt = 0u;
+        if (threadIdx.x == 0) nxt = atomicAdd(F.next, 1u);  // answered while this item runs
+        if (item < nA) {
+            const int64_t r = item / static_cast<unsigned>(P.cpr);
+            const int sub = static_cast<int>(item % static_cast<unsigned>(P.cpr));
+            int cnt = P.nv_full - sub * CH;
+            cnt = cnt < CH ? cnt : CH;
+            const Elem* row = static_cast<const Elem*>(P.logits) + r * P.row_stride;
+            softmax_chunk<Tag, VEC, CH, UPT>(P, row, r, sub, cnt, sm);  // thread 0 stores the chunk's partial
+            if (threadIdx.x == 0) red_release_add_u32(&F.req_ticket[r / P.rows_per_req], 1u);
+        } else if (item < nD) {
+            const int64_t b = item - nA;
+            if (threadIdx.x == 0)
+                s_ok = wait_count_bounded(&F.req_ticket[b], static_cast<unsigned>(P.rows_per_req * P.cpr),
+                                          F.wait_budget, F.error) ? 1u : 0u;
+            __syncthreads();
+            if (s_ok) {
+                __threadfence();
+                epilogue_rejection<Tag>(P, b, sm);  // reads the partials through L2
+                __threadfence();                    // the decision's stores, before the flag
+                __syncthreads();
+                if (threadIdx.x == 0) {
+                    F.req_ticket[b] = 0u;
+                    st_release_u32(&F.decided[b], 1u);
+                }
+            }
+        } else if (item < nM) {
+            const unsigned j = item - nD;
+            const int64_t b = j / cpr2;
+            const int sub = static_cast<int>(j % cpr2);
+            if (threadIdx.x == 0) s_ok = wait_flag_bounded(&F.decided[b], F.wait_budget, F.error) ? 1u : 0u;
+            __syncthreads();
+            if (s_ok) {
+                __threadfence();
+                const RejState st = load_state_cg(Q.state + b);
+                if (st.valid) resample_chunk<Tag, VEC>(Q, st, b, sub, red2);  // CTA-uniform
+            }
+            __threadfence();  // the chunk's mass stores, before the count
+            __syncthreads();
+            if (threadIdx.x == 0) red_release_add_u32(&F.res_ticket[b], 1u);
+        } else {
+            const int64_t b = item - nM;
+            if (threadIdx.x == 0) s_ok = wait_count_bounded(&F.res_ticket[b], cpr2, F.wait_budget, F.error) ? 1u : 0u;
+            __syncthreads();
+            if (s_ok && threadIdx.x < 32) {
+                __threadfence();
+                const RejState st = load_state_cg(Q.state + b);
+                if (ld_acquire_u32(&F.decided[b]) != 0u) token_search<Tag, VEC>(Q, st, b);
+            }
+            __syncthreads();
+            if (threadIdx.x == 0 && s_ok) {  // every resample chunk of b has read the flag
+                F.res_ticket[b] = 0u;
+                F.decided[b] = 0u;
+            }
+        }
+        if (threadIdx.x == 0) s_next = nxt;
+        __syncthreads();
+        item = s_next;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const unsigned e = atomicAdd(F.exits, 1u);
+        if (e == gridDim.x - 1u) {  // every CTA has drawn past the end
+            *F.next = 0u;
+            *F.exits = 0u;
+        }
     }
 }
 
