@@ -529,7 +529,9 @@ struct SoftmaxReducer {
             float Mc = mw;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(FULL_MASK, Mc, o));
-            double t = sw > 0.0 ? sw * exp((static_cast<double>(mw) - static_cast<double>(Mc)) * invT_d) : 0.0;
+            // A part with no mass adds nothing; NaN (a NaN or +inf logit) carries
+            // through, so the row is found undefined, as in maxsum_merge.
+            double t = sw != 0.0 ? sw * exp((static_cast<double>(mw) - static_cast<double>(Mc)) * invT_d) : 0.0;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(FULL_MASK, t, o);
             if (lane == 0) {

@@ -1,4 +1,4 @@
-"""The request-by-request rejection kernel (specdec_set_rejection_fused):
+"""The request-by-request rejection kernel (specdec_set_rejection_fused, one work item per CTA or a persistent grid):
 results identical, bit for bit, to the four-kernel path on the same inputs
 (which the other rejection tests hold against the oracle), across shapes,
 dtypes, the scalar path, invalid rows and out-of-range drafts, back-to-back
@@ -26,22 +26,23 @@ def both_paths(ver, r, offset=0, x=None, q=None, d=None):
     q = dev_f32(r.q) if q is None else q
     d = dev_i32(r.drafts) if d is None else d
     res = {}
-    for fused in (True, False):
+    for fused in (1, 0, 2):
         prev = sd.specdec_set_rejection_fused(fused)
         try:
             res[fused] = [host(t) for t in ver.rejection(x, q, d, r.temperature, r.seed, offset)]
         finally:
             sd.specdec_set_rejection_fused(prev)
-    for a, b in zip(res[True], res[False]):
-        if a.dtype == np.float32:
-            a, b = a.view(np.uint32), b.view(np.uint32)
-        assert np.array_equal(a, b)
-    return res[True]
+    for mode in (0, 2):
+        for a, b in zip(res[1], res[mode]):
+            if a.dtype == np.float32:
+                a, b = a.view(np.uint32), b.view(np.uint32)
+            assert np.array_equal(a, b), mode
+    return res[1]
 
 
 def test_fused_is_the_default():
     require_cuda()
-    assert sd.specdec_set_rejection_fused(True) is True
+    assert sd.specdec_set_rejection_fused(1) == 1
 
 
 def test_fused_equals_four_kernels_qwen(V_):
@@ -83,13 +84,26 @@ def test_fused_scalar_path_and_strides(V_):
     both_paths(V_, r, x=x)
 
 
-def test_fused_back_to_back_and_graph_replay(V_):
+@pytest.mark.parametrize("mode", [1, 2])
+def test_fused_back_to_back_and_graph_replay(V_, mode):
     """Counters and flags return to zero: calls of different shapes on one
-    workspace, then a replayed graph of several calls, equal single calls."""
+    workspace, then a replayed graph of several calls, equal single calls
+    (mode 1: one work item per CTA; mode 2: the persistent grid)."""
+    import torch
+    prev = sd.specdec_set_rejection_fused(mode)
+    try:
+        _back_to_back(V_)
+    finally:
+        sd.specdec_set_rejection_fused(prev)
+
+
+def _back_to_back(V_):
     import torch
     shapes = [(32, 4, 151936), (5, 1, 1000), (40, 6, 7000)]
     rs = [gen.rejection_qwen(seed=50 + i, B=B, k=k, V=V) for i, (B, k, V) in enumerate(shapes)]
+    prev = sd.specdec_set_rejection_fused(1)
     want = [both_paths(V_, r) for r in rs]
+    sd.specdec_set_rejection_fused(prev)
     ins = [(dev_logits(r.target, r.dtype), dev_f32(r.q), dev_i32(r.drafts)) for r in rs]
     outs = [(torch.empty(r.B, dtype=torch.int32, device="cuda"), torch.empty(r.B, r.k + 1, dtype=torch.int32,
                                                                             device="cuda"),
