@@ -84,7 +84,7 @@ typedef enum {
     SPECDEC_ERR_UNSUPPORTED = 2, /* dtype or mode not supported */
     SPECDEC_ERR_WORKSPACE = 3,   /* workspace null, too small or misaligned */
     SPECDEC_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
-    SPECDEC_ERR_TIMEOUT = 5      /* a wait of the fused rejection kernel gave up (specdec_workspace_check) */
+    SPECDEC_ERR_TIMEOUT = 5      /* reserved: no kernel of this version waits on another */
 } specdec_status;
 
 typedef enum { SPECDEC_F32 = 0, SPECDEC_BF16 = 1 } specdec_dtype;
@@ -453,49 +453,6 @@ const char* specdec_status_string(specdec_status status);
  * own kernels are safe.  The setting is read when a call is enqueued (and
  * baked into a captured graph). */
 int specdec_set_prefetch_inputs(int enable);
-
-/* Rejection-sampling calls in the fixed layout with at most 8192 requests
- * (specdec_verify_rejection and specdec_verify_rejection_slice) run as ONE
- * kernel that works request by request (process-wide; returns the previous
- * setting; default 1): a CTA that finishes a request's last target-row chunk
- * takes that request's accept decision, and the chunks of its row h are
- * resampled as soon as the decision is published, while later requests'
- * rows still stream.  With enable = 0 they run as four kernels (softmax
- * pass, decisions, chunk masses of row h, token search), each waiting for
- * the whole batch.  Results are identical.  The fused kernel's CTAs wait on
- * one another (each wait is for a request decided by a CTA that started
- * earlier); every wait gives up after about a second, sets the workspace's
- * error word and lets the call finish with that request's results undefined
- * (see specdec_workspace_check).  The setting is read when a call is
- * enqueued. */
-int specdec_set_rejection_fused(int enable);
-
-/* How the argmax and top-8 streaming passes (greedy, top-8, tree) read their
- * chunks on the 16-byte vector path (process-wide; returns the previous
- * setting; default 0): 0 = each thread loads its vectors into registers, a
- * batch at a time; 1 = one thread of each CTA hands the chunk to the
- * bulk-copy engine (1-D cp.async.bulk copies into the CTA's shared memory,
- * one mbarrier per 8 KB piece) and the warps reduce the pieces as they land.
- * Results are identical.  The setting is read when a call is enqueued. */
-int specdec_set_stream_bulk(int enable);
-
-/* Synchronises `stream`, then reads the workspace's error word: SPECDEC_OK,
- * or SPECDEC_ERR_TIMEOUT when a wait of the fused rejection kernel (or of a
- * bulk-copy streaming pass for its copies) gave up
- * since the workspace was last initialised (the results of that call are
- * undefined, and the workspace must be initialised again with
- * specdec_workspace_init before its next use).  SPECDEC_ERR_WORKSPACE for a
- * null, misaligned or too small workspace.  This entry point synchronises;
- * none of the verify calls do. */
-specdec_status specdec_workspace_check(const void* ws, size_t ws_bytes, struct CUstream_st* stream);
-
-/* Exercises the bounded wait of the fused rejection kernel without a fault:
- * enqueues one thread that waits on a workspace flag nothing ever sets, for
- * budget_cycles SM clock cycles (1 .. 2e9), after which the wait gives up and
- * sets the error word, exactly as a wait of the fused kernel would.  A
- * following specdec_workspace_check returns SPECDEC_ERR_TIMEOUT. */
-specdec_status specdec_selftest_wait_timeout(void* ws, size_t ws_bytes, long long budget_cycles,
-                                             struct CUstream_st* stream);
 
 /* SPECDEC_ABI_VERSION of the loaded library. */
 int specdec_abi_version(void);

@@ -128,14 +128,6 @@ def lib():
             getattr(L, f).restype = i32
         L.specdec_set_prefetch_inputs.argtypes = [i32]
         L.specdec_set_prefetch_inputs.restype = i32
-        L.specdec_set_stream_bulk.argtypes = [i32]
-        L.specdec_set_stream_bulk.restype = i32
-        L.specdec_set_rejection_fused.argtypes = [i32]
-        L.specdec_set_rejection_fused.restype = i32
-        L.specdec_workspace_check.argtypes = [P, sz, P]
-        L.specdec_workspace_check.restype = i32
-        L.specdec_selftest_wait_timeout.argtypes = [P, sz, ctypes.c_longlong, P]
-        L.specdec_selftest_wait_timeout.restype = i32
         L.specdec_tier_update.argtypes = [P, ctypes.c_double, ctypes.c_double]
         L.specdec_tier_update.restype = ctypes.c_double
         L.specdec_tier_select.argtypes = [P, i32, ctypes.c_double]
@@ -331,30 +323,6 @@ def specdec_set_prefetch_inputs(enable: bool) -> bool:
     previous kernel of the stream has finished (see the header for when that
     is safe).  Returns the previous setting."""
     return bool(lib().specdec_set_prefetch_inputs(1 if enable else 0))
-
-
-def specdec_set_rejection_fused(enable) -> int:
-    """Process-wide: fixed-layout rejection calls of up to 8192 requests run as
-    the one request-by-request kernel (default) or as four kernels.  Returns
-    the previous setting."""
-    return lib().specdec_set_rejection_fused(int(enable))
-
-
-def specdec_set_stream_bulk(enable: bool) -> bool:
-    """Process-wide: the argmax and top-8 streaming passes stage each chunk in
-    shared memory with bulk copies (True) or load into registers (False,
-    default).  Returns the previous setting."""
-    return bool(lib().specdec_set_stream_bulk(1 if enable else 0))
-
-
-def specdec_workspace_check(ws, nbytes: int, stream=None) -> int:
-    """Synchronises the stream and returns SPECDEC_ERR_TIMEOUT if a wait of
-    the fused rejection kernel gave up since the workspace was initialised."""
-    return lib().specdec_workspace_check(_ptr(ws), nbytes, _stream(stream))
-
-
-def specdec_selftest_wait_timeout(ws, nbytes: int, budget_cycles: int, stream=None) -> int:
-    return lib().specdec_selftest_wait_timeout(_ptr(ws), nbytes, int(budget_cycles), _stream(stream))
 
 
 class specdec_tier_state(ctypes.Structure):

@@ -5,9 +5,6 @@
 // starts sit at a fixed place, so a workspace initialised once serves calls
 // of any shape; each call returns those words to zero before it ends.
 //   [0, 256 KiB)            top-8 thresholds, one word per row (first 65536 rows)
-//   then                    control words of the fused rejection kernel
-//                           (index counter, error word, per-request counters
-//                           and flags for up to kFusedMaxB requests)
 //   then                    streaming-pass partials, one slot per chunk
 //   then (rejection only)   per-request RejState, per-chunk and per-unit masses
 //                           of row h
@@ -23,15 +20,12 @@
 #include "verify_resample.cuh"
 #include "verify_stats.cuh"
 #include "verify_ngram.cuh"
-#include "verify_fused.cuh"
-#include "verify_bulk.cuh"
 
 namespace specdec {
 namespace {
 
 constexpr size_t kThetaBase = 0;
-constexpr size_t kCtlBase = kThetaBase + static_cast<size_t>(kThetaRows) * sizeof(unsigned);
-constexpr size_t kPartialBase = (kCtlBase + kCtlWords * sizeof(unsigned) + 255) / 256 * 256;
+constexpr size_t kPartialBase = kThetaBase + static_cast<size_t>(kThetaRows) * sizeof(unsigned);
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -82,20 +76,6 @@ constexpr int kMaxDevices = 64;
 // rows before the previous kernel of the stream has finished.
 std::atomic<int> g_prefetch_inputs{0};
 
-// specdec_set_stream_bulk: the argmax and top-8 streaming passes stage their
-// chunks in shared memory with bulk copies (1) or load into registers (0).
-std::atomic<int> g_stream_bulk{0};
-
-// specdec_set_rejection_fused: fixed-layout rejection calls of up to
-// kFusedMaxB requests run as the one fused kernel (1) or as the four kernels
-// (0).
-std::atomic<int> g_rejection_fused{1};
-
-// Clock cycles a CTA of the fused rejection kernel waits for a request's
-// decision before it gives up (about a second at B200 clocks; a decision
-// normally comes within microseconds).
-constexpr long long kWaitBudgetCycles = 2000000000LL;
-
 bool vector_path_ok(const void* p, int64_t stride, int esize) {
     return (reinterpret_cast<uintptr_t>(p) % 16 == 0) && ((stride * esize) % 16 == 0);
 }
@@ -103,18 +83,6 @@ bool vector_path_ok(const void* p, int64_t stride, int esize) {
 bool rows_fit(int64_t rows, int64_t row_stride, int V) {
     // Every element offset must fit comfortably in 63 bits.
     return row_stride >= V && row_stride <= (int64_t(1) << 40) && rows * row_stride < (int64_t(1) << 52);
-}
-
-// CTAs of a persistent kernel: as many as the current device keeps resident.
-template <class Kernel>
-cudaError_t persistent_ctas(Kernel fn, unsigned* out) {
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, NT, 0);
-    if (e != cudaSuccess) return e;
-    *out = static_cast<unsigned>((per_sm > 0 ? per_sm : 1) * (sms > 0 ? sms : 1));
-    return cudaSuccess;
 }
 
 // Launch with programmatic stream serialisation: the kernel may be scheduled
@@ -135,30 +103,6 @@ cudaError_t launch_pdl(Kernel fn, dim3 grid, int dyn, cudaStream_t stream, const
     return cudaLaunchKernelEx(&cfg, fn, P);
 }
 
-// The bulk-copy streaming kernel of a mode: its shared-memory ring (the
-// chunk) exceeds the default 48 KB for top-8, so the limit is raised once per
-// device.
-template <class Tag, int VEC, int MODE>
-cudaError_t launch_bulk_pass(const Pass1Params& P, dim3 grid, cudaStream_t stream) {
-    constexpr int CH = chunk_vecs(VEC, mode_u(MODE));
-    constexpr int kBytes = CH * 16;
-    static std::atomic<unsigned long long> ready{0};  // bit d: device d set up
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const unsigned long long bit = 1ull << (dev & 63);
-    if (!(ready.load(std::memory_order_acquire) & bit)) {
-        e = cudaFuncSetAttribute(verify_pass1_bulk_kernel<Tag, VEC, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(verify_pass1_bulk_kernel<Tag, VEC, MODE>,
-                                     cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        if (e != cudaSuccess) return e;
-        ready.fetch_or(bit, std::memory_order_release);
-    }
-    return launch_pdl(verify_pass1_bulk_kernel<Tag, VEC, MODE>, grid, kBytes, stream, P);
-}
-
 // The streaming pass (one CTA per chunk; trees stream like greedy argmax),
 // then the request epilogues (one CTA per request).
 template <class Tag, int VEC, int MODE>
@@ -166,15 +110,8 @@ specdec_status launch_pass1(Pass1Params P, cudaStream_t stream) {
     constexpr int STREAM_MODE = MODE == MODE_TREE ? MODE_ARGMAX : MODE;
     if (P.R > 0x7fffffff || P.cpr > 65535) return SPECDEC_ERR_UNSUPPORTED;  // grid limits
     const dim3 grid(static_cast<unsigned>(P.R), static_cast<unsigned>(P.cpr));
-    cudaError_t e;
-    if constexpr (VEC > 1 && STREAM_MODE != MODE_SOFTMAX) {
-        e = g_stream_bulk.load(std::memory_order_relaxed) ? launch_bulk_pass<Tag, VEC, STREAM_MODE>(P, grid, stream)
-                                                           : launch_pdl(verify_pass1_kernel<Tag, VEC, STREAM_MODE>,
-                                                                        grid, 0, stream, P);
-    } else {
-        e = launch_pdl(verify_pass1_kernel<Tag, VEC, STREAM_MODE>, grid, 0, stream, P);
-    }
-    if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
+    if (launch_pdl(verify_pass1_kernel<Tag, VEC, STREAM_MODE>, grid, 0, stream, P) != cudaSuccess)
+        return SPECDEC_ERR_CUDA;
     if constexpr (MODE == MODE_TOP8) {
         const int rows = P.k + 1 < kTop8EpiWarps ? P.k + 1 : kTop8EpiWarps;  // a warp per row
         if (launch_pdl(verify_top8_epilogue_kernel<Tag>, dim3(static_cast<unsigned>(P.B)), 0, stream, P, 32 * rows) !=
@@ -234,11 +171,11 @@ specdec_status dispatch_stats(specdec_dtype dt, bool vec, StatsParams S, cudaStr
 
 bool dtype_ok(specdec_dtype dt) { return dt == SPECDEC_F32 || dt == SPECDEC_BF16; }
 
-// Pass-1 partial bytes per chunk: one argmax key, 8 keys (top-8), or one
-// (max, sum) pair (softmax).
-constexpr size_t kArgmaxChunkBytes = kPartsPerChunk * sizeof(uint64_t);
-constexpr size_t kTop8ChunkBytes = kPartsPerChunk * 8 * sizeof(uint64_t);
-constexpr size_t kSoftmaxChunkBytes = kPartsPerChunk * sizeof(SoftmaxPartial);
+// Pass-1 partial bytes per chunk: one argmax key per warp, 8 keys per warp
+// (top-8), or one (max, sum) pair per warp (softmax).
+constexpr size_t kArgmaxChunkBytes = NWARPS * sizeof(uint64_t);
+constexpr size_t kTop8ChunkBytes = NWARPS * 8 * sizeof(uint64_t);
+constexpr size_t kSoftmaxChunkBytes = NWARPS * sizeof(SoftmaxPartial);
 size_t slot_bytes(specdec_mode mode) {
     if (mode == SPECDEC_MODE_GREEDY) return kArgmaxChunkBytes > kTop8ChunkBytes ? kArgmaxChunkBytes : kTop8ChunkBytes;
     if (mode == SPECDEC_MODE_REJECTION) return kSoftmaxChunkBytes;
@@ -266,7 +203,6 @@ void fill_common(Pass1Params& P, const void* logits, int64_t row_stride, int V, 
     P.rows_per_req = rows_per_req;
     P.B = B;
     P.theta_row = reinterpret_cast<unsigned*>(base + kThetaBase);
-    P.bulk_error = reinterpret_cast<unsigned*>(base + kCtlBase) + 1;
     P.partials = base + L.partials1;
 }
 
@@ -370,16 +306,8 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     P.req_base = req_base;
     const bool stats = entropy != nullptr && offsets == nullptr && k > 0;
     P.row_stat = stats ? reinterpret_cast<RowStat*>(static_cast<char*>(ws) + L.row_stat) : nullptr;
-    const uint64_t n_pass1 = static_cast<uint64_t>(L.NC);
-    const uint64_t n_total = n_pass1 + static_cast<uint64_t>(B) * static_cast<uint64_t>(L.cpr2);
-    const int fused_mode = g_rejection_fused.load(std::memory_order_relaxed);
-    const uint64_t n_total_p = n_pass1 + 2ull * static_cast<uint64_t>(B) + static_cast<uint64_t>(B) * L.cpr2;
-    const bool fused = fused_mode != 0 && offsets == nullptr && !stats && B <= kFusedMaxB &&
-                       n_total_p < 0x7fffffffull;
-    if (!fused) {
-        st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
-        if (st != SPECDEC_OK) return st;
-    }
+    st = dispatch_pass1<MODE_SOFTMAX>(dtype, vec, P, s);
+    if (st != SPECDEC_OK) return st;
     Pass2Params Q;
     memset(&Q, 0, sizeof(Q));
     Q.logits = target_logits;
@@ -400,52 +328,6 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     Q.chunk_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.masses);
     Q.unit_mass = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.units);
     Q.out_tokens = out_tokens;
-    if (fused) {
-        FusedParams F;
-        memset(&F, 0, sizeof(F));
-        F.p1 = P;
-        F.p1.prefetch_inputs = 0;  // the kernel waits for the previous one before its first access
-        F.p2 = Q;
-        unsigned* ctl = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kCtlBase);
-        F.next = ctl;
-        F.error = ctl + 1;
-        F.req_ticket = ctl + kCtlHeadWords;
-        F.decided = F.req_ticket + kFusedMaxB;
-        F.res_ticket = F.decided + kFusedMaxB;
-        F.n_pass1 = static_cast<unsigned>(n_pass1);
-        F.wait_budget = kWaitBudgetCycles;
-        F.exits = ctl + 3;
-        cudaError_t e;
-        if (fused_mode == 2) {
-            F.n_total = static_cast<unsigned>(n_total_p);
-            unsigned ctas = 0;
-            if (dtype == SPECDEC_BF16)
-                e = vec ? persistent_ctas(verify_rejection_persistent_kernel<BF16Tag, 8>, &ctas)
-                        : persistent_ctas(verify_rejection_persistent_kernel<BF16Tag, 1>, &ctas);
-            else
-                e = vec ? persistent_ctas(verify_rejection_persistent_kernel<F32Tag, 4>, &ctas)
-                        : persistent_ctas(verify_rejection_persistent_kernel<F32Tag, 1>, &ctas);
-            if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
-            const dim3 grid(ctas < F.n_total ? ctas : F.n_total);
-            if (dtype == SPECDEC_BF16)
-                e = vec ? launch_pdl(verify_rejection_persistent_kernel<BF16Tag, 8>, grid, 0, s, F)
-                        : launch_pdl(verify_rejection_persistent_kernel<BF16Tag, 1>, grid, 0, s, F);
-            else
-                e = vec ? launch_pdl(verify_rejection_persistent_kernel<F32Tag, 4>, grid, 0, s, F)
-                        : launch_pdl(verify_rejection_persistent_kernel<F32Tag, 1>, grid, 0, s, F);
-        } else {
-            F.n_total = static_cast<unsigned>(n_total);
-            const dim3 grid(static_cast<unsigned>(n_total));
-            if (dtype == SPECDEC_BF16)
-                e = vec ? launch_pdl(verify_rejection_fused_kernel<BF16Tag, 8>, grid, 0, s, F)
-                        : launch_pdl(verify_rejection_fused_kernel<BF16Tag, 1>, grid, 0, s, F);
-            else
-                e = vec ? launch_pdl(verify_rejection_fused_kernel<F32Tag, 4>, grid, 0, s, F)
-                        : launch_pdl(verify_rejection_fused_kernel<F32Tag, 1>, grid, 0, s, F);
-        }
-        if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
-        return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
-    }
     st = dispatch_pass2(dtype, vec, Q, s);
     if (st != SPECDEC_OK || !stats) return st;
     StatsParams S;
@@ -1023,38 +905,6 @@ specdec_status specdec_ngram_propose(const int32_t* tokens, int64_t token_stride
 }
 
 int specdec_set_prefetch_inputs(int enable) { return g_prefetch_inputs.exchange(enable ? 1 : 0); }
-
-int specdec_set_stream_bulk(int enable) { return g_stream_bulk.exchange(enable ? 1 : 0); }
-
-int specdec_set_rejection_fused(int enable) { return g_rejection_fused.exchange(enable < 0 || enable > 2 ? 1 : enable); }
-
-specdec_status specdec_workspace_check(const void* ws, size_t ws_bytes, struct CUstream_st* stream) {
-    if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % 16 != 0 || ws_bytes < kPartialBase)
-        return SPECDEC_ERR_WORKSPACE;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(s) != cudaSuccess) return SPECDEC_ERR_CUDA;
-    unsigned err = 0;
-    if (cudaMemcpy(&err, static_cast<const char*>(ws) + kCtlBase + sizeof(unsigned), sizeof(err),
-                   cudaMemcpyDeviceToHost) != cudaSuccess)
-        return SPECDEC_ERR_CUDA;
-    return err != 0u ? SPECDEC_ERR_TIMEOUT : SPECDEC_OK;
-}
-
-specdec_status specdec_selftest_wait_timeout(void* ws, size_t ws_bytes, long long budget_cycles,
-                                             struct CUstream_st* stream) {
-    if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % 16 != 0 || ws_bytes < kPartialBase)
-        return SPECDEC_ERR_WORKSPACE;
-    if (budget_cycles < 1 || budget_cycles > kWaitBudgetCycles) return SPECDEC_ERR_INVALID_ARG;
-    unsigned* ctl = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + kCtlBase);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(1);
-    cfg.blockDim = dim3(32);
-    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaLaunchKernelEx(&cfg, verify_wait_selftest_kernel, static_cast<const unsigned*>(ctl + 2), ctl + 1,
-                           budget_cycles) != cudaSuccess)
-        return SPECDEC_ERR_CUDA;
-    return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
-}
 
 double specdec_tier_update(specdec_tier_state* state, double accepted, double decay) {
     if (state == nullptr || !(decay >= 0.0 && decay < 1.0) || !(accepted >= 0.0 && accepted <= SPECDEC_MAX_K))

@@ -8,8 +8,8 @@
 // times larger than what the GPU keeps resident, so the hardware block
 // scheduler hands chunks to SMs as they free up and no SM waits for a slower
 // one.  Every thread issues its loads of the chunk at once; each warp reduces
-// its part (argmax key, top-8 keys, or softmax max/sum) and the CTA merges
-// the warps' results into one partial per chunk.
+// its part (argmax key, top-8 keys, or softmax max/sum) and stores one
+// partial per (chunk, warp).
 //
 // The request epilogues run as a second kernel (one CTA per request,
 // launched with programmatic stream serialisation so it is resident before
@@ -91,11 +91,6 @@ static_assert(kUTop8 >= kU, "the top-8 chunks must not be smaller than the other
 
 constexpr int kCandBuf = 64;  // top-8 candidate buffer per warp
 
-// Partials the streaming pass stores per chunk: its CTA merges its warps'
-// results first (one argmax key, one (max, sum) pair, or 8 top-8 keys per
-// chunk), so the request epilogues read 1/NWARPS as many.
-constexpr int kPartsPerChunk = 1;
-
 struct SoftmaxPartial {
     float M;
     float pad;
@@ -115,7 +110,7 @@ struct Pass1Params {
     int B;
     // workspace
     unsigned* theta_row;        // [kThetaRows] top-8 thresholds (ordered keys)
-    void* partials;             // [R * cpr * kPartsPerChunk] slots
+    void* partials;             // [R * cpr * NWARPS] slots
     // greedy / rejection
     const int32_t* drafts;
     int k;                      // drafts per request (packed layout: the bound max_k)
@@ -145,7 +140,6 @@ struct Pass1Params {
     RowStat* row_stat;          // [rows] every row's (M, Z), or null
     uint32_t req_base;          // Philox request index of request 0 (a slice of a larger batch)
     int prefetch_inputs;            // the argmax pass may load rows before the previous kernel ends
-    unsigned* bulk_error;           // the workspace's error word (bulk-copy path)
     // vocabulary-sharded greedy
     int vocab_offset;               // global index of this shard's column 0
     uint64_t* shard_keys;           // [R, kk] out: this shard's row keys, global indices
@@ -172,8 +166,6 @@ struct Pass1Smem {
     int drafts[kMaxRowsPerReq];
     float rowM[kMaxRowsPerReq];
     double rowZ[kMaxRowsPerReq];
-    float wM[NWARPS];                  // softmax: per-warp (max, sum) before the chunk merge
-    double wS[NWARPS];
 };
 struct TreeArrays {
     uint64_t key[kTreeNodes];
@@ -299,15 +291,10 @@ struct ArgmaxReducer {
         const bool up = m > best.v;
         if (__any_sync(FULL_MASK, up)) best = argmax_raise<Tag, 1>(w, idx, up, m);
     }
-    // CTA-collective: the chunk's best key (the largest of the warps').
-    __device__ __forceinline__ void end(int64_t, int, uint64_t chunk, const Pass1Params& P, Pass1Smem& sm) {
-        const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-        if (lane == 0) sm.red[wp] = best.i >= 0 ? make_key(best.v, best.i) : 0ull;
-        __syncthreads();
-        if (wp == 0) {
-            const uint64_t k = warp_max_u64(lane < NWARPS ? sm.red[lane] : 0ull);
-            if (lane == 0) static_cast<uint64_t*>(P.partials)[chunk] = k;
-        }
+    __device__ __forceinline__ void end(int64_t, int, uint64_t chunk, const Pass1Params& P, Pass1Smem&) {
+        if ((threadIdx.x & 31) == 0)
+            static_cast<uint64_t*>(P.partials)[chunk * NWARPS + (threadIdx.x >> 5)] =
+                best.i >= 0 ? make_key(best.v, best.i) : 0ull;
     }
 };
 
@@ -453,16 +440,19 @@ struct Top8Reducer {
                                     sm.cand[wp]);
         }
     }
-    // CTA-collective: the chunk's best 8 keys (the 8 best of the warps' 8
-    // best, a warp's being its buffered candidates when no more than 8 and
-    // never merged, else its merged list).  The chunk's 8th best also raises
-    // the row's shared threshold for the row's chunks that start later.
-    __device__ __forceinline__ void end(int64_t r, int, uint64_t chunk, const Pass1Params& P, Pass1Smem& sm) {
+    // Each warp stores 8 keys that include its best 8 of the chunk: its
+    // buffered candidates as they are when no more than 8 and never merged,
+    // else its merged best 8.  On a row's first sub-chunk the CTA also takes
+    // the chunk's 8th best (CTA-collective) to raise the row's shared
+    // threshold for the row's later chunks.
+    __device__ __forceinline__ void end(int64_t r, int sub, uint64_t chunk, const Pass1Params& P, Pass1Smem& sm) {
         const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
         if (st.merged || st.cnt > 8) st = top8_merge(st, sm.wtop[wp], sm.cand[wp]);
         __syncwarp();
         uint64_t mine = 0ull;
         if (lane < 8) mine = st.merged ? sm.wtop[wp][lane] : (lane < st.cnt ? sm.cand[wp][lane] : 0ull);
+        if (lane < 8) static_cast<uint64_t*>(P.partials)[(chunk * NWARPS + wp) * 8 + lane] = mine;
+        if (sub != 0 || r >= kThetaRows) return;
         if (lane < 8) sm.stage[wp * 8 + lane] = mine;
         __syncthreads();
         if (wp == 0) {
@@ -473,10 +463,8 @@ struct Top8Reducer {
                 const uint64_t kk = sm.stage[i];
                 if (kk > l[7]) top8_insert(l, kk);
             }
-            const uint64_t top = warp_top8(l);
-            if (lane < 8) static_cast<uint64_t*>(P.partials)[chunk * 8 + lane] = top;
-            const uint64_t k7 = __shfl_sync(FULL_MASK, top, 7);
-            if (lane == 0 && k7 != 0ull && r < kThetaRows) atomicMax(&P.theta_row[r], static_cast<unsigned>(k7 >> 32));
+            const uint64_t k7 = __shfl_sync(FULL_MASK, warp_top8(l), 7);
+            if (lane == 0 && k7 != 0ull) atomicMax(&P.theta_row[r], static_cast<unsigned>(k7 >> 32));
         }
     }
 };
@@ -485,8 +473,8 @@ struct Top8Reducer {
 // logits (NaN ignored), then S = sum exp((l - M)/T) over the part, fp32 exp
 // and sum within a vector, fp64 across vectors and lanes.  The part's
 // elements are held in registers, so the max is known before any exp is
-// taken and no rescaling is needed within a part; the CTA then merges its
-// warps' parts into one (M, S) partial per chunk.
+// taken and no rescaling is needed; no CTA barrier is involved.  One (M, S)
+// partial per (chunk, warp).
 template <class Tag, int VEC>
 struct SoftmaxReducer {
     float invT;
@@ -509,38 +497,16 @@ struct SoftmaxReducer {
         for (int e = 0; e < VEC; ++e) s += exp2f((VecOps<Tag, VEC>::elem(w, e) - M) * log2e_invT);
         return static_cast<double>(s);
     }
-    // CTA-collective: store the chunk's (M, S), merged from the warps' parts:
-    // M = the largest warp max, S = sum over warps of S_w exp2((M_w - M)
-    // log2(e)/T) in fp64 (lane w of warp 0 takes warp w's term; the sum runs
-    // in a fixed order).
-    __device__ __forceinline__ void store(float M, double S, uint64_t chunk, const Pass1Params& P,
-                                          Pass1Smem& sm) const {
-        const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    // Warp-collective: store (M, S) of the warp's part of the chunk.
+    __device__ __forceinline__ void store(float M, double S, uint64_t chunk, const Pass1Params& P) const {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(FULL_MASK, S, o);
-        if (lane == 0) {
-            sm.wM[wp] = M;
-            sm.wS[wp] = S;
-        }
-        __syncthreads();
-        if (wp == 0) {
-            const float mw = lane < NWARPS ? sm.wM[lane] : -FLT_MAX;
-            const double sw = lane < NWARPS ? sm.wS[lane] : 0.0;
-            float Mc = mw;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(FULL_MASK, Mc, o));
-            // A part with no mass adds nothing; NaN (a NaN or +inf logit) carries
-            // through, so the row is found undefined, as in maxsum_merge.
-            double t = sw != 0.0 ? sw * exp((static_cast<double>(mw) - static_cast<double>(Mc)) * invT_d) : 0.0;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(FULL_MASK, t, o);
-            if (lane == 0) {
-                SoftmaxPartial sp;
-                sp.M = Mc;
-                sp.pad = 0.0f;
-                sp.S = t;
-                static_cast<SoftmaxPartial*>(P.partials)[chunk] = sp;
-            }
+        if ((threadIdx.x & 31) == 0) {
+            SoftmaxPartial sp;
+            sp.M = M;
+            sp.pad = 0.0f;
+            sp.S = S;
+            static_cast<SoftmaxPartial*>(P.partials)[chunk * NWARPS + (threadIdx.x >> 5)] = sp;
         }
     }
 };
@@ -551,7 +517,7 @@ template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_TREE> { using typ
 template <class Tag, int VEC> struct ReducerFor<Tag, VEC, MODE_TOP8> { using type = Top8Reducer<Tag, VEC>; };
 
 // ---------------------------------------------------------------------------
-// Row merges for the epilogues: warp-collective, over the row's cpr
+// Row merges for the epilogues: warp-collective, over the row's cpr * NWARPS
 // partials.  A row whose partials hold no element above -inf (argmax) or
 // fewer than 8 elements above NaN (top-8) is rescanned exactly, element by
 // element, so NaN and -inf rank correctly.
@@ -566,7 +532,7 @@ template <class Tag>
 __device__ void merge_argmax_rows(const Pass1Params& P, int64_t r0, int n, uint64_t* keys) {
     constexpr int kRowB = 9, kJB = 3;
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    const int np = P.cpr * kPartsPerChunk;
+    const int np = P.cpr * NWARPS;
     const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r0 * np;
     for (int t0 = wp; t0 < n; t0 += NWARPS * kRowB) {
         uint64_t best[kRowB];
@@ -616,7 +582,7 @@ template <class Tag>
 __device__ uint64_t row_top8_key(const Pass1Params& P, int64_t r) {
     constexpr int KB = 16;  // keys per lane per batch
     const int lane = threadIdx.x & 31;
-    const int nk = P.cpr * kPartsPerChunk * 8;
+    const int nk = P.cpr * NWARPS * 8;
     const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r * nk;
     const uint64_t floor_key = r < kThetaRows ? static_cast<uint64_t>(__ldcg(&P.theta_row[r])) << 32 : 0ull;
     uint64_t l[8];
@@ -670,7 +636,7 @@ __device__ void row_top8_warp(const Pass1Params& P, int64_t r, uint64_t* surv, u
     constexpr int KB = 16;  // keys per lane per batch
     const int lane = threadIdx.x & 31;
     const unsigned lt_mask = (1u << lane) - 1u;
-    const int nk = P.cpr * kPartsPerChunk * 8;
+    const int nk = P.cpr * NWARPS * 8;
     const uint64_t* p = static_cast<const uint64_t*>(P.partials) + r * nk;
     unsigned fl = 0u;
     if (lane == 0 && r < kThetaRows) fl = __ldcg(&P.theta_row[r]);
@@ -942,7 +908,7 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
     }
     for (int t = wp; t <= k; t += NWARPS) {
         const int64_t r = g.row0 + t;
-        const int np = P.cpr * kPartsPerChunk;
+        const int np = P.cpr * NWARPS;
         const SoftmaxPartial* p = static_cast<const SoftmaxPartial*>(P.partials) + r * np;
         MaxSum acc;
         acc.M = -FLT_MAX;
@@ -1082,7 +1048,7 @@ __device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typena
     }
     if (has_tail) S += static_cast<double>(exp2f((tail - M) * P.log2e_invT));
     if (P.prefetch_inputs) grid_dependency_wait();  // the pass began without waiting
-    red.store(M, S, static_cast<uint64_t>(r) * P.cpr + sub, P, sm);
+    red.store(M, S, static_cast<uint64_t>(r) * P.cpr + sub, P);
 }
 
 // ---------------------------------------------------------------------------
@@ -1366,7 +1332,7 @@ __global__ void __launch_bounds__(NT) verify_shard_softmax_rows_kernel(const Pas
     grid_launch_dependents();
     const int64_t r = static_cast<int64_t>(blockIdx.x) * NWARPS + wp;  // a warp per row
     if (r >= P.R) return;  // warp-uniform
-    const int np = P.cpr * kPartsPerChunk;
+    const int np = P.cpr * NWARPS;
     const SoftmaxPartial* p = static_cast<const SoftmaxPartial*>(P.partials) + r * np;
     MaxSum acc;
     acc.M = -FLT_MAX;

@@ -172,8 +172,8 @@ __device__ __forceinline__ double warp_sum_transpose(double (&v)[N]) {
 // loads of a batch of kU vectors before any arithmetic.
 // ---------------------------------------------------------------------------
 template <class Tag, int VEC>
-__device__ __forceinline__ void resample_chunk(const Pass2Params& P, const RejState& st, int64_t b, int sub,
-                                               double (&red)[2][NWARPS]) {
+__global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P) {
+    __shared__ double red[2][NWARPS];
     using Elem = typename Tag::storage;
     constexpr int CH = chunk_vecs(VEC, kU2);
     constexpr int UPT = chunk_upt(VEC, kU2);
@@ -183,6 +183,14 @@ __device__ __forceinline__ void resample_chunk(const Pass2Params& P, const RejSt
     static_assert(NV == 2 || NV == 4 || NV == 8 || NV == 16, "kU2 must be 1, 2, 4 or 8");
     const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
     const int t = static_cast<int>(threadIdx.x);
+
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    const int64_t b = blockIdx.x;
+    const int sub = static_cast<int>(blockIdx.y);
+    const RejState st = P.state[b];
+    if (!st.valid) return;  // CTA-uniform
     const Pass2Row R = pass2_row<Tag>(P, st);
     const Elem* row = static_cast<const Elem*>(R.row);
     const int cnt = chunk_count(P.nv_full, sub, VEC, kU2);
@@ -266,17 +274,6 @@ __device__ __forceinline__ void resample_chunk(const Pass2Params& P, const RejSt
     }
 }
 
-template <class Tag, int VEC>
-__global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P) {
-    __shared__ double red[2][NWARPS];
-    grid_dependency_wait();
-    grid_launch_dependents();
-    const int64_t b = blockIdx.x;
-    const RejState st = P.state[b];
-    if (!st.valid) return;  // CTA-uniform
-    resample_chunk<Tag, VEC>(P, st, b, static_cast<int>(blockIdx.y), red);
-}
-
 // ---------------------------------------------------------------------------
 // Token search, one warp per request.
 // ---------------------------------------------------------------------------
@@ -356,13 +353,19 @@ __device__ __forceinline__ int warp_find_level(const double2* m, int n, bool use
     return last;
 }
 
-// The token of request b (warp-collective; one warp per request).
 template <class Tag, int VEC>
-__device__ __forceinline__ void token_search(const Pass2Params& P, const RejState& st, int64_t b) {
+__global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass2Params P) {
     using Elem = typename Tag::storage;
     constexpr int CH = chunk_vecs(VEC, kU2);
     constexpr int UPC = units_per_chunk(VEC);
     const int lane = threadIdx.x & 31;
+
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    const int64_t b = static_cast<int64_t>(blockIdx.x) * NWARPS + (threadIdx.x >> 5);
+    if (b >= P.B) return;  // warp-uniform
+    const RejState st = P.state[b];
     if (!st.valid) {  // the statistics pass already wrote -1 everywhere
         if (P.shard_totals != nullptr && lane == 0) P.shard_token[b] = -1;
         return;
@@ -504,15 +507,6 @@ __device__ __forceinline__ void token_search(const Pass2Params& P, const RejStat
         if (P.shard_totals == nullptr) P.out_tokens[out_at] = token;
         else P.shard_token[b] = P.vocab_offset + token;
     }
-}
-
-template <class Tag, int VEC>
-__global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass2Params P) {
-    grid_dependency_wait();
-    grid_launch_dependents();
-    const int64_t b = static_cast<int64_t>(blockIdx.x) * NWARPS + (threadIdx.x >> 5);
-    if (b >= P.B) return;  // warp-uniform
-    token_search<Tag, VEC>(P, P.state[b], b);
 }
 
 // Vocabulary-sharded rejection: this shard's total (residual, target) mass

@@ -81,8 +81,8 @@ def test_static_scratch_binding_refuses_other_devices(monkeypatch):
 def _inputs(name):
     if name == "llama3":
         return gen.greedy_llama3(), 0
-    if name == "large_batch":
-        return gen.greedy_large_batch(), 8
+    if name == "large_batch":  # 128 of the large batch's requests: within the fixed scratch
+        return gen.greedy_large_batch(B=128), 8
     if name == "large_batch_16":  # the first 16 requests of the large batch: fewer rows, same scratch words
         inp = _inputs("large_batch")[0]
         return gen.GreedyInputs("large_batch_16", inp.dtype, inp.logits[:16].copy(), inp.drafts[:16].copy(), 16,
