@@ -261,6 +261,18 @@ specdec_status greedy_impl(const void* logits, specdec_dtype dtype, int64_t row_
     P.topk_ids = topk_ids;
     P.topk_vals = topk_vals;
     if (topk > 0) return dispatch_pass1<MODE_TOP8>(dtype, vec, P, s);
+    if (static_cast<int64_t>(k + 1) * V * elem_size(dtype) <= kSmallRequestBytes) {
+        // small requests: the whole verification in one launch, a CTA per request
+        cudaError_t e;
+        if (dtype == SPECDEC_BF16)
+            e = vec ? launch_pdl(verify_small_greedy_kernel<BF16Tag, 8>, dim3(static_cast<unsigned>(B)), 0, s, P)
+                    : launch_pdl(verify_small_greedy_kernel<BF16Tag, 1>, dim3(static_cast<unsigned>(B)), 0, s, P);
+        else
+            e = vec ? launch_pdl(verify_small_greedy_kernel<F32Tag, 4>, dim3(static_cast<unsigned>(B)), 0, s, P)
+                    : launch_pdl(verify_small_greedy_kernel<F32Tag, 1>, dim3(static_cast<unsigned>(B)), 0, s, P);
+        if (e != cudaSuccess) return SPECDEC_ERR_CUDA;
+        return cudaGetLastError() == cudaSuccess ? SPECDEC_OK : SPECDEC_ERR_CUDA;
+    }
     return dispatch_pass1<MODE_ARGMAX>(dtype, vec, P, s);
 }
 

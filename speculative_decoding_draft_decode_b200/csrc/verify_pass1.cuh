@@ -1191,6 +1191,72 @@ __global__ void __launch_bounds__(32 * kTop8EpiWarps) verify_top8_epilogue_kerne
 }
 
 // ---------------------------------------------------------------------------
+// Greedy verification of small requests in one kernel (no top-k): one CTA
+// per request, one warp per row (rows dealt round-robin to the 8 warps).  A
+// warp streams its row 32 consecutive vectors per step, kSmallBatch steps of
+// loads in flight, with the argmax reducer of the streaming pass (ties to the
+// lowest index: a later step never wins a tie), rescans exactly a row with no
+// element above -inf, and the CTA then runs the accept scan.  For requests of
+// at most kSmallRequestBytes this replaces the streaming pass and the
+// request epilogue (two launches and a kernel boundary) by one launch.
+// ---------------------------------------------------------------------------
+constexpr int kSmallBatch = 8;                  // 16-byte loads in flight per lane
+constexpr int64_t kSmallRequestBytes = 32768;   // logit bytes of a request
+
+template <class Tag, int VEC>
+__global__ void __launch_bounds__(NT) verify_small_greedy_kernel(const Pass1Params P) {
+    __shared__ Pass1Smem sm;
+    using Elem = typename Tag::storage;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int64_t b = blockIdx.x;
+    const ReqGeom g = req_geom(P, b);
+    if (!g.ok) {
+        if (threadIdx.x == 0) P.accept_len[b] = -1;
+        return;
+    }
+    const int k = g.kb;
+    const int dr = static_cast<int>(threadIdx.x) < k ? P.drafts[g.d0 + threadIdx.x] : 0;
+    for (int t = wp; t <= k; t += NWARPS) {
+        const Elem* row = static_cast<const Elem*>(P.logits) + (g.row0 + t) * P.row_stride;
+        ArgmaxReducer<Tag, VEC> red;
+        red.begin(0, 0, P, sm);
+        for (int j0 = 0; j0 < P.nv_full; j0 += 32 * kSmallBatch) {
+            uint4 w[kSmallBatch];
+#pragma unroll
+            for (int q = 0; q < kSmallBatch; ++q) {
+                const int j = j0 + q * 32 + lane;
+                w[q] = make_uint4(0u, 0u, 0u, 0u);
+                if (j < P.nv_full) RowLoader<Tag, VEC>::raw(row, j, w[q]);
+            }
+#pragma unroll
+            for (int q = 0; q < kSmallBatch; ++q) {
+                const int j = j0 + q * 32 + lane;
+                red.vec(w[q], j * VEC, j < P.nv_full, sm);
+            }
+        }
+        for (int x0 = P.nv_full * VEC; x0 < P.V; x0 += 32) {  // the ragged row end
+            const int x = x0 + lane;
+            const bool ok = x < P.V;
+            red.scalar(ok ? load_scalar<Tag>(row + x) : 0.0f, x, ok, sm);
+        }
+        uint64_t key = red.best.i >= 0 ? make_key(red.best.v, red.best.i) : 0ull;
+        if (key == 0ull) {  // no element above -inf: exact rescan
+            for (int x = lane; x < P.V; x += 32) {
+                const uint64_t kx = make_key(load_scalar<Tag>(row + x), x);
+                key = kx > key ? kx : key;
+            }
+            key = warp_max_u64(key);
+        }
+        if (lane == 0) sm.am[t] = key_index(key);
+    }
+    if (static_cast<int>(threadIdx.x) < k) sm.drafts[threadIdx.x] = dr;
+    __syncthreads();
+    greedy_accept(P, b, g, sm.drafts, sm.am);
+}
+
+// ---------------------------------------------------------------------------
 // Vocabulary-sharded greedy verification (Arctic page, "Speculator
 // optimisation": the logits are sharded over the vocabulary as the scorer's
 // tensor parallelism leaves them; each shard takes its own TopK, the shards'

@@ -90,6 +90,21 @@ def test_greedy_ragged_vocab(V_, V, dtype):
     check_greedy(V_, inp, topk=8)
 
 
+@pytest.mark.parametrize("dtype,k,V", [("f32", 3, 2048), ("f32", 3, 2049), ("bf16", 7, 2048), ("bf16", 7, 2049),
+                                       ("bf16", 0, 16384), ("f32", 1, 4095), ("bf16", 15, 1031)])
+def test_greedy_small_request_path_boundary(V_, dtype, k, V):
+    """Requests of at most 32 KB of logits take the one-launch path (a CTA per
+    request); one element more takes the streaming pass and the epilogue.
+    Both sides of the boundary, ragged row ends included, against the
+    oracle, with NaN rows and ties mixed in."""
+    inp = gen.greedy_synthetic(seed=k * 7 + V, B=9, k=k, V=V, alpha=0.7, sigma=2.0, dtype=dtype)
+    if dtype == "f32":
+        inp.logits[1, 0, :] = np.nan
+        inp.logits[2, k, :] = -np.inf
+        inp.logits[3, 0, ::3] = inp.logits[3, 0].max()
+    check_greedy(V_, inp)
+
+
 @pytest.mark.parametrize("k", [0, 1, 31, 32])
 def test_greedy_k_extremes(V_, k):
     inp = gen.greedy_synthetic(seed=100 + k, B=7, k=k, V=3000, alpha=0.9, dtype="bf16")
