@@ -211,6 +211,18 @@ def resample_bytes(inp, outs):
     return int(inp.V * (es * ok.sum() + 4 * (ok & (al < inp.k)).sum())) + extra
 
 
+SMALL_REQUEST_BYTES = 32768  # greedy requests up to this many logit bytes verify in one launch (no top-k)
+
+
+def greedy_launches(inp):
+    """Kernels one greedy call launches: one for requests of at most 32 KB of
+    logits without top-k (a CTA per request), else the streaming pass and the
+    request epilogue."""
+    es = 2 if inp.dtype == gen.BF16 else 4
+    k = inp.max_k if isinstance(inp, gen.RaggedInputs) else inp.k
+    return 1 if inp.topk == 0 and (k + 1) * inp.V * es <= SMALL_REQUEST_BYTES else 2
+
+
 def setup_calls(inp, sets, ver, device):
     """Static outputs and a list of per-set call closures (each one C-ABI
     call on the current stream)."""
@@ -251,7 +263,7 @@ def setup_calls(inp, sets, ver, device):
         for s in sets:
             calls.append(lambda s=s: ver.greedy_ragged(s["logits"], s["drafts"], s["offsets"], T, inp.max_k,
                                                        topk=inp.topk, counters=ctr, out=outs[:4]))
-        kernels = 2  # streaming pass + request epilogue (acceptance counters fused)
+        kernels = greedy_launches(inp)  # streaming pass + request epilogue (acceptance counters fused)
     else:
         k1 = inp.k + 1
         al = torch.empty(B, dtype=torch.int32, device=device)
@@ -261,7 +273,7 @@ def setup_calls(inp, sets, ver, device):
         outs = (al, ot, ids, vals)
         for s in sets:
             calls.append(lambda s=s: ver.greedy(s["logits"], s["drafts"], topk=inp.topk, out=outs))
-        kernels = 2  # streaming pass + request epilogue
+        kernels = greedy_launches(inp)  # streaming pass + request epilogue, or one launch for small requests
     return calls, outs, kernels
 
 

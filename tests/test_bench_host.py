@@ -128,6 +128,16 @@ def test_resample_bytes_follow_the_accepted_lengths(stats):
     assert bench.resample_bytes(_greedy(4, 3, 1000, gen.F32), (al,)) == 0
 
 
+def test_greedy_launch_count():
+    """One launch for requests of at most 32 KB of logits without top-k (the
+    tiny batch), two otherwise."""
+    assert bench.greedy_launches(gen.GreedyInputs("s", gen.F32, None, None, 4, 4, 1000)) == 1
+    assert bench.greedy_launches(gen.GreedyInputs("s", gen.F32, None, None, 4, 3, 2048)) == 1
+    assert bench.greedy_launches(gen.GreedyInputs("s", gen.F32, None, None, 4, 3, 2049)) == 2
+    assert bench.greedy_launches(gen.GreedyInputs("s", gen.F32, None, None, 4, 4, 1000, topk=8)) == 2
+    assert bench.greedy_launches(gen.GreedyInputs("s", gen.BF16, None, None, 64, 5, 128256)) == 2
+
+
 def test_rows_of_each_layout():
     g = _greedy(7, 3, 50, gen.F32)
     assert bench.rows_of(g) == 28 and bench.rows_of(g, 2) == 8
