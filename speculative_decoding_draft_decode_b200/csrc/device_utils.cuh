@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <float.h>
 #include <stdint.h>
 
 #include "geometry.h"
@@ -198,6 +199,47 @@ __device__ __forceinline__ MaxSum warp_maxsum(MaxSum v, double invT) {
         v = lower ? maxsum_merge(v, w, invT) : maxsum_merge(w, v, invT);
     }
     return v;
+}
+
+// Warp-collective merge of a row's n (max, sum) partials p[0, n): each lane
+// loads its partials once (kB at a time, read through L2); per batch the
+// lanes take the batch max, then one exp per partial, independent of one
+// another, and batches merge pairwise.  A partial with S == 0 adds nothing;
+// a NaN S (a NaN or +inf logit) makes S NaN.
+template <class Partial>
+__device__ __forceinline__ MaxSum warp_row_maxsum(const Partial* p, int n, double invT) {
+    constexpr int kB = 8;
+    const int lane = threadIdx.x & 31;
+    MaxSum acc;
+    acc.M = -FLT_MAX;
+    acc.S = 0.0;
+    for (int i0 = 0; i0 < n; i0 += 32 * kB) {
+        float pm[kB];
+        double ps[kB];
+#pragma unroll
+        for (int j = 0; j < kB; ++j) {
+            const int i = i0 + 32 * j + lane;
+            pm[j] = i < n ? __ldcg(&p[i].M) : -FLT_MAX;
+            ps[j] = i < n ? __ldcg(&p[i].S) : 0.0;
+        }
+        float m = -FLT_MAX;
+#pragma unroll
+        for (int j = 0; j < kB; ++j)
+            if (ps[j] != 0.0) m = fmaxf(m, pm[j]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, o));
+        double s = 0.0;
+#pragma unroll
+        for (int j = 0; j < kB; ++j)
+            if (ps[j] != 0.0) s += ps[j] * exp((static_cast<double>(pm[j]) - static_cast<double>(m)) * invT);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(FULL_MASK, s, o);
+        MaxSum b;
+        b.M = m;
+        b.S = s;
+        acc = i0 == 0 ? b : maxsum_merge(acc, b, invT);
+    }
+    return acc;
 }
 
 __device__ __forceinline__ MaxSum block_maxsum(MaxSum v, double invT, MaxSum* red) {

@@ -910,22 +910,7 @@ __device__ void epilogue_rejection(const Pass1Params& P, int64_t b, Pass1Smem& s
         const int64_t r = g.row0 + t;
         const int np = P.cpr * NWARPS;
         const SoftmaxPartial* p = static_cast<const SoftmaxPartial*>(P.partials) + r * np;
-        MaxSum acc;
-        acc.M = -FLT_MAX;
-        acc.S = 0.0;
-        constexpr int kPB = 8;  // partials per lane per batch, loaded together
-        for (int i0 = lane; i0 < np; i0 += 32 * kPB) {
-            MaxSum x[kPB];
-#pragma unroll
-            for (int j = 0; j < kPB; ++j) {
-                const int i = i0 + 32 * j;
-                x[j].M = i < np ? __ldcg(&p[i].M) : -FLT_MAX;
-                x[j].S = i < np ? __ldcg(&p[i].S) : 0.0;
-            }
-#pragma unroll
-            for (int j = 0; j < kPB; ++j) acc = maxsum_merge(acc, x[j], P.invT_d);
-        }
-        acc = warp_maxsum(acc, P.invT_d);
+        const MaxSum acc = warp_row_maxsum(p, np, P.invT_d);
         if (lane == 0) {
             sm.rowM[t] = acc.M;
             sm.rowZ[t] = acc.S;
@@ -1400,22 +1385,7 @@ __global__ void __launch_bounds__(NT) verify_shard_softmax_rows_kernel(const Pas
     if (r >= P.R) return;  // warp-uniform
     const int np = P.cpr * NWARPS;
     const SoftmaxPartial* p = static_cast<const SoftmaxPartial*>(P.partials) + r * np;
-    MaxSum acc;
-    acc.M = -FLT_MAX;
-    acc.S = 0.0;
-    constexpr int kPB = 8;
-    for (int i0 = lane; i0 < np; i0 += 32 * kPB) {
-        MaxSum x[kPB];
-#pragma unroll
-        for (int j = 0; j < kPB; ++j) {
-            const int i = i0 + 32 * j;
-            x[j].M = i < np ? __ldcg(&p[i].M) : -FLT_MAX;
-            x[j].S = i < np ? __ldcg(&p[i].S) : 0.0;
-        }
-#pragma unroll
-        for (int j = 0; j < kPB; ++j) acc = maxsum_merge(acc, x[j], P.invT_d);
-    }
-    acc = warp_maxsum(acc, P.invT_d);
+    const MaxSum acc = warp_row_maxsum(p, np, P.invT_d);
     if (lane == 0) {
         ShardRowStat st = {};
         st.M = acc.M;

@@ -365,6 +365,16 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
 
     const int64_t b = static_cast<int64_t>(blockIdx.x) * NWARPS + (threadIdx.x >> 5);
     if (b >= P.B) return;  // warp-uniform
+    // The state and the request's chunk masses are loaded together (the
+    // masses' address does not depend on the state).
+    const double2* cm = P.chunk_mass + b * P.cpr;
+    constexpr int kCM = 4;  // chunk masses per lane in the first round
+    double2 cmv[kCM];
+#pragma unroll
+    for (int j = 0; j < kCM; ++j) {
+        const int c = lane + 32 * j;
+        cmv[j] = c < P.cpr ? __ldcg(&cm[c]) : make_double2(0.0, 0.0);
+    }
     const RejState st = P.state[b];
     if (!st.valid) {  // the statistics pass already wrote -1 everywhere
         if (P.shard_totals != nullptr && lane == 0) P.shard_token[b] = -1;
@@ -373,9 +383,13 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
     const int64_t out_at = st.row;  // the drawn token's slot is row h's
 
     // Totals of r and p over the chunk masses, then u_res * S.
-    const double2* cm = P.chunk_mass + b * P.cpr;
     double tr = 0.0, tp = 0.0;
-    for (int c = lane; c < P.cpr; c += 32) {
+#pragma unroll
+    for (int j = 0; j < kCM; ++j) {
+        tr += cmv[j].x;
+        tp += cmv[j].y;
+    }
+    for (int c = lane + 32 * kCM; c < P.cpr; c += 32) {
         const double2 x = __ldcg(&cm[c]);
         tr += x.x;
         tp += x.y;
