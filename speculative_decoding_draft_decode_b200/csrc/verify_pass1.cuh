@@ -172,9 +172,8 @@ struct TreeArrays {
     int am[kTreeNodes];
     int par[kTreeNodes];
     int tok[kTreeNodes];
-    int anc[kTreeNodes];
-    int dep[kTreeNodes];
-    int ok[kTreeNodes];
+    int anc[2][kTreeNodes];  // pointer jumping, double-buffered: the ancestor reached
+    int st[2][kTreeNodes];   // and (edges summed << 1) | (all those edges match)
 };
 struct Pass1SmemTree : Pass1Smem {
     TreeArrays t;
@@ -616,6 +615,14 @@ __device__ uint64_t row_top8_key(const Pass1Params& P, int64_t r) {
 // The top-8 epilogue's shared memory: per warp a survivor list, per row the
 // merged 8 best, and the request's drafts and argmaxes.
 constexpr int kSurv = 128;
+// Keys per lane per batch in the top-8 epilogue's row merge, and whether the
+// 8 best survivors are placed by rank (1) or by eight warp-max rounds (0).
+#ifndef SPECDEC_TOP8_EPI_KB
+#define SPECDEC_TOP8_EPI_KB 8
+#endif
+#ifndef SPECDEC_TOP8_EPI_RANK
+#define SPECDEC_TOP8_EPI_RANK 1
+#endif
 constexpr int kTop8EpiWarps = 16;
 struct Top8EpiSmem {
     uint64_t surv[kTop8EpiWarps][kSurv];
@@ -633,7 +640,7 @@ struct Top8EpiSmem {
 // which rescans the row exactly when its partials hold fewer than 8 keys.
 template <class Tag>
 __device__ void row_top8_warp(const Pass1Params& P, int64_t r, uint64_t* surv, uint64_t* top) {
-    constexpr int KB = 16;  // keys per lane per batch
+    constexpr int KB = SPECDEC_TOP8_EPI_KB;  // keys per lane per batch
     const int lane = threadIdx.x & 31;
     const unsigned lt_mask = (1u << lane) - 1u;
     const int nk = P.cpr * NWARPS * 8;
@@ -659,8 +666,17 @@ __device__ void row_top8_warp(const Pass1Params& P, int64_t r, uint64_t* surv, u
         }
     }
     __syncwarp();
-    uint64_t mine;
     if (cnt >= 8 && cnt <= kSurv) {
+#if SPECDEC_TOP8_EPI_RANK
+        // The keys are distinct, so each survivor's rank (the survivors above
+        // it) places it directly: the 8 of rank < 8 are the row's 8 best.
+        for (int i = lane; i < cnt; i += 32) {
+            const uint64_t kx = surv[i];
+            int rank = 0;
+            for (int j = 0; j < cnt; ++j) rank += surv[j] > kx ? 1 : 0;
+            if (rank < 8) top[rank] = kx;
+        }
+#else
         uint64_t l[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) l[e] = 0ull;
@@ -668,11 +684,13 @@ __device__ void row_top8_warp(const Pass1Params& P, int64_t r, uint64_t* surv, u
             const uint64_t kx = surv[i];
             if (kx > l[7]) top8_insert(l, kx);
         }
-        mine = warp_top8(l);
+        const uint64_t mine = warp_top8(l);
+        if (lane < 8) top[lane] = mine;
+#endif
     } else {
-        mine = row_top8_key<Tag>(P, r);
+        const uint64_t mine = row_top8_key<Tag>(P, r);
+        if (lane < 8) top[lane] = mine;
     }
-    if (lane < 8) top[lane] = mine;
     __syncwarp();
 }
 
@@ -804,49 +822,41 @@ __device__ void epilogue_tree(const Pass1Params& P, int64_t b, Pass1SmemTree& sm
     bad = __syncthreads_or(bad);
     int32_t* nodes_out = P.accept_nodes + b * md;
     int32_t* out = P.out_tokens + b * (md + 1);
+    int cur = 0;  // the buffer holding the latest round
     if (!bad) {
         for (int c = threadIdx.x; c < n1; c += NT) {
-            const int p = ts.par[c];
-            ts.anc[c] = p;
-            ts.dep[c] = c == 0 ? 0 : 1;
+            ts.anc[0][c] = ts.par[c];
             const int t = ts.tok[c];
-            ts.ok[c] = c == 0 ? 1 : (t >= 0 && t < P.V && t == ts.am[p]);
+            const int ok = c == 0 ? 1 : (t >= 0 && t < P.V && t == ts.am[ts.par[c]]);
+            ts.st[0][c] = ((c == 0 ? 0 : 1) << 1) | ok;
         }
         __syncthreads();
         // Pointer jumping: after each round every node has summed the depth and
         // AND-ed the match flags of twice as many ancestors.  After the rounds
         // with span <= max_depth, a node has covered min(depth, 2 * last span)
         // > max_depth edges, so every node within max_depth of the root is
-        // complete and every deeper node shows a depth above max_depth.
+        // complete and every deeper node shows a depth above max_depth.  Each
+        // round reads one buffer and writes the other: one barrier per round.
         for (int span = 1; span <= md && span < n1; span <<= 1) {
-            int na[PER], nd[PER], no[PER];
-#pragma unroll
-            for (int q = 0; q < PER; ++q) {
-                const int c = threadIdx.x + q * NT;
-                if (c < n1) {
-                    const int a = ts.anc[c];
-                    if (a >= 0) {
-                        na[q] = ts.anc[a];
-                        nd[q] = ts.dep[c] + ts.dep[a];
-                        no[q] = ts.ok[c] & ts.ok[a];
-                    } else {
-                        na[q] = a;
-                        nd[q] = ts.dep[c];
-                        no[q] = ts.ok[c];
-                    }
+            const int nxt = cur ^ 1;
+            for (int c = threadIdx.x; c < n1; c += NT) {
+                const int a = ts.anc[cur][c];
+                const int sc = ts.st[cur][c];
+                if (a >= 0) {
+                    const int sa = ts.st[cur][a];
+                    ts.anc[nxt][c] = ts.anc[cur][a];
+                    ts.st[nxt][c] = (((sc >> 1) + (sa >> 1)) << 1) | (sc & sa & 1);
+                } else {
+                    ts.anc[nxt][c] = a;
+                    ts.st[nxt][c] = sc;
                 }
             }
             __syncthreads();
-#pragma unroll
-            for (int q = 0; q < PER; ++q) {
-                const int c = threadIdx.x + q * NT;
-                if (c < n1) { ts.anc[c] = na[q]; ts.dep[c] = nd[q]; ts.ok[c] = no[q]; }
-            }
-            __syncthreads();
+            cur = nxt;
         }
         int deep = 0;
         for (int c = threadIdx.x; c < n1; c += NT)
-            if (ts.dep[c] > md) deep = 1;
+            if ((ts.st[cur][c] >> 1) > md) deep = 1;
         bad = __syncthreads_or(deep);
     }
     if (bad) {
@@ -856,15 +866,17 @@ __device__ void epilogue_tree(const Pass1Params& P, int64_t b, Pass1SmemTree& sm
         return;
     }
     uint64_t key = 0ull;
-    for (int c = threadIdx.x; c < n1; c += NT)
-        if (ts.ok[c]) {
+    for (int c = threadIdx.x; c < n1; c += NT) {
+        const int sc = ts.st[cur][c];
+        if (sc & 1) {
             const uint64_t kk =
-                (static_cast<uint64_t>(ts.dep[c]) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(c));
+                (static_cast<uint64_t>(sc >> 1) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(c));
             key = kk > key ? kk : key;
         }
+    }
     key = block_max_u64(key, sm.red);
     const int best = key_index(key);
-    const int d = ts.dep[best];
+    const int d = ts.st[cur][best] >> 1;
     for (int i = d + threadIdx.x; i < md; i += NT) nodes_out[i] = -1;
     for (int i = d + 1 + threadIdx.x; i <= md; i += NT) out[i] = -1;
     if (threadIdx.x == 0) {
@@ -1159,8 +1171,12 @@ __global__ void __launch_bounds__(32 * kTop8EpiWarps) verify_top8_epilogue_kerne
                 float val = __uint_as_float(0x7fc00000u);
                 if (key != 0ull) {
                     id = key_index(key);
-                    val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride +
-                                           id);
+                    // The key holds the value exactly unless it is zero (-0
+                    // and +0 share a key) or NaN: only those are read back.
+                    val = key_value(key);
+                    if (!(val != 0.0f && val == val))
+                        val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) +
+                                               r * P.row_stride + id);
                 }
                 P.topk_ids[r * P.topk + e] = id;
                 P.topk_vals[r * P.topk + e] = val;
@@ -1271,9 +1287,12 @@ __global__ void __launch_bounds__(NT) verify_shard_rows_kernel(const Pass1Params
         if (lane < 8) {
             const uint64_t key = sm.top[wp][lane];
             float val = __uint_as_float(0x7fc00000u);
-            if (key != 0ull)
-                val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride +
-                                       key_index(key));
+            if (key != 0ull) {
+                val = key_value(key);  // exact unless zero (-0 and +0 share a key) or NaN
+                if (!(val != 0.0f && val == val))
+                    val = load_scalar<Tag>(static_cast<const typename Tag::storage*>(P.logits) + r * P.row_stride +
+                                           key_index(key));
+            }
             P.shard_keys[r * 8 + lane] = globalize(key, P.vocab_offset);
             P.shard_vals[r * 8 + lane] = val;
         }
