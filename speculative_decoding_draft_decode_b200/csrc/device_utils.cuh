@@ -171,6 +171,16 @@ __device__ __forceinline__ void block_top8(uint64_t (&l)[8], uint64_t* stage, ui
     __syncthreads();
 }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32), one
+// instruction where exp2f takes several: the streaming passes take one per
+// element.  Results below 2^-126 flush to zero; next to the row's largest
+// term (2^0) they are below fp32 resolution of any sum that holds it.
+__device__ __forceinline__ float ex2_sfu(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Softmax statistics (running max M of the raw logits, S = sum exp((l - M)/T))
 // merged in fp64.  A side with S == 0 contributes nothing.
 struct MaxSum {

@@ -493,7 +493,7 @@ struct SoftmaxReducer {
         if (!ok) return 0.0;
         float s = 0.0f;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) s += exp2f((VecOps<Tag, VEC>::elem(w, e) - M) * log2e_invT);
+        for (int e = 0; e < VEC; ++e) s += ex2_sfu((VecOps<Tag, VEC>::elem(w, e) - M) * log2e_invT);
         return static_cast<double>(s);
     }
     // Warp-collective: store (M, S) of the warp's part of the chunk.
@@ -1043,7 +1043,7 @@ __device__ __forceinline__ void softmax_chunk(const Pass1Params& P, const typena
             S += red.vec_sum(x, true, M);
         }
     }
-    if (has_tail) S += static_cast<double>(exp2f((tail - M) * P.log2e_invT));
+    if (has_tail) S += static_cast<double>(ex2_sfu((tail - M) * P.log2e_invT));
     if (P.prefetch_inputs) grid_dependency_wait();  // the pass began without waiting
     red.store(M, S, static_cast<uint64_t>(r) * P.cpr + sub, P);
 }

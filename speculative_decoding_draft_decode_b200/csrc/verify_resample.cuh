@@ -110,7 +110,7 @@ struct ResidualVec {
         RowLoader<Tag, VEC>::unpack(l, lv);
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
-            p[e] = exp2f((lv[e] - M) * l2) * invZ;
+            p[e] = ex2_sfu((lv[e] - M) * l2) * invZ;
             r[e] = has_q ? fmaxf(0.0f, p[e] - qv(e)) : p[e];
         }
     }
@@ -121,7 +121,7 @@ template <class Tag>
 __device__ __forceinline__ void residual_scalar(const typename Tag::storage* row, const float* qrow, int x,
                                                 bool has_q, float M, float l2, float invZ, float& p, float& r) {
     const float l = load_scalar<Tag>(row + x);
-    p = exp2f((l - M) * l2) * invZ;
+    p = ex2_sfu((l - M) * l2) * invZ;
     r = has_q ? fmaxf(0.0f, p - __ldg(qrow + x)) : p;
 }
 
