@@ -125,6 +125,17 @@ __device__ __forceinline__ void residual_scalar(const typename Tag::storage* row
     r = has_q ? fmaxf(0.0f, p - __ldg(qrow + x)) : p;
 }
 
+// Sum of one vector's values, in fp32 and in index order; fp64 from there
+// on.  The chunk and unit masses and the token search's lane totals all take
+// it, so the search's levels add the same numbers.
+template <int VEC>
+__device__ __forceinline__ float vec_total(const float (&x)[VEC]) {
+    float s = x[0];
+#pragma unroll
+    for (int e = 1; e < VEC; ++e) s += x[e];
+    return s;
+}
+
 struct Pass2Row {
     const void* row;
     const float* qrow;
@@ -211,11 +222,8 @@ __global__ void __launch_bounds__(NT) verify_resample_kernel(const Pass2Params P
             if (stream_pos(u0 + u, t) < cnt) {
                 float p[VEC], r[VEC];
                 v[u].values(R.has_q, st.M, P.log2e_invT, R.invZ, p, r);
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    ar += static_cast<double>(r[e]);
-                    ap += static_cast<double>(p[e]);
-                }
+                ar = static_cast<double>(vec_total<VEC>(r));
+                ap = static_cast<double>(vec_total<VEC>(p));
             }
             m[u] = ar;
             m[kU2 + u] = ap;
@@ -488,9 +496,8 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
             }
         }
         double ls = 0.0;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e)
-            if (e < nx) ls += static_cast<double>(m[e]);
+        if (nx == VEC) ls = static_cast<double>(vec_total<VEC>(m));
+        else if (nx == 1) ls = static_cast<double>(m[0]);
         double incl = ls;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
