@@ -356,6 +356,30 @@ def test_tree_depth_bound_small(V_, md):
                                           dtype="bf16"))
 
 
+@pytest.mark.parametrize("n1", [96, 127, 128, 129, 160])
+def test_tree_mid_size_deep_and_invalid(V_, n1):
+    """Trees of 96 to 160 nodes against the oracle: an invalid parent,
+    duplicate-token siblings, a chain past the depth bound, and a broom whose
+    31-edge handle sits exactly at (and one over) the bound."""
+    rng = np.random.default_rng(n1)
+    par = np.array([-1] + [int(rng.integers((c - 1) // 4, (c - 1) // 2 + 1)) for c in range(1, n1)], np.int32)
+    t = gen.tree_synthetic(seed=n1, B=6, parents=par, V=777, p_agree=0.9, max_depth=32, dtype="bf16")
+    t.parents[1, n1 - 1] = n1 - 1          # a node that is its own parent: invalid
+    t.node_tokens[2, 1:] = t.node_tokens[2, 1]
+    t.parents[3] = np.array([-1] + list(range(n1 - 1)), np.int32)  # a chain deeper than 32: invalid
+    got = check_tree(V_, t)
+    assert got[0][1] == -1 and got[0][3] == -1 and got[0].max() >= 1
+    t.max_depth = 5
+    check_tree(V_, t)
+    broom = np.array([-1] + [c - 1 if c <= 31 else 0 for c in range(1, n1)], np.int32)
+    tb = gen.tree_synthetic(seed=n1 + 1, B=4, parents=broom, V=500, p_agree=0.97, max_depth=31, dtype="f32")
+    got = check_tree(V_, tb)
+    assert (got[0] >= 0).all() and got[0].max() >= 8
+    tb.max_depth = 30
+    got = check_tree(V_, tb)
+    assert (got[0] == -1).all()
+
+
 def test_tree_single_node(V_):
     t = gen.tree_synthetic(seed=2, B=4, parents=np.array([-1], np.int32), V=100, dtype="f32", max_depth=1)
     got = check_tree(V_, t)
