@@ -171,6 +171,14 @@ __device__ __forceinline__ void block_top8(uint64_t (&l)[8], uint64_t* stage, ui
     __syncthreads();
 }
 
+// log2 x on the special-function unit (PTX lg2.approx.f32, subnormal inputs
+// included): one instruction.
+__device__ __forceinline__ float lg2_sfu(float x) {
+    float y;
+    asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32), one
 // instruction where exp2f takes several: the streaming passes take one per
 // element.  Results below 2^-126 flush to zero; next to the row's largest

@@ -353,7 +353,7 @@ specdec_status rejection_impl(const void* target_logits, specdec_dtype dtype, in
     S.cpr = static_cast<int>(L.cpr2);
     S.B = B;
     S.k = k;
-    S.invT = static_cast<float>(invT_d);
+    S.log2e_invT = P.log2e_invT;
     S.state = state;
     S.row_stat = P.row_stat;
     S.chunk_stats = reinterpret_cast<double2*>(static_cast<char*>(ws) + L.chunk_stats);

@@ -16,9 +16,11 @@
 // Two kernels after the request epilogue of the softmax pass:
 //   verify_stats_kernel           one CTA per (row (b, i < k), chunk): the
 //                                 chunk's sums of the entropy and JS terms
-//                                 (one exp and two logs per element in fp32,
-//                                 fp32 sums within a 16-byte vector, fp64
-//                                 across vectors);
+//                                 (per element in fp32 on the special-function
+//                                 unit: exp2, log2 q, and log2 m only where
+//                                 p and q differ by more than 3x, a series
+//                                 elsewhere; fp32 sums within a 16-byte
+//                                 vector, fp64 across vectors);
 //   verify_stats_epilogue_kernel  one warp per (b, i): the chunk sums in
 //                                 index order, then the outputs.
 #pragma once
@@ -44,7 +46,7 @@ struct StatsParams {
     int cpr;  // chunks per row (resample geometry)
     int B;
     int k;
-    float invT;
+    float log2e_invT;         // log2(e) / T
     const RejState* state;    // [B] validity
     const RowStat* row_stat;  // [B * (k + 1)]
     double2* chunk_stats;     // [B * k, cpr] (entropy sum, D_JS sum before the 1/2)
@@ -52,18 +54,53 @@ struct StatsParams {
     double* js;               // [B, k]
 };
 
-// The entropy and Jensen-Shannon terms of one element, from log p (known
-// from the row statistics: (l - M) / T - ln Z, so p needs one exp and no
-// log) and q: h -= q log q, d += p (log p - log m) + q (log q - log m).
-__device__ __forceinline__ void stat_terms(float lp, float q, float& h, float& d) {
-    const float p = expf(lp);
-    const float lm = logf(0.5f * (p + q));
+// f(delta) = (1 + delta) ln(1 + delta) + (1 - delta) ln(1 - delta), the
+// Jensen-Shannon term of an element over its m = (p + q) / 2 with
+// delta = (p - q) / (p + q), from its Taylor series sum_n delta^(2n) /
+// (n (2n - 1)) for |delta| <= 1/2: nine terms, the rest below 2e-8 of the
+// sum.  No logarithm of two nearly equal numbers is taken.
+__device__ __forceinline__ float js_series(float delta) {
+    const float z = delta * delta;
+    float s = 1.0f / 153.0f;        // n = 9
+    s = fmaf(s, z, 1.0f / 120.0f);  // n = 8
+    s = fmaf(s, z, 1.0f / 91.0f);
+    s = fmaf(s, z, 1.0f / 66.0f);
+    s = fmaf(s, z, 1.0f / 45.0f);
+    s = fmaf(s, z, 1.0f / 28.0f);
+    s = fmaf(s, z, 1.0f / 15.0f);
+    s = fmaf(s, z, 1.0f / 6.0f);
+    s = fmaf(s, z, 1.0f);           // n = 1
+    return s * z;
+}
+
+// The entropy and Jensen-Shannon terms of one element (nats), from
+// lp2 = log2 p (known from the row statistics: (l - M) log2(e) / T -
+// log2 Z) and q: h -= q ln q; d += m f(delta), which is p ln(p / m) +
+// q ln(q / m).  Where |delta| > 1/2 that log form is well conditioned
+// (|ln(p / m)|, |ln(q / m)| >= ln(4/3)) and is used with the
+// special-function unit's log2; elsewhere the series.  Elements with
+// p + q below the smallest normal float add nothing.
+__device__ __forceinline__ void stat_terms_log2(float lp2, float q, float& h, float& d) {
+    constexpr float kLn2 = 0.693147180559945309f;
+    const float p = ex2_sfu(lp2);
+    float lq2 = 0.0f;
     if (q > 0.0f) {
-        const float lq = logf(q);
-        h -= q * lq;
-        d += q * (lq - lm);
+        lq2 = lg2_sfu(q);
+        h -= kLn2 * (q * lq2);
     }
-    if (p > 0.0f) d += p * (lp - lm);
+    const float sum = p + q;
+    if (sum >= FLT_MIN) {
+        const float delta = __fdividef(p - q, sum);
+        if (fabsf(delta) <= 0.5f) {
+            d += 0.5f * sum * js_series(delta);
+        } else {
+            const float lm2 = lg2_sfu(0.5f * sum);
+            float t = 0.0f;
+            if (p > 0.0f) t += p * (lp2 - lm2);
+            if (q > 0.0f) t += q * (lq2 - lm2);
+            d += kLn2 * t;
+        }
+    }
 }
 
 template <class Tag, int VEC>
@@ -84,7 +121,7 @@ __global__ void __launch_bounds__(NT) verify_stats_kernel(const StatsParams P) {
     const int sub = static_cast<int>(blockIdx.y);
     if (!P.state[b].valid) return;  // CTA-uniform
     const RowStat rs = P.row_stat[b * (P.k + 1) + i];
-    const float lnZ = static_cast<float>(log(rs.Z));
+    const float l2Z = static_cast<float>(log2(rs.Z));
     const Elem* row = static_cast<const Elem*>(P.logits) + (b * (P.k + 1) + i) * P.row_stride;
     const float* qrow = P.q + x * P.q_stride;
     const int cnt = chunk_count(P.nv_full, sub, VEC, kU2);
@@ -104,7 +141,9 @@ __global__ void __launch_bounds__(NT) verify_stats_kernel(const StatsParams P) {
                 RowLoader<Tag, VEC>::unpack(v[u].l, lv);
                 float hv = 0.0f, dv = 0.0f;  // one vector in fp32, then fp64
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) stat_terms((lv[e] - rs.M) * P.invT - lnZ, v[u].qv(e), hv, dv);
+                for (int e = 0; e < VEC; ++e) {
+                    stat_terms_log2((lv[e] - rs.M) * P.log2e_invT - l2Z, v[u].qv(e), hv, dv);
+                }
                 h += static_cast<double>(hv);
                 d += static_cast<double>(dv);
             }
@@ -114,7 +153,7 @@ __global__ void __launch_bounds__(NT) verify_stats_kernel(const StatsParams P) {
         const int xe = P.nv_full * VEC + lane;
         if (xe < P.V) {
             float hv = 0.0f, dv = 0.0f;
-            stat_terms((load_scalar<Tag>(row + xe) - rs.M) * P.invT - lnZ, __ldg(qrow + xe), hv, dv);
+            stat_terms_log2((load_scalar<Tag>(row + xe) - rs.M) * P.log2e_invT - l2Z, __ldg(qrow + xe), hv, dv);
             h += static_cast<double>(hv);
             d += static_cast<double>(dv);
         }
