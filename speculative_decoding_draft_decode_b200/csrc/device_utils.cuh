@@ -171,11 +171,19 @@ __device__ __forceinline__ void block_top8(uint64_t (&l)[8], uint64_t* stage, ui
     __syncthreads();
 }
 
-// log2 x on the special-function unit (PTX lg2.approx.f32, subnormal inputs
-// included): one instruction.
+// log2 x on the special-function unit (PTX lg2.approx.ftz.f32): one
+// instruction; a subnormal x counts as zero (result -inf), so callers keep
+// x >= FLT_MIN.
 __device__ __forceinline__ float lg2_sfu(float x) {
     float y;
-    asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 1/x on the special-function unit (PTX rcp.approx.ftz.f32).
+__device__ __forceinline__ float rcp_sfu(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 

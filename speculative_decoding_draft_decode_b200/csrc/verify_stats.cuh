@@ -16,11 +16,13 @@
 // Two kernels after the request epilogue of the softmax pass:
 //   verify_stats_kernel           one CTA per (row (b, i < k), chunk): the
 //                                 chunk's sums of the entropy and JS terms
-//                                 (per element in fp32 on the special-function
-//                                 unit: exp2, log2 q, and log2 m only where
-//                                 p and q differ by more than 3x, a series
-//                                 elsewhere; fp32 sums within a 16-byte
-//                                 vector, fp64 across vectors);
+//                                 (per element in fp32: exp2, log2 q, log2 m
+//                                 and 1/(p + q) on the special-function unit;
+//                                 the log form where p and q differ by more
+//                                 than a factor 3, a series elsewhere, both
+//                                 evaluated without branches; fp32 sums
+//                                 within a 16-byte vector, fp64 across
+//                                 vectors);
 //   verify_stats_epilogue_kernel  one warp per (b, i): the chunk sums in
 //                                 index order, then the outputs.
 #pragma once
@@ -78,29 +80,26 @@ __device__ __forceinline__ float js_series(float delta) {
 // log2 Z) and q: h -= q ln q; d += m f(delta), which is p ln(p / m) +
 // q ln(q / m).  Where |delta| > 1/2 that log form is well conditioned
 // (|ln(p / m)|, |ln(q / m)| >= ln(4/3)) and is used with the
-// special-function unit's log2; elsewhere the series.  Elements with
-// p + q below the smallest normal float add nothing.
+// special-function unit's log2; elsewhere the series.  Both forms are
+// evaluated and one is selected, so the warp never diverges.  Elements with
+// q below the smallest normal float add no entropy, and elements with
+// p + q below 2^-125 add nothing; a NaN q makes d NaN.
 __device__ __forceinline__ void stat_terms_log2(float lp2, float q, float& h, float& d) {
     constexpr float kLn2 = 0.693147180559945309f;
+    constexpr float kTiny = 2.3509887e-38f;  // 2^-125: (p + q) / 2 stays normal
     const float p = ex2_sfu(lp2);
-    float lq2 = 0.0f;
-    if (q > 0.0f) {
-        lq2 = lg2_sfu(q);
-        h -= kLn2 * (q * lq2);
-    }
+    const bool qn = q >= FLT_MIN;
+    const float lq2 = lg2_sfu(qn ? q : 1.0f);  // 0 where q is below FLT_MIN
+    h -= qn ? kLn2 * (q * lq2) : 0.0f;
     const float sum = p + q;
-    if (sum >= FLT_MIN) {
-        const float delta = __fdividef(p - q, sum);
-        if (fabsf(delta) <= 0.5f) {
-            d += 0.5f * sum * js_series(delta);
-        } else {
-            const float lm2 = lg2_sfu(0.5f * sum);
-            float t = 0.0f;
-            if (p > 0.0f) t += p * (lp2 - lm2);
-            if (q > 0.0f) t += q * (lq2 - lm2);
-            d += kLn2 * t;
-        }
-    }
+    const float m = 0.5f * sum;
+    const float delta = (p - q) * rcp_sfu(sum);
+    const float lm2 = lg2_sfu(m);
+    const float tp = p > 0.0f ? p * (lp2 - lm2) : 0.0f;
+    const float tl = kLn2 * (tp + q * (lq2 - lm2));
+    const float ts = m * js_series(delta);
+    const float t = fabsf(delta) <= 0.5f ? ts : tl;
+    d += sum < kTiny ? 0.0f : t;
 }
 
 template <class Tag, int VEC>
