@@ -61,3 +61,26 @@ def test_adasd_stats_small(V_, V, dtype, T):
     drafts = np.argmax(q, axis=-1).astype(np.int32)
     target = gen.f32_to_bf16_bits(tgt) if dtype == "bf16" else tgt
     _check(V_, gen.RejectionInputs("adasd", dtype, target, q, drafts, B, k, V, temperature=T, seed=5, offset=2))
+
+
+def test_adasd_stats_series_boundary(V_):
+    """q built from the target's own softmax times fixed ratios: 3 and 1/3
+    (|delta| = 1/2, where the kernel switches between its series and its log
+    form), 1 +- 1e-3 (tiny delta), 1 (p = q, D_JS near 0), 0, and subnormal
+    values; against the oracle."""
+    rng = np.random.default_rng(11)
+    B, k, V = 8, 4, 3001
+    tgt = (rng.standard_normal((B, k + 1, V)) * 1.5).astype(np.float32)
+    z = tgt[:, :k].astype(np.float64)
+    p = np.exp(z - z.max(-1, keepdims=True))
+    p /= p.sum(-1, keepdims=True)
+    ratios = np.array([3.0, 1.0 / 3.0, 1.0 + 1e-3, 1.0 - 1e-3, 1.0, 0.0, 2.9999, 0.33334])
+    r = ratios[rng.integers(0, len(ratios), (B, k, V))]
+    r[0] = 1.0                               # p = q everywhere
+    r[1] = 3.0                               # every element exactly at the switch
+    q = (p * r).astype(np.float32)
+    q[2, 0, :40] = np.float32(1e-39)         # subnormal q
+    q[3, 1, :] = np.float32(1e-39)           # a whole row of subnormal q
+    drafts = np.argmax(q, axis=-1).astype(np.int32)
+    _check(V_, gen.RejectionInputs("adasd_boundary", "f32", tgt, q, drafts, B, k, V, temperature=1.0, seed=9,
+                                   offset=0))
