@@ -100,12 +100,12 @@ __device__ __forceinline__ int key_index(uint64_t key) {
 // Warp and CTA reductions
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        uint64_t w = __shfl_xor_sync(FULL_MASK, v, o);
-        v = w > v ? w : v;
-    }
-    return v;
+    // Two warp reductions of 32-bit words (one instruction each): the largest
+    // high word, then the largest low word among the lanes holding it.
+    const unsigned hi = static_cast<unsigned>(v >> 32);
+    const unsigned mh = __reduce_max_sync(FULL_MASK, hi);
+    const unsigned ml = __reduce_max_sync(FULL_MASK, hi == mh ? static_cast<unsigned>(v) : 0u);
+    return (static_cast<uint64_t>(mh) << 32) | ml;
 }
 
 // CTA-wide maximum; `red` is NWARPS words of shared memory.  Every thread
@@ -293,8 +293,7 @@ __device__ __forceinline__ double block_sum_f64(double v, double* red) {
 
 __device__ __forceinline__ int block_max_int(int v, int* red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(FULL_MASK, v, o));
+    v = __reduce_max_sync(FULL_MASK, v);
     if (lane == 0) red[warp] = v;
     __syncthreads();
     int r = red[0];
@@ -305,8 +304,7 @@ __device__ __forceinline__ int block_max_int(int v, int* red) {
 
 __device__ __forceinline__ int block_min_int(int v, int* red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(FULL_MASK, v, o));
+    v = __reduce_min_sync(FULL_MASK, v);
     if (lane == 0) red[warp] = v;
     __syncthreads();
     int r = red[0];

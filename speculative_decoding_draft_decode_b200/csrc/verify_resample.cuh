@@ -356,9 +356,7 @@ __device__ __forceinline__ int warp_find_level(const double2* m, int n, bool use
         return __shfl_sync(FULL_MASK, hit, src);
     }
     found = false;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(FULL_MASK, last, o));
-    return last;
+    return __reduce_max_sync(FULL_MASK, last);
 }
 
 template <class Tag, int VEC>
@@ -517,11 +515,8 @@ __global__ void __launch_bounds__(NT) verify_resample_epilogue_kernel(const Pass
                 run += v;
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            hit = min(hit, __shfl_xor_sync(FULL_MASK, hit, o));
-            last = max(last, __shfl_xor_sync(FULL_MASK, last, o));
-        }
+        hit = __reduce_min_sync(FULL_MASK, hit);
+        last = __reduce_max_sync(FULL_MASK, last);
         token = hit != INT_MAX ? hit : (last >= 0 ? last : P.V - 1);
     }
     if (lane == 0) {
