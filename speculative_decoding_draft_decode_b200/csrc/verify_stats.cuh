@@ -19,7 +19,7 @@
 //                                 (per element in fp32: exp2, log2 q, log2 m
 //                                 and 1/(p + q) on the special-function unit;
 //                                 the log form where p and q differ by more
-//                                 than a factor 3, a series elsewhere, both
+//                                 than a factor 5/3, a series elsewhere, both
 //                                 evaluated without branches; fp32 sums
 //                                 within a 16-byte vector, fp64 across
 //                                 vectors);
@@ -51,54 +51,52 @@ struct StatsParams {
     float log2e_invT;         // log2(e) / T
     const RejState* state;    // [B] validity
     const RowStat* row_stat;  // [B * (k + 1)]
-    double2* chunk_stats;     // [B * k, cpr] (entropy sum, D_JS sum before the 1/2)
+    double2* chunk_stats;     // [B * k, cpr] (entropy sum, D_JS sum before the 1/2), in bits
     double* entropy;          // [B, k]
     double* js;               // [B, k]
 };
 
-// f(delta) = (1 + delta) ln(1 + delta) + (1 - delta) ln(1 - delta), the
-// Jensen-Shannon term of an element over its m = (p + q) / 2 with
-// delta = (p - q) / (p + q), from its Taylor series sum_n delta^(2n) /
-// (n (2n - 1)) for |delta| <= 1/2: nine terms, the rest below 2e-8 of the
-// sum.  No logarithm of two nearly equal numbers is taken.
-__device__ __forceinline__ float js_series(float delta) {
+// f(delta) / ln 2, where f(delta) = (1 + delta) ln(1 + delta) + (1 - delta)
+// ln(1 - delta) is the Jensen-Shannon term of an element over its
+// m = (p + q) / 2, delta = (p - q) / (p + q): from the Taylor series
+// f = sum_n delta^(2n) / (n (2n - 1)), five terms for |delta| <= 1/4 (the
+// rest is below 1.5e-8 of the sum), each coefficient divided by ln 2 once.
+// No logarithm of two nearly equal numbers is taken.
+__device__ __forceinline__ float js_series_log2(float delta) {
+    constexpr float kInvLn2 = 1.44269504088896341f;
     const float z = delta * delta;
-    float s = 1.0f / 153.0f;        // n = 9
-    s = fmaf(s, z, 1.0f / 120.0f);  // n = 8
-    s = fmaf(s, z, 1.0f / 91.0f);
-    s = fmaf(s, z, 1.0f / 66.0f);
-    s = fmaf(s, z, 1.0f / 45.0f);
-    s = fmaf(s, z, 1.0f / 28.0f);
-    s = fmaf(s, z, 1.0f / 15.0f);
-    s = fmaf(s, z, 1.0f / 6.0f);
-    s = fmaf(s, z, 1.0f);           // n = 1
+    float s = kInvLn2 / 45.0f;           // n = 5
+    s = fmaf(s, z, kInvLn2 / 28.0f);     // n = 4
+    s = fmaf(s, z, kInvLn2 / 15.0f);     // n = 3
+    s = fmaf(s, z, kInvLn2 / 6.0f);      // n = 2
+    s = fmaf(s, z, kInvLn2);             // n = 1
     return s * z;
 }
 
-// The entropy and Jensen-Shannon terms of one element (nats), from
-// lp2 = log2 p (known from the row statistics: (l - M) log2(e) / T -
-// log2 Z) and q: h -= q ln q; d += m f(delta), which is p ln(p / m) +
-// q ln(q / m).  Where |delta| > 1/2 that log form is well conditioned
-// (|ln(p / m)|, |ln(q / m)| >= ln(4/3)) and is used with the
-// special-function unit's log2; elsewhere the series.  Both forms are
-// evaluated and one is selected, so the warp never diverges.  Elements with
-// q below the smallest normal float add no entropy, and elements with
-// p + q below 2^-125 add nothing; a NaN q makes d NaN.
+// The entropy and Jensen-Shannon terms of one element in bits (the
+// epilogue multiplies the sums by ln 2), from lp2 = log2 p (known from the
+// row statistics: (l - M) log2(e) / T - log2 Z) and q: h -= q log2 q;
+// d += m f(delta) / ln 2, which is p log2(p / m) + q log2(q / m).  Where
+// |delta| > 1/4 that log form is well conditioned (|log2(p / m)|,
+// |log2(q / m)| >= log2(5/4)) and is used with the special-function unit's
+// log2; elsewhere the series.  Both forms are evaluated and one is
+// selected, so the warp never diverges.  Elements with q below the smallest
+// normal float add no entropy, and elements with p + q below 2^-125 add
+// nothing; a NaN q makes d NaN.
 __device__ __forceinline__ void stat_terms_log2(float lp2, float q, float& h, float& d) {
-    constexpr float kLn2 = 0.693147180559945309f;
     constexpr float kTiny = 2.3509887e-38f;  // 2^-125: (p + q) / 2 stays normal
     const float p = ex2_sfu(lp2);
     const bool qn = q >= FLT_MIN;
     const float lq2 = lg2_sfu(qn ? q : 1.0f);  // 0 where q is below FLT_MIN
-    h -= qn ? kLn2 * (q * lq2) : 0.0f;
+    h -= qn ? q * lq2 : 0.0f;
     const float sum = p + q;
     const float m = 0.5f * sum;
     const float delta = (p - q) * rcp_sfu(sum);
     const float lm2 = lg2_sfu(m);
     const float tp = p > 0.0f ? p * (lp2 - lm2) : 0.0f;
-    const float tl = kLn2 * (tp + q * (lq2 - lm2));
-    const float ts = m * js_series(delta);
-    const float t = fabsf(delta) <= 0.5f ? ts : tl;
+    const float tl = fmaf(q, lq2 - lm2, tp);
+    const float ts = m * js_series_log2(delta);
+    const float t = fabsf(delta) <= 0.25f ? ts : tl;
     d += sum < kTiny ? 0.0f : t;
 }
 
@@ -201,9 +199,10 @@ __global__ void __launch_bounds__(NT) verify_stats_epilogue_kernel(const StatsPa
         h += __shfl_xor_sync(FULL_MASK, h, o);
         d += __shfl_xor_sync(FULL_MASK, d, o);
     }
-    if (lane == 0) {
-        P.entropy[x] = h;
-        P.js[x] = sqrt(fmax(0.0, 0.5 * d));
+    if (lane == 0) {  // the sums are in bits
+        constexpr double kLn2 = 0.693147180559945309417;
+        P.entropy[x] = kLn2 * h;
+        P.js[x] = sqrt(fmax(0.0, 0.5 * kLn2 * d));
     }
 }
 
