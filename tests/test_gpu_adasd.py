@@ -12,7 +12,7 @@ from gpu_util import dev_f32, dev_i32, dev_logits, host, require_cuda
 pytestmark = pytest.mark.gpu
 
 # fp32 per element (SFU exp2 and log2, a series where p and q are within a
-# factor 3) with fp64 sums: relative error ~1e-6 at most
+# factor 5/3) with fp64 sums: relative error ~1e-6 at most
 RTOL, ATOL = 2e-5, 1e-6
 
 
@@ -64,20 +64,21 @@ def test_adasd_stats_small(V_, V, dtype, T):
 
 
 def test_adasd_stats_series_boundary(V_):
-    """q built from the target's own softmax times fixed ratios: 3 and 1/3
-    (|delta| = 1/2, where the kernel switches between its series and its log
-    form), 1 +- 1e-3 (tiny delta), 1 (p = q, D_JS near 0), 0, and subnormal
-    values; against the oracle."""
+    """q built from the target's own softmax times fixed ratios: 5/3 and 3/5
+    (|delta| = 1/4, where the kernel switches between its series and its log
+    form) and values just beside them, 3 and 1/3 (the log form), 1 +- 1e-3
+    (tiny delta), 1 (p = q, D_JS near 0), 0, and subnormal values; against
+    the oracle."""
     rng = np.random.default_rng(11)
     B, k, V = 8, 4, 3001
     tgt = (rng.standard_normal((B, k + 1, V)) * 1.5).astype(np.float32)
     z = tgt[:, :k].astype(np.float64)
     p = np.exp(z - z.max(-1, keepdims=True))
     p /= p.sum(-1, keepdims=True)
-    ratios = np.array([3.0, 1.0 / 3.0, 1.0 + 1e-3, 1.0 - 1e-3, 1.0, 0.0, 2.9999, 0.33334])
+    ratios = np.array([5.0 / 3.0, 0.6, 1.6666, 0.60001, 3.0, 1.0 / 3.0, 1.0 + 1e-3, 1.0 - 1e-3, 1.0, 0.0])
     r = ratios[rng.integers(0, len(ratios), (B, k, V))]
     r[0] = 1.0                               # p = q everywhere
-    r[1] = 3.0                               # every element exactly at the switch
+    r[1] = 5.0 / 3.0                         # every element at the switch
     q = (p * r).astype(np.float32)
     q[2, 0, :40] = np.float32(1e-39)         # subnormal q
     q[3, 1, :] = np.float32(1e-39)           # a whole row of subnormal q
