@@ -201,6 +201,10 @@ specdec_status specdec_verify_tree(const void* logits, specdec_dtype dtype, int6
  *                 D_JS = (KL(p || m) + KL(q || m)) / 2, m = (p + q) / 2, in
  *                 nats; p_i = softmax(l_i / T)
  * (0 log 0 = 0; NaN for a request whose target distributions are undefined).
+ * Per element the terms are computed in fp32 and summed in fp64: within
+ * 2e-5 relative (or 1e-6 absolute) of the fp64 definition; q values below
+ * the smallest normal float (1.2e-38) add no entropy, and elements whose
+ * p + q is below 2^-125 add nothing to D_JS.
  * The verification itself is unchanged: the page gives no rule for turning
  * the statistics into thresholds.  Two more kernels are enqueued, which read
  * target rows 0..k-1 and the q rows once more. */
